@@ -1,0 +1,227 @@
+"""CPU oracle for the ConvRot256 INT8 linear path (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's ``cpu_baseline`` / ``--impl reference`` legs are the only callers.
+The CUDA product path never imports this package, and this package imports
+nothing from the product.
+
+The arithmetic lives in ``convrot_oracle.c`` (plain C, IEEE fp32, no
+contraction); this module compiles it with gcc on first use and wraps it with
+numpy arrays. BF16 values travel as numpy ``uint16`` bit patterns.
+
+What each function follows (page title, section):
+  - ``rot256``: ConvRot256 as named in the sglang PR "Tune Kitchen INT8 row
+    splitting for SM120" (Accuracy Test) and called a Hadamard rotation in the
+    ComfyUI-AppleSilicon-FP8 README ("What it fixes", row 17); read as the
+    normalised Sylvester Walsh-Hadamard transform, stages h = 1..128, then /16.
+  - ``quantize_rows``: comfy-kitchen 0.2.40, "Huawei Ascend backend"
+    (quantize_int8_rowwise, quantize_and_rotate_rowwise); s = absmax/127,
+    q = round-half-even(y/s) clamped to [-127, 127].
+  - ``gemm_i32`` / ``epilogue`` / ``int8_linear``: ComfyUI-AppleSilicon-FP8
+    README row 17 (INT8 x INT8 -> INT32, per-row rescale + bias in the store
+    epilogue) and comfy-kitchen "int8_linear".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "convrot_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+          "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle library with gcc (in-tree) and return its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _P(t):
+    return ctypes.POINTER(t)
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # A test may point this at a deliberately broken copy of the
+            # oracle to show that the pins catch the mistake.
+            override = os.environ.get("CONVROT_ORACLE_LIB")
+            L = ctypes.CDLL(override if override else build())
+            i64, f32p = ctypes.c_int64, _P(ctypes.c_float)
+            u16p, i8p, i32p = _P(ctypes.c_uint16), _P(ctypes.c_int8), _P(ctypes.c_int32)
+            L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+            L.oracle_bf16_to_f32.restype = ctypes.c_float
+            L.oracle_f32_to_bf16_rne.argtypes = [ctypes.c_float]
+            L.oracle_f32_to_bf16_rne.restype = ctypes.c_uint16
+            L.oracle_rot256.argtypes = [f32p]
+            L.oracle_rot256.restype = None
+            L.oracle_quant_row.argtypes = [f32p, i64, i8p, f32p]
+            L.oracle_quant_row.restype = None
+            L.oracle_quantize_rows_bf16.argtypes = [u16p, i64, i64, i64, ctypes.c_int, i8p, f32p]
+            L.oracle_quantize_rows_bf16.restype = ctypes.c_int
+            L.oracle_rotate_quant_weight.argtypes = [f32p, i64, i64, i8p, f32p]
+            L.oracle_rotate_quant_weight.restype = ctypes.c_int
+            L.oracle_gemm_i32.argtypes = [i8p, i8p, i64, i64, i64, i32p]
+            L.oracle_gemm_i32.restype = None
+            L.oracle_epilogue.argtypes = [i32p, f32p, f32p, u16p, i64, i64, u16p]
+            L.oracle_epilogue.restype = None
+            L.oracle_linear_rows.argtypes = [i8p, f32p, i8p, f32p, u16p, i64, i64,
+                                             _P(ctypes.c_int64), i64, u16p]
+            L.oracle_linear_rows.restype = None
+            L.oracle_num_threads.argtypes = []
+            L.oracle_num_threads.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray, ct):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(_P(ct))
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's row loops use (OMP_NUM_THREADS, else all cores)."""
+    return lib().oracle_num_threads()
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(x) -> np.ndarray:
+    """fp32 -> bf16 bits, round-to-nearest-even (the oracle's own C routine)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    L = lib()
+    out = np.empty(x.shape, np.uint16)
+    flat, fo = x.reshape(-1), out.reshape(-1)
+    for i in range(flat.size):
+        fo[i] = L.oracle_f32_to_bf16_rne(float(flat[i]))
+    return out
+
+
+def rot256(v) -> np.ndarray:
+    """ConvRot256 of one block (or of each row of a [R, 256] array), fp32."""
+    a = np.array(v, dtype=np.float32, copy=True)
+    flat = a.reshape(-1, 256)
+    L = lib()
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        L.oracle_rot256(_ptr(row, ctypes.c_float))
+        flat[r] = row
+    return flat.reshape(a.shape)
+
+
+def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row symmetric INT8 quantisation of fp32 rows [R, K] (no rotation)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    y2 = y.reshape(-1, y.shape[-1])
+    R, K = y2.shape
+    q = np.empty((R, K), np.int8)
+    s = np.empty(R, np.float32)
+    L = lib()
+    for r in range(R):
+        row = np.ascontiguousarray(y2[r])
+        qr = np.empty(K, np.int8)
+        sr = np.empty(1, np.float32)
+        L.oracle_quant_row(_ptr(row, ctypes.c_float), K, _ptr(qr, ctypes.c_int8),
+                           _ptr(sr, ctypes.c_float))
+        q[r], s[r] = qr, sr[0]
+    return q, s
+
+
+def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = None):
+    """quantize_and_rotate_rowwise (rotate=True) or quantize_int8_rowwise
+    (rotate=False) on BF16 rows. ``X_bits`` is uint16 [M, ldx]; the first K
+    columns of each row are used (K defaults to ldx)."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, ld = X_bits.shape
+    K = ld if K is None else K
+    Qx = np.empty((M, K), np.int8)
+    s_x = np.empty(M, np.float32)
+    rc = lib().oracle_quantize_rows_bf16(_ptr(X_bits, ctypes.c_uint16), M, K, ld, int(rotate),
+                                         _ptr(Qx, ctypes.c_int8), _ptr(s_x, ctypes.c_float))
+    if rc:
+        raise ValueError(f"oracle_quantize_rows_bf16 failed ({rc}): K={K} must be a multiple of 256")
+    return Qx, s_x
+
+
+def rotate_quant_weight(W) -> tuple[np.ndarray, np.ndarray]:
+    """Offline weight preparation: ConvRot256 along K, then per-output-row INT8."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Qw = np.empty((N, K), np.int8)
+    s_w = np.empty(N, np.float32)
+    rc = lib().oracle_rotate_quant_weight(_ptr(W, ctypes.c_float), N, K, _ptr(Qw, ctypes.c_int8),
+                                          _ptr(s_w, ctypes.c_float))
+    if rc:
+        raise ValueError(f"oracle_rotate_quant_weight failed ({rc})")
+    return Qw, s_w
+
+
+def gemm_i32(Qx: np.ndarray, Qw: np.ndarray) -> np.ndarray:
+    Qx = np.ascontiguousarray(Qx, dtype=np.int8)
+    Qw = np.ascontiguousarray(Qw, dtype=np.int8)
+    M, K = Qx.shape
+    N, K2 = Qw.shape
+    assert K == K2
+    acc = np.empty((M, N), np.int32)
+    lib().oracle_gemm_i32(_ptr(Qx, ctypes.c_int8), _ptr(Qw, ctypes.c_int8), M, N, K,
+                          _ptr(acc, ctypes.c_int32))
+    return acc
+
+
+def epilogue(acc, s_x, s_w, bias_bits=None) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    s_x = np.ascontiguousarray(s_x, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    M, N = acc.shape
+    Y = np.empty((M, N), np.uint16)
+    bp = None
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        bp = _ptr(bias_bits, ctypes.c_uint16)
+    lib().oracle_epilogue(_ptr(acc, ctypes.c_int32), _ptr(s_x, ctypes.c_float),
+                          _ptr(s_w, ctypes.c_float), bp, M, N, _ptr(Y, ctypes.c_uint16))
+    return Y
+
+
+def linear_rows(Qx, s_x, Qw, s_w, bias_bits, rows) -> np.ndarray:
+    """Output rows ``rows`` of the linear, each computed on its own."""
+    Qx = np.ascontiguousarray(Qx, dtype=np.int8)
+    Qw = np.ascontiguousarray(Qw, dtype=np.int8)
+    s_x = np.ascontiguousarray(s_x, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    N, K = Qw.shape
+    Y = np.empty((rows.size, N), np.uint16)
+    bp = None
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        bp = _ptr(bias_bits, ctypes.c_uint16)
+    lib().oracle_linear_rows(_ptr(Qx, ctypes.c_int8), _ptr(s_x, ctypes.c_float),
+                             _ptr(Qw, ctypes.c_int8), _ptr(s_w, ctypes.c_float), bp, N, K,
+                             _ptr(rows, ctypes.c_int64), rows.size, _ptr(Y, ctypes.c_uint16))
+    return Y
+
+
+def int8_linear(X_bits, Qw, s_w, bias_bits=None):
+    """The whole forward: quantize_and_rotate_rowwise on X, INT32 GEMM, epilogue.
+    Returns (Y bits [M,N], Qx, s_x, acc)."""
+    Qx, s_x = quantize_rows_bf16(X_bits, rotate=True)
+    acc = gemm_i32(Qx, Qw)
+    return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc

@@ -1,0 +1,226 @@
+/*
+ * CPU oracle for the ConvRot256 INT8 linear path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this library. The product path (the
+ * CUDA library) shares no code with it and never calls it.
+ *
+ * It is deliberately plain and slow: every step is written out in the order of
+ * the method's definition, in IEEE single precision with round-to-nearest-even
+ * and no operation fused or reordered (compile with -ffp-contract=off and
+ * without -ffast-math). Rows are spread over OpenMP threads; that changes no
+ * arithmetic, because every output element is computed by one thread alone.
+ *
+ * Sources for what is computed:
+ *  - comfy-kitchen 0.2.40 (PyPI page), "Huawei Ascend backend" and "HIP
+ *    backend": quantize_int8_rowwise (dynamic per-row INT8),
+ *    quantize_and_rotate_rowwise (rotation fused with the per-row quantiser),
+ *    int8_linear (activation quantisation then INT8 matmul).
+ *  - sglang PR "Tune Kitchen INT8 row splitting for SM120", "Accuracy Test":
+ *    BF16 activations and bias, INT8 weights, FP32 row scales, ConvRot256.
+ *  - ComfyUI-AppleSilicon-FP8 README, "What it fixes" table, row 17: rotate
+ *    the activation online, per-row quantise it, INT8 x INT8 -> INT32, then a
+ *    per-row rescale plus bias in the store epilogue; row 12: the INT32 sums
+ *    stay well inside the int32 range.
+ * The pages name ConvRot256 and call it a Hadamard rotation but print no
+ * formula. The reading taken here: the normalised 256-point Walsh-Hadamard
+ * transform (Sylvester order, no random signs), as 8 butterfly stages with
+ * h = 1, 2, 4, ..., 128 followed by an exact multiply by 1/16. Scale
+ * s = absmax / 127 (IEEE division), code = round-half-even(y / s) clamped to
+ * [-127, 127]; an all-zero row gets s = 0 and all-zero codes. Epilogue:
+ * y = bf16_rne(((float(acc) * s_x) * s_w) + float(bias)), each step rounded
+ * to fp32; a missing bias adds +0.0f.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ROT_N 256
+
+/* BF16 -> fp32 is exact: the bf16 bits are the upper half of the fp32 bits. */
+float oracle_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* fp32 -> BF16 by the definition of round-to-nearest-even on the upper 16
+ * bits: keep the upper half, and add one unit in its last place when the
+ * discarded lower half is above one half, or exactly one half with an odd
+ * kept part. Overflow carries into the exponent and gives infinity, as IEEE
+ * rounding does. NaN is never produced by this path's arithmetic. */
+uint16_t oracle_f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t kept = u >> 16;
+    uint32_t rest = u & 0xFFFFu;
+    if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))
+        kept += 1u;
+    return (uint16_t)kept;
+}
+
+/* ConvRot256 on one block of 256 values, in place. */
+void oracle_rot256(float *v) {
+    for (int h = 1; h < ROT_N; h <<= 1) {
+        for (int i = 0; i < ROT_N; ++i) {
+            if ((i & h) == 0) {
+                float a = v[i];
+                float c = v[i + h];
+                v[i] = a + c;
+                v[i + h] = a - c;
+            }
+        }
+    }
+    for (int i = 0; i < ROT_N; ++i)
+        v[i] = v[i] * 0.0625f;
+}
+
+/* Dynamic symmetric per-row INT8 quantisation of one row y[0..K). */
+void oracle_quant_row(const float *y, int64_t K, int8_t *q, float *s_out) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(y[k]);
+        if (a > amax)
+            amax = a;
+    }
+    float s = amax / 127.0f;
+    *s_out = s;
+    if (amax == 0.0f) {
+        memset(q, 0, (size_t)K);
+        return;
+    }
+    for (int64_t k = 0; k < K; ++k) {
+        float t = y[k] / s;
+        float r = nearbyintf(t); /* default rounding mode: ties to even */
+        if (r > 127.0f)
+            r = 127.0f;
+        if (r < -127.0f)
+            r = -127.0f;
+        q[k] = (int8_t)r;
+    }
+}
+
+/* quantize_and_rotate_rowwise on BF16 rows: widen, ConvRot256 every 256-block
+ * of the row, then quantise the whole rotated row. X has row stride ldx
+ * (elements). rotate == 0 skips the rotation (plain quantize_int8_rowwise). */
+int oracle_quantize_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                              int rotate, int8_t *Qx, float *s_x) {
+    if (K % ROT_N != 0 || ldx < K)
+        return 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        float *buf = (float *)malloc((size_t)K * sizeof(float));
+        if (!buf) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t m = 0; m < M; ++m) {
+                const uint16_t *row = X + m * ldx;
+                for (int64_t k = 0; k < K; ++k)
+                    buf[k] = oracle_bf16_to_f32(row[k]);
+                if (rotate)
+                    for (int64_t b = 0; b < K; b += ROT_N)
+                        oracle_rot256(buf + b);
+                oracle_quant_row(buf, K, Qx + m * K, s_x + m);
+            }
+            free(buf);
+        }
+    }
+    return err;
+}
+
+/* Offline weight preparation: fp32 W [N,K] (row stride K), rotated along K
+ * with the same ConvRot256, then quantised per output row. */
+int oracle_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw, float *s_w) {
+    if (K % ROT_N != 0)
+        return 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        float *buf = (float *)malloc((size_t)K * sizeof(float));
+        if (!buf) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t n = 0; n < N; ++n) {
+                memcpy(buf, W + n * K, (size_t)K * sizeof(float));
+                for (int64_t b = 0; b < K; b += ROT_N)
+                    oracle_rot256(buf + b);
+                oracle_quant_row(buf, K, Qw + n * K, s_w + n);
+            }
+            free(buf);
+        }
+    }
+    return err;
+}
+
+/* acc[m][n] = sum_k Qx[m][k] * Qw[n][k], exact in int32 while K * 127^2 < 2^31. */
+void oracle_gemm_i32(const int8_t *Qx, const int8_t *Qw, int64_t M, int64_t N, int64_t K,
+                     int32_t *acc) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const int8_t *a = Qx + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const int8_t *b = Qw + n * K;
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int32_t)a[k] * (int32_t)b[k];
+            acc[m * N + n] = s;
+        }
+    }
+}
+
+/* Y[m][n] = bf16_rne(((float(acc) * s_x[m]) * s_w[n]) + float(bias[n])). */
+static uint16_t epilogue_one(int32_t acc, float sx, float sw, float b) {
+    float f = (float)acc; /* int32 -> fp32, round to nearest even */
+    f = f * sx;
+    f = f * sw;
+    f = f + b;
+    return oracle_f32_to_bf16_rne(f);
+}
+
+void oracle_epilogue(const int32_t *acc, const float *s_x, const float *s_w, const uint16_t *bias,
+                     int64_t M, int64_t N, uint16_t *Y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float b = bias ? oracle_bf16_to_f32(bias[n]) : 0.0f;
+            Y[m * N + n] = epilogue_one(acc[m * N + n], s_x[m], s_w[n], b);
+        }
+}
+
+/* Rows of the linear computed one by one from already-quantised activations:
+ * Y_rows[i][n] for row index rows[i] of Qx. Used to check sampled rows of a
+ * full-size output without forming the whole INT32 product. */
+void oracle_linear_rows(const int8_t *Qx, const float *s_x, const int8_t *Qw, const float *s_w,
+                        const uint16_t *bias, int64_t N, int64_t K, const int64_t *rows,
+                        int64_t nrows, uint16_t *Y_rows) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int8_t *a = Qx + rows[i] * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const int8_t *b = Qw + n * K;
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int32_t)a[k] * (int32_t)b[k];
+            float bb = bias ? oracle_bf16_to_f32(bias[n]) : 0.0f;
+            Y_rows[i * N + n] = epilogue_one(s, s_x[rows[i]], s_w[n], bb);
+        }
+    }
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

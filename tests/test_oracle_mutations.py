@@ -1,0 +1,49 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU),
+builds it, and runs the pin suite against that copy: the suite must fail.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "stage_order_descending": ("for (int h = 1; h < ROT_N; h <<= 1) {",
+                               "for (int h = ROT_N / 2; h >= 1; h >>= 1) {"),
+    "butterfly_sign_swapped": ("v[i + h] = a - c;", "v[i + h] = c - a;"),
+    "no_normalisation": ("v[i] = v[i] * 0.0625f;", "v[i] = v[i] * 1.0f;"),
+    "reciprocal_instead_of_division": ("float t = y[k] / s;", "float t = y[k] * (1.0f / s);"),
+    "round_half_away": ("float r = nearbyintf(t);", "float r = roundf(t);"),
+    "truncate": ("float r = nearbyintf(t);", "float r = truncf(t);"),
+    "max_without_abs": ("float a = fabsf(y[k]);", "float a = y[k];"),
+    "scale_over_128": ("float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+    "gemm_transposed_weight": ("const int8_t *b = Qw + n * K;\n            int32_t s = 0;\n            for (int64_t k = 0; k < K; ++k)\n                s += (int32_t)a[k] * (int32_t)b[k];\n            acc[m * N + n] = s;",
+                               "int32_t s = 0;\n            for (int64_t k = 0; k < K; ++k)\n                s += (int32_t)a[k] * (int32_t)Qw[(k % N) * K + (n % K)];\n            acc[m * N + n] = s;"),
+    "epilogue_drops_weight_scale": ("    f = f * sw;\n", "    (void)sw;\n"),
+    "epilogue_bias_dropped": ("    f = f + b;\n", "    (void)b;\n"),
+    "bf16_truncates": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (0)"),
+    "bf16_ties_away": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (rest >= 0x8000u)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    old, new = MUTATIONS[name]
+    src = open(oracle._SRC).read()
+    assert old in src, f"mutation {name} no longer applies"
+    mut = tmp_path / "mut.c"
+    mut.write_text(src.replace(old, new, 1))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, str(mut), "-o", str(so), "-lm"],
+                          stderr=subprocess.DEVNULL)
+    env = dict(os.environ, CONVROT_ORACLE_LIB=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
