@@ -1,0 +1,402 @@
+"""Throughput of the ConvRot256 INT8 linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step is one forward of the whole path on one batch: the fused
+ConvRot256 rotate + per-row INT8 quantiser over X [M, K] (bf16), then the
+tcgen05 INT8 GEMM with the fused scale/bias/BF16 epilogue into Y [M, N].
+The weights are prepared once before timing (offline weight rotation and
+quantisation, as the method stores them). Default workload: the QKV-style
+projection M32700/K5376/N16128 (the shape the sglang PR "Tune Kitchen INT8
+row splitting for SM120" times in its Benchmark & Profiling table).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream (one pair per kernel), with a 256 MiB write between
+steps to flush the 126 MB L2; barrier + synchronize around the region; the
+max over ranks. Ranks (torchrun, one per GPU) each run their own batch of M
+rows against their own copy of the weights: rows are independent, so there
+is no collective on the data path ("replicas", weak scaling).
+
+Rank 0 prints ONE JSON line. `--impl reference` times the CPU oracle (plain
+C, OpenMP over rows) on a bounded sample of rows of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "INT8 linear TOPS (2MNK/s): ConvRot256 rotate+quantize + INT8 GEMM + epilogue"
+UNIT = "TOPS"
+PAGE_MS = {"qkv_m32700_k5376_n16128": 10.5752, "ragged_m8193_k5376_n16128": 2.7743}
+L2_FLUSH_BYTES = 256 << 20
+NOMINAL_INT8_OVER_BF16 = 2.0  # dense tensor peaks: 4.5 POPS int8 / 2.25 PFLOP/s bf16
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.lines: list[tuple[float, str]] = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+
+        def pump():
+            for line in self.proc.stdout:
+                self.lines.append((time.time(), line.strip()))
+
+        self.thread = threading.Thread(target=pump, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 10:
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [l for (t, l) in self.lines if t0 <= t <= t1 + 0.05]
+        if not rows:
+            rows = [l for (_, l) in self.lines[-3:]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in rows:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[2]))
+                smax.append(float(f[3]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float):
+    """Time the oracle on a bounded sample of rows (quantise + linear rows).
+    Returns (TOPS, rows, seconds, threads)."""
+    import oracle
+
+    def run(rows):
+        t = time.perf_counter()
+        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows])
+        oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
+        return time.perf_counter() - t
+
+    probe = 8
+    dt = run(probe)
+    rows = int(max(probe, min(cfg.M, probe * seconds / max(dt, 1e-6))))
+    dt = run(rows)
+    tops = 2.0 * rows * cfg.N * cfg.K / dt / 1e12
+    return tops, rows, dt, oracle.num_threads()
+
+
+def oracle_inputs(cfg):
+    import oracle
+
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw, s_w = oracle.rotate_quant_weight(W.numpy())
+    return workloads.bf16_bits(X), Qw, s_w, workloads.bf16_bits(bias)
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+
+    X_bits, Qw, s_w, bias_bits = oracle_inputs(cfg)
+    total_budget = 150.0
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    t_probe = time.perf_counter()
+    Qx, s_x = oracle.quantize_rows_bf16(X_bits[:4])
+    oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(4))
+    t_row = (time.perf_counter() - t_probe) / 4
+    rows = int(max(1, min(cfg.M, per_step / max(t_row, 1e-9))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows])
+        oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
+        dt = time.perf_counter() - t
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    tops = 2.0 * rows * cfg.N * cfg.K / (ms / 1e3) / 1e12
+    sample = (f"{rows} of {cfg.M} rows per step (quantize_and_rotate_rowwise of those rows + "
+              f"their {cfg.N} outputs each), oracle in plain C on host cores")
+    line = {"metric": METRIC, "value": tops, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "impl": "reference",
+            "config": config_dict(cfg, world),
+            "cpu_baseline": {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": tops, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(cfg, world):
+    return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "seed": cfg.seed,
+            "x_dist": cfg.x_dist, "outlier_channels": cfg.n_outlier,
+            "parallelism": f"replicas x{world} (rows independent, no collective)",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); X is also larger than L2",
+            "weights": "rotated + quantised once before timing (offline)"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import int8_quantized_linear_convrot256_b200 as ck
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    P = peaks()
+
+    X, W, bias = workloads.make_inputs(cfg)
+    Xd = X.to(dev)
+    bd = bias.to(dev)
+    Qw, s_w = ck.rotate_quant_weight(W.to(dev))
+    Wcpu = W
+    M, N, K = cfg.M, cfg.N, cfg.K
+    Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
+    s_x = torch.empty((M,), dtype=torch.float32, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ck.clear_device_error()
+
+    def step():
+        ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        ev[i][1].record(stream)
+        ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clocks.stop()
+    status = ck.device_error()
+    if status != ck.CK_OK:
+        raise RuntimeError(f"device error during the timed region: {ck.status_string(status)}")
+
+    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    s_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    ms_step = sum(s_ms) / len(s_ms)
+    ms_q = sum(q_ms) / len(q_ms)
+    ms_g = sum(g_ms) / len(g_ms)
+    if world > 1:
+        t = torch.tensor([ms_step, ms_q, ms_g], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_q, ms_g = t.tolist()
+
+    # ---- end to end through the public composite call, host buffers
+    X_host = X.pin_memory()
+    Y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd2 = torch.empty_like(Xd)
+    e2e_steps = max(1, min(args.steps, 10))
+    for _ in range(2):
+        Xd2.copy_(X_host, non_blocking=True)
+        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws)
+        Y_host.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xd2.copy_(X_host, non_blocking=True)
+        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws)
+        Y_host.copy_(Y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = t.item()
+
+    ops = 2.0 * M * N * K
+    value = world * ops / (ms_step / 1e3) / 1e12
+    e2e_value = world * ops / (ms_e2e / 1e3) / 1e12
+    gemm_tops = ops / (ms_g / 1e3) / 1e12
+    q_bytes = 3.0 * M * K + 4.0 * M
+    q_gbs = q_bytes / (ms_q / 1e3) / 1e9
+    int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(prof):
+        try:
+            d = json.load(open(prof))
+            if d.get("workload") == cfg.name:
+                traffic = d.get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            X_bits = workloads.bf16_bits(X)
+            import oracle
+
+            Qw_o, s_w_o = oracle.rotate_quant_weight(Wcpu.numpy())
+            tops, rows, dt, cores = oracle_sample(cfg, X_bits, Qw_o, s_w_o,
+                                                  workloads.bf16_bits(bias), args.cpu_seconds)
+            cpu = {"value": tops, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": f"{rows} of {cfg.M} rows (rotate+quantise and all {cfg.N} outputs of "
+                             f"those rows) in {dt:.1f} s, plain C oracle, OpenMP over rows"}
+        page_ms = PAGE_MS.get(cfg.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": (value / world) / (ops / (page_ms / 1e3) / 1e12) if page_ms else None,
+            "dtype": "int8", "data": "synthetic", "impl": "ours",
+            "config": config_dict(cfg, world),
+            "roofline": {"kernel": "gemm_i8_kernel (tcgen05 kind::i8 + fused epilogue)",
+                         "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
+                         "peak_source": f"{P['source']} bf16 burst {P['bf16_tflops']} TFLOP/s x "
+                                        f"nominal int8/bf16 ratio {NOMINAL_INT8_OVER_BF16}",
+                         "frac_of_spec_4500": gemm_tops / 4500.0,
+                         "ms_per_launch": ms_g},
+            "quantizer": {"kernel": "quant_rows_kernel (ConvRot256 + per-row INT8)",
+                          "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",
+                          "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
+                          "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
+                    "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
+                    "call": "ck_int8_linear with X copied from pinned host memory and Y copied back"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks.summary(t_wall0, t_wall1),
+        }
+    return line
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.HEADLINE.name, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = workloads.BY_NAME[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, cfg, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,204 @@
+/*
+ * ck.h — C ABI of the B200 (sm_100a) ConvRot256 INT8 linear library (libck.so).
+ *
+ * The method (sources are web pages, cited by title and section):
+ *  - comfy-kitchen 0.2.40 (PyPI page), "Huawei Ascend backend" and "HIP backend":
+ *    quantize_int8_rowwise, quantize_and_rotate_rowwise (a ConvRot rotation
+ *    fused with the dynamic per-row INT8 quantiser) and int8_linear (that
+ *    quantiser on the activation, then an INT8 matmul).
+ *  - sglang PR "Tune Kitchen INT8 row splitting for SM120", "Accuracy Test":
+ *    BF16 activations and bias, INT8 weights, FP32 row scales, ConvRot256;
+ *    outputs do not depend on how the M rows are split across calls.
+ *  - ComfyUI-AppleSilicon-FP8 README, "What it fixes" row 17: rotate the
+ *    activation online, quantise it per row, INT8 x INT8 -> INT32, with the
+ *    per-row rescale and the bias fused into the store epilogue; row 12: the
+ *    INT32 sums stay inside the int32 range.
+ *
+ * Definitions this library implements (the pages name the steps but print no
+ * formulas; these are the readings taken):
+ *  - ConvRot256: along K, every block of 256 consecutive values is replaced by
+ *    its normalised Walsh-Hadamard transform, computed in fp32 as 8 butterfly
+ *    stages h = 1, 2, 4, ..., 128 ((a, c) -> (a + c, a - c) on indices i and
+ *    i + h with bit h of i clear), then multiplied by 1/16.
+ *  - Per-row quantisation of a rotated row y[0..K): s = absmax(y) / 127
+ *    (one IEEE fp32 division), q[k] = round-half-even(y[k] / s) clamped to
+ *    [-127, 127] (-128 is never produced). A row of zeros gets s = 0, q = 0.
+ *  - Linear: acc[m][n] = sum_k Qx[m][k] * Qw[n][k] in int32 (exact for
+ *    K <= 132864), then Y[m][n] = bf16_rne(((float(acc) * s_x[m]) * s_w[n])
+ *    + float(bias[n])), every step an fp32 operation rounded to nearest even;
+ *    a NULL bias adds +0.0f.
+ *
+ * Conventions for every entry point:
+ *  - Every pointer argument is DEVICE memory (cudaMalloc, a PyTorch CUDA
+ *    tensor, ...) on the current device, owned by the caller. The library
+ *    allocates nothing, keeps no pointer after returning, and never
+ *    synchronises the stream or the device (except ck_get_device_error).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and runs asynchronously: on CK_OK the results are valid once the
+ *    stream reaches that point.
+ *  - All matrices are row-major. BF16 values are passed as their 16-bit
+ *    patterns (ck_bf16 is binary-compatible with __nv_bfloat16).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    non-CK_OK status means nothing was enqueued. Checks, in order:
+ *    CK_ERR_INVALID_VALUE (NULL pointer where one is required, negative size,
+ *    K <= 0, ldx < K), CK_ERR_UNSUPPORTED_SHAPE (K % 256 != 0, K > 132864,
+ *    N % 8 != 0, M or N >= 2^31), CK_ERR_MISALIGNED (an address or row stride
+ *    not 16-byte aligned where stated), CK_ERR_WORKSPACE, then
+ *    CK_ERR_ARCH (current device is not compute capability 10.0) and
+ *    CK_ERR_CUDA (a CUDA runtime call or launch failed).
+ *  - M == 0 (and N == 0 for the linear) is valid and enqueues nothing.
+ *  - The functions are thread-safe and may be called concurrently on
+ *    different streams; calls that write the same buffers must be ordered
+ *    by the caller.
+ *  - Device-side waits inside the kernels are bounded (about 4 s). If one
+ *    runs out the kernel records CK_ERR_DEVICE_TIMEOUT in a per-device error
+ *    word, stops its work and returns; outputs of that call are then
+ *    undefined. ck_get_device_error() reports it.
+ */
+#ifndef CK_H_
+#define CK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary-compatible with cudaStream_t. */
+typedef struct CUstream_st *ck_stream_t;
+
+/* A bfloat16 value as its bit pattern. */
+typedef uint16_t ck_bf16;
+
+typedef enum ck_status {
+    CK_OK = 0,
+    CK_ERR_INVALID_VALUE = 1,
+    CK_ERR_UNSUPPORTED_SHAPE = 2,
+    CK_ERR_MISALIGNED = 3,
+    CK_ERR_WORKSPACE = 4,
+    CK_ERR_ARCH = 5,
+    CK_ERR_CUDA = 6,
+    CK_ERR_DEVICE_TIMEOUT = 7
+} ck_status;
+
+/* Largest K for which |acc| <= K * 127^2 stays below 2^31, rounded down to a
+ * multiple of 256. */
+#define CK_MAX_K 132864
+
+/*
+ * Offline weight preparation (ComfyUI-AppleSilicon-FP8 README, row 17: the
+ * weights of a ConvRot checkpoint are stored rotated; sglang PR, Accuracy
+ * Test: INT8 weights with FP32 row scales).
+ *   W   [N, K] fp32, row stride K, 16-byte aligned.  (input)
+ *   Qw  [N, K] int8, row stride K, 16-byte aligned.  (output) ConvRot256 of
+ *       each row of W, quantised per row.
+ *   s_w [N] fp32, 16-byte aligned.                   (output) row scales.
+ * Requires K % 256 == 0 and K <= CK_MAX_K; N >= 0.
+ */
+ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw, float *s_w,
+                                 ck_stream_t stream);
+
+/*
+ * quantize_and_rotate_rowwise (comfy-kitchen, "Huawei Ascend backend" and
+ * "HIP backend": the fused ConvRot quantiser): ConvRot256 of every row of X,
+ * then dynamic per-row INT8 quantisation, in one pass over X.
+ *   X   [M, K] bf16 with row stride ldx elements (ldx >= K, ldx % 8 == 0),
+ *       16-byte aligned.                                      (input)
+ *   Qx  [M, K] int8, row stride K, 16-byte aligned.            (output)
+ *   s_x [M] fp32, 4-byte aligned.                              (output)
+ * Requires K % 256 == 0 and K <= CK_MAX_K.
+ */
+ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                     int8_t *Qx, float *s_x, ck_stream_t stream);
+
+/*
+ * quantize_int8_rowwise (comfy-kitchen, "Huawei Ascend backend"): the same
+ * per-row quantiser without the rotation. Same arguments and rules as
+ * ck_quantize_rotate_rowwise.
+ */
+ck_status ck_quantize_int8_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t *Qx, float *s_x, ck_stream_t stream);
+
+/*
+ * Bytes of device workspace ck_int8_linear needs for M rows of K features:
+ * the INT8 codes (M*K bytes) and the row scales (4*M bytes), each part
+ * rounded up to 256 bytes. Returns 0 for M <= 0 or K <= 0.
+ */
+size_t ck_int8_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * int8_linear (comfy-kitchen, "Huawei Ascend backend"; ComfyUI-AppleSilicon-FP8
+ * README, row 17): Y = bf16(((INT32 GEMM of the rotated, per-row quantised X
+ * with Qw) * s_x) * s_w + bias). Two kernels on `stream`: the fused
+ * rotate+quantise pass writes the codes and row scales into `workspace`, then
+ * the tcgen05 INT8 GEMM applies the epilogue as it stores Y. M may be any
+ * size (no row splitting): the ragged last tile is handled in the same launch.
+ *   X         [M, K] bf16, row stride ldx (ldx >= K, ldx % 8 == 0), 16-B aligned.
+ *   Qw        [N, K] int8 (already rotated, from ck_rotate_quant_weight),
+ *             row stride K, 16-B aligned.
+ *   s_w       [N] fp32, 16-B aligned.
+ *   bias      [N] bf16, 16-B aligned, or NULL (adds +0.0f).
+ *   Y         [M, N] bf16, row stride N, 16-B aligned.   (output)
+ *   workspace >= ck_int8_linear_workspace_bytes(M, K) bytes, 256-B aligned;
+ *             its contents on return are the codes (first M*K bytes) and the
+ *             row scales (at offset round_up(M*K, 256)).
+ * Requires K % 256 == 0, K <= CK_MAX_K, N % 8 == 0.
+ */
+ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
+                         const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                         void *workspace, size_t workspace_bytes, ck_stream_t stream);
+
+/*
+ * The GEMM and fused epilogue alone, on activations already quantised (by
+ * ck_quantize_rotate_rowwise):
+ *   Qx [M, K] int8 (16-B aligned), s_x [M] fp32 (4-B aligned), Qw/s_w/bias/Y as
+ *   for ck_int8_linear. Requires K % 256 == 0, K <= CK_MAX_K, N % 8 == 0.
+ */
+ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t *Qw,
+                                const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                                int64_t N, int64_t K, ck_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char *ck_status_string(ck_status status);
+
+/*
+ * Synchronises the current device, then returns CK_ERR_DEVICE_TIMEOUT if any
+ * kernel of this library on it gave up on a bounded wait since the last
+ * ck_clear_device_error(), CK_ERR_CUDA if the synchronisation itself failed,
+ * else CK_OK.
+ */
+ck_status ck_get_device_error(void);
+
+/* Resets the current device's error word (synchronous with the device). */
+ck_status ck_clear_device_error(void);
+
+/* ---- test hooks (used by the test suite; stable, but not part of the method) ---- */
+
+/*
+ * The INT32 accumulators of the GEMM, without the epilogue:
+ *   acc [M, N] int32, row stride N, 16-B aligned.  (output)
+ * Same kernel and tiling as ck_int8_gemm_rowscale.
+ */
+ck_status ck_test_int8_gemm_i32(const int8_t *Qx, const int8_t *Qw, int32_t *acc, int64_t M,
+                                int64_t N, int64_t K, ck_stream_t stream);
+
+/* Same as ck_quantize_int8_rowwise (the quantiser without the rotation). */
+ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                            int8_t *Qx, float *s_x, ck_stream_t stream);
+
+/*
+ * Fault injection for the bounded waits, host side only: with mode 1 the next
+ * GEMM launch on this thread's current device runs with its TMA producer
+ * issuing nothing, so the MMA warp's wait for the first stage can never be
+ * satisfied; the kernel must then record CK_ERR_DEVICE_TIMEOUT and return
+ * instead of hanging. The flag is consumed by that launch. mode 0 clears it.
+ * wait_limit_ns (> 0) replaces the default bound (about 4 s) for that launch.
+ */
+ck_status ck_test_inject_producer_stall(int mode, int64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CK_H_ */

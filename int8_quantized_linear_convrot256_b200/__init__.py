@@ -1,0 +1,253 @@
+"""ConvRot256 INT8 linear for NVIDIA B200 (sm_100a).
+
+Thin Python binding of ``libck.so`` (the C ABI declared in ``include/ck.h``):
+every function here only checks and marshals its arguments and calls the
+entry point of the same name; all arithmetic runs in the library's CUDA
+kernels. PyTorch supplies device memory and streams. There is no CPU path:
+if ``libck.so`` is missing, importing this package raises ImportError, and a
+call on a device that is not a B200 raises ``CKError`` (CK_ERR_ARCH).
+
+    import int8_quantized_linear_convrot256_b200 as ck
+    Qw, s_w = ck.rotate_quant_weight(W_fp32_cuda)          # offline, once
+    Y = ck.int8_linear(X_bf16_cuda, Qw, s_w, bias_bf16)    # per forward
+
+Method (web pages, by title and section): comfy-kitchen 0.2.40 "Huawei
+Ascend backend" (quantize_int8_rowwise, quantize_and_rotate_rowwise,
+int8_linear); sglang PR "Tune Kitchen INT8 row splitting for SM120",
+Accuracy Test (BF16 activations and bias, INT8 weights, FP32 row scales,
+ConvRot256); ComfyUI-AppleSilicon-FP8 README row 17 (rotate online, per-row
+quantise, INT8 x INT8 -> INT32, rescale + bias fused into the store).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libck.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "ck.h")
+
+CK_OK = 0
+CK_ERR_INVALID_VALUE = 1
+CK_ERR_UNSUPPORTED_SHAPE = 2
+CK_ERR_MISALIGNED = 3
+CK_ERR_WORKSPACE = 4
+CK_ERR_ARCH = 5
+CK_ERR_CUDA = 6
+CK_ERR_DEVICE_TIMEOUT = 7
+MAX_K = 132864
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m int8_quantized_linear_convrot256_b200.build`"
+        " (there is no CPU fallback)")
+
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+_st = ctypes.c_int
+
+lib = ctypes.CDLL(LIB_PATH)
+_SIGS = {
+    "ck_rotate_quant_weight": (_st, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "ck_quantize_rotate_rowwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ck_quantize_int8_rowwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ck_int8_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "ck_int8_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                             ctypes.c_size_t, _vp]),
+    "ck_int8_gemm_rowscale": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_status_string": (ctypes.c_char_p, [_st]),
+    "ck_get_device_error": (_st, []),
+    "ck_clear_device_error": (_st, []),
+    "ck_test_int8_gemm_i32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_test_quantize_rowwise_norotate": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ck_test_inject_producer_stall": (_st, [ctypes.c_int, _i64]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class CKError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def status_string(status: int) -> str:
+    return lib.ck_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != CK_OK:
+        raise CKError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if t.numel() and t.stride(-1) != 1:
+        raise ValueError(f"{name} must have unit stride in its last dimension")
+
+
+def _rows_contiguous(t: torch.Tensor, name: str) -> None:
+    if t.numel() and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_bytes(M: int, K: int) -> int:
+    return int(lib.ck_int8_linear_workspace_bytes(M, K))
+
+
+def rotate_quant_weight(W: torch.Tensor, Qw: torch.Tensor | None = None,
+                        s_w: torch.Tensor | None = None, stream=None):
+    """Offline: ConvRot256 along K and per-output-row INT8 of fp32 W [N, K]."""
+    _need(W, "W", torch.float32, 2)
+    _rows_contiguous(W, "W")
+    N, K = W.shape
+    if Qw is None:
+        Qw = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if s_w is None:
+        s_w = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _need(Qw, "Qw", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    _check(lib.ck_rotate_quant_weight(_ptr(W), N, K, _ptr(Qw), _ptr(s_w), _stream(stream)),
+           "ck_rotate_quant_weight")
+    return Qw, s_w
+
+
+def _quant(fn, name, X, Qx, s_x, stream):
+    _need(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    if Qx is None:
+        Qx = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if s_x is None:
+        s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _need(Qx, "Qx", torch.int8, 2)
+    _rows_contiguous(Qx, "Qx")
+    _need(s_x, "s_x", torch.float32, 1)
+    _check(fn(_ptr(X), M, K, ldx, _ptr(Qx), _ptr(s_x), _stream(stream)), name)
+    return Qx, s_x
+
+
+def quantize_rotate_rowwise(X: torch.Tensor, Qx=None, s_x=None, stream=None):
+    """quantize_and_rotate_rowwise: ConvRot256 + per-row INT8 of bf16 X [M, K]
+    (row stride X.stride(0)). Returns (Qx int8 [M, K], s_x fp32 [M])."""
+    return _quant(lib.ck_quantize_rotate_rowwise, "ck_quantize_rotate_rowwise", X, Qx, s_x, stream)
+
+
+def quantize_int8_rowwise(X: torch.Tensor, Qx=None, s_x=None, stream=None):
+    """quantize_int8_rowwise: per-row INT8 of bf16 X [M, K] without rotation."""
+    return _quant(lib.ck_quantize_int8_rowwise, "ck_quantize_int8_rowwise", X, Qx, s_x, stream)
+
+
+def test_quantize_rowwise_norotate(X: torch.Tensor, Qx=None, s_x=None, stream=None):
+    return _quant(lib.ck_test_quantize_rowwise_norotate, "ck_test_quantize_rowwise_norotate",
+                  X, Qx, s_x, stream)
+
+
+test_quantize_rowwise_norotate.__test__ = False
+
+
+def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[M, N] = bf16(((int8 GEMM of rotate+quantised X with Qw) * s_x) * s_w + bias)."""
+    _need(X, "X", torch.bfloat16, 2)
+    _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
+    _need(s_w, "s_w", torch.float32, 1)
+    M, K = X.shape
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, Qw {tuple(Qw.shape)}, s_w {tuple(s_w.shape)}")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    need = workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_int8_linear(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out), M, N, K,
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)), "ck_int8_linear")
+    return out
+
+
+def int8_gemm_rowscale(Qx: torch.Tensor, s_x: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                       bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """The GEMM + fused epilogue on already quantised activations."""
+    _need(Qx, "Qx", torch.int8, 2)
+    _rows_contiguous(Qx, "Qx")
+    _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
+    _need(s_x, "s_x", torch.float32, 1)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    M, K = Qx.shape
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_x.shape[0] != M or s_w.shape[0] != N:
+        raise ValueError("shape mismatch between Qx, s_x, Qw and s_w")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Qx.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    _check(lib.ck_int8_gemm_rowscale(_ptr(Qx), _ptr(s_x), _ptr(Qw), _ptr(s_w), _ptr(bias),
+                                     _ptr(out), M, N, K, _stream(stream)), "ck_int8_gemm_rowscale")
+    return out
+
+
+def test_int8_gemm_i32(Qx: torch.Tensor, Qw: torch.Tensor, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Raw INT32 accumulators of the GEMM (test hook)."""
+    _need(Qx, "Qx", torch.int8, 2)
+    _need(Qw, "Qw", torch.int8, 2)
+    M, K = Qx.shape
+    N = Qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=Qx.device)
+    _check(lib.ck_test_int8_gemm_i32(_ptr(Qx), _ptr(Qw), _ptr(out), M, N, K, _stream(stream)),
+           "ck_test_int8_gemm_i32")
+    return out
+
+
+test_int8_gemm_i32.__test__ = False
+
+
+def device_error() -> int:
+    """Synchronises the device; returns CK_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait."""
+    return int(lib.ck_get_device_error())
+
+
+def clear_device_error() -> None:
+    _check(lib.ck_clear_device_error(), "ck_clear_device_error")
+
+
+def inject_producer_stall(mode: int = 1, wait_limit_ns: int = 0) -> None:
+    _check(lib.ck_test_inject_producer_stall(mode, wait_limit_ns), "ck_test_inject_producer_stall")

@@ -1,0 +1,306 @@
+// C ABI of libck.so: host-side validation, per-device state, TMA tensor maps
+// and the launches. Declarations and the contract of every entry point are in
+// include/ck.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "ck.h"
+#include "ck_device.cuh"
+#include "internal.h"
+
+namespace {
+
+// Per-device error word for bounded waits that ran out (CK_ERR_DEVICE_TIMEOUT).
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kBlock = 256;
+
+struct DeviceState {
+    bool ready = false;
+    bool arch_ok = false;
+    int num_sms = 0;
+    unsigned *err = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+thread_local int t_stall_next = 0;
+thread_local int64_t t_stall_limit_ns = 0;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+ck_status check_k(int64_t K) {
+    if (K <= 0) return CK_ERR_INVALID_VALUE;
+    if (K % kBlock != 0 || K > CK_MAX_K) return CK_ERR_UNSUPPORTED_SHAPE;
+    return CK_OK;
+}
+
+// Returns the state of the current device, initialising it once (arch check,
+// SM count, address of the error word, tensor-map encoder).
+ck_status device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CK_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &st = g_dev[dev];
+    if (!st.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return CK_ERR_CUDA;
+        st.arch_ok = (major == 10 && minor == 0);
+        st.num_sms = sms;
+        if (st.arch_ok) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return CK_ERR_CUDA;
+            st.err = static_cast<unsigned *>(p);
+            if (!g_encode) {
+                void *fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                        cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || fn == nullptr)
+                    return CK_ERR_CUDA;
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+        }
+        st.ready = true;
+    }
+    if (!st.arch_ok) return CK_ERR_ARCH;
+    *out = &st;
+    return CK_OK;
+}
+
+// Row-major [rows, K] int8 matrix, box = box_rows x 128 bytes, 128-byte swizzle,
+// out-of-range elements read as zero.
+ck_status make_tmap_i8(CUtensorMap *tm, const void *base, int64_t rows, int64_t K, int box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(ck::kGemmBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const float *s_w,
+                   const ck_bf16 *bias, ck_bf16 *Y, int32_t *acc, int64_t M, int64_t N, int64_t K,
+                   DeviceState *st, cudaStream_t stream) {
+    CUtensorMap tmA, tmB;
+    std::memset(&tmA, 0, sizeof tmA);
+    std::memset(&tmB, 0, sizeof tmB);
+    ck_status s = make_tmap_i8(&tmA, Qx, M, K, ck::kGemmBM);
+    if (s != CK_OK) return s;
+    s = make_tmap_i8(&tmB, Qw, N, K, ck::kGemmBN);
+    if (s != CK_OK) return s;
+    ck::GemmParams p{};
+    p.s_x = s_x;
+    p.s_w = s_w;
+    p.bias = bias;
+    p.Y = Y;
+    p.acc = acc;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.err = st->err;
+    p.wait_limit_ns = ck::kDefaultWaitLimitNs;
+    p.stall_producer = 0;
+    if (t_stall_next) {
+        p.stall_producer = 1;
+        if (t_stall_limit_ns > 0) p.wait_limit_ns = static_cast<uint64_t>(t_stall_limit_ns);
+        t_stall_next = 0;
+        t_stall_limit_ns = 0;
+    }
+    cudaError_t e = ck::launch_gemm_i8(tmA, tmB, p, acc != nullptr, st->num_sms, stream);
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8_t *Qx,
+                       float *s_x, bool rotate, ck_stream_t stream) {
+    if (M < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (ldx < K && K > 0) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && (!X || !Qx || !s_x)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (M >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return CK_OK;
+    if (!aligned16(X) || !aligned16(Qx) || !aligned4(s_x) || ldx % 8 != 0) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, Qx, s_x,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status gemm_args(const int8_t *Qx, const int8_t *Qw, const void *Y, int64_t M, int64_t N,
+                    int64_t K) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (M > 0 && N > 0 && (!Qx || !Qw || !Y)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    return CK_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw, float *s_w,
+                                 ck_stream_t stream) {
+    if (N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (N > 0 && (!W || !Qw || !s_w)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return CK_OK;
+    if (!aligned16(W) || !aligned16(Qw) || !aligned16(s_w)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e =
+        ck::launch_quant_rows_f32(W, N, K, Qw, s_w, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                     int8_t *Qx, float *s_x, ck_stream_t stream) {
+    return quant_common(X, M, K, ldx, Qx, s_x, true, stream);
+}
+
+ck_status ck_quantize_int8_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t *Qx, float *s_x, ck_stream_t stream) {
+    return quant_common(X, M, K, ldx, Qx, s_x, false, stream);
+}
+
+ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                            int8_t *Qx, float *s_x, ck_stream_t stream) {
+    return quant_common(X, M, K, ldx, Qx, s_x, false, stream);
+}
+
+size_t ck_int8_linear_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return round256(size_t(M) * size_t(K)) + round256(size_t(M) * 4);
+}
+
+ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
+                         const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                         void *workspace, size_t workspace_bytes, ck_stream_t stream) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && N > 0 && (!X || !Qw || !s_w || !Y || !workspace)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Qw) || !aligned16(s_w) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CK_ERR_MISALIGNED;
+    if (workspace_bytes < ck_int8_linear_workspace_bytes(M, K)) return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    int8_t *Qx = static_cast<int8_t *>(workspace);
+    float *s_x = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                           round256(size_t(M) * size_t(K)));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, true, Qx, s_x, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
+}
+
+ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t *Qw,
+                                const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                                int64_t N, int64_t K, ck_stream_t stream) {
+    ck_status s = gemm_args(Qx, Qw, Y, M, N, K);
+    if (s != CK_OK) return s;
+    if (M > 0 && N > 0 && (!s_x || !s_w)) return CK_ERR_INVALID_VALUE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(Qx) || !aligned4(s_x) || !aligned16(Qw) || !aligned16(s_w) || !aligned16(Y) ||
+        (bias && !aligned16(bias)))
+        return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+ck_status ck_test_int8_gemm_i32(const int8_t *Qx, const int8_t *Qw, int32_t *acc, int64_t M,
+                                int64_t N, int64_t K, ck_stream_t stream) {
+    ck_status s = gemm_args(Qx, Qw, acc, M, N, K);
+    if (s != CK_OK) return s;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(Qx) || !aligned16(Qw) || !aligned16(acc)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return run_gemm(Qx, nullptr, Qw, nullptr, nullptr, nullptr, acc, M, N, K, st,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char *ck_status_string(ck_status status) {
+    switch (status) {
+        case CK_OK: return "CK_OK";
+        case CK_ERR_INVALID_VALUE: return "CK_ERR_INVALID_VALUE: null pointer, negative size, K <= 0 or ldx < K";
+        case CK_ERR_UNSUPPORTED_SHAPE: return "CK_ERR_UNSUPPORTED_SHAPE: K % 256 != 0, K > 132864, N % 8 != 0 or M/N >= 2^31";
+        case CK_ERR_MISALIGNED: return "CK_ERR_MISALIGNED: pointer or row stride not 16-byte aligned";
+        case CK_ERR_WORKSPACE: return "CK_ERR_WORKSPACE: workspace smaller than ck_int8_linear_workspace_bytes";
+        case CK_ERR_ARCH: return "CK_ERR_ARCH: current device is not compute capability 10.0 (B200)";
+        case CK_ERR_CUDA: return "CK_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+        case CK_ERR_DEVICE_TIMEOUT: return "CK_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    }
+    return "unknown ck_status";
+}
+
+ck_status ck_get_device_error(void) {
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CK_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, st->err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return CK_ERR_CUDA;
+    return v ? static_cast<ck_status>(v) : CK_OK;
+}
+
+ck_status ck_clear_device_error(void) {
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CK_ERR_CUDA;
+    const unsigned zero = 0;
+    if (cudaMemcpy(st->err, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+        return CK_ERR_CUDA;
+    return CK_OK;
+}
+
+ck_status ck_test_inject_producer_stall(int mode, int64_t wait_limit_ns) {
+    if (mode != 0 && mode != 1) return CK_ERR_INVALID_VALUE;
+    if (wait_limit_ns < 0) return CK_ERR_INVALID_VALUE;
+    t_stall_next = mode;
+    t_stall_limit_ns = mode ? wait_limit_ns : 0;
+    return CK_OK;
+}
+
+}  // extern "C"

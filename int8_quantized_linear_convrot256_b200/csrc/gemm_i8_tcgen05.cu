@@ -1,0 +1,347 @@
+// Dense INT8 x INT8 -> INT32 GEMM on the sm_100a tensor cores (tcgen05
+// kind::i8) with the dequantisation epilogue fused into the store.
+//
+// What is computed (ComfyUI-AppleSilicon-FP8 README, "What it fixes" row 17:
+// INT8 x INT8 -> INT32, then the per-row rescale and the bias in the store
+// epilogue so the int32 product never reaches global memory; sglang PR "Tune
+// Kitchen INT8 row splitting for SM120", Accuracy Test: INT8 weights, FP32
+// row scales, BF16 bias and output):
+//   acc[m][n] = sum_k Qx[m][k] * Qw[n][k]                      (exact, int32)
+//   Y[m][n]   = bf16_rne(((float(acc) * s_x[m]) * s_w[n]) + float(bias[n]))
+//
+// Design:
+//  * Persistent CTAs, one per SM (192 KB of shared memory each), walking
+//    128 x 256 output tiles in groups of 16 M-tiles so that concurrently
+//    running CTAs share the same A rows and B columns in L2.
+//  * Warp roles: warp 0 = TMA producer (one lane), warp 1 = MMA issuer (one
+//    lane; the warp also owns the TMEM allocation), warps 2-5 = epilogue.
+//  * 4-stage shared-memory ring of K-blocks (128 int8 along K): A 128 x 128,
+//    B 256 x 128, both K-major with the 128-byte swizzle, loaded by 2-D TMA.
+//    Out-of-range rows (ragged M, ragged N) are zero-filled by TMA, so any M
+//    runs in one launch.
+//  * tcgen05.mma kind::i8, M = 128, N = 256, K = 32 per instruction, int32
+//    accumulators in TMEM; two accumulator buffers (2 x 256 columns = all
+//    512) so the epilogue of one tile overlaps the main loop of the next.
+//  * Epilogue: tcgen05.ld 32 lanes x 32 columns per warp, fp32 math with
+//    explicit _rn intrinsics in the definition's order, BF16 pack, 16-byte
+//    stores clipped at M and N.
+//  * Every wait is bounded; on expiry the kernel records a timeout in the
+//    device error word, lets in-flight copies and MMAs finish, frees TMEM
+//    and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ck_device.cuh"
+#include "internal.h"
+
+namespace ck {
+namespace {
+
+constexpr int BM = kGemmBM;
+constexpr int BN = kGemmBN;
+constexpr int BK = kGemmBK;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK;
+constexpr int kBBytes = BN * BK;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kAccBufs = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr int kEpilogueThreads = 128;
+constexpr int kGroupM = 16;
+constexpr int kUmmaK = 32;  // int8 elements (bytes) per tcgen05.mma
+
+struct alignas(8) Control {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[kAccBufs];
+    uint64_t tmem_empty[kAccBufs];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + sizeof(Control);
+
+// Instruction descriptor: D = S32 (bits 4-5 = 2), A and B signed 8-bit
+// (bits 7-9 and 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at
+// bits 24-28.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
+                            (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major operand written by TMA with
+// the 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart
+// (stride byte offset), descriptor version 1, layout type 2 (128B swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+           (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int &mt, int &nt) {
+    const int per_group = kGroupM * num_n;
+    const int g = tile / per_group;
+    const int r = tile - g * per_group;
+    const int first_m = g * kGroupM;
+    const int gsz = min(kGroupM, num_m - first_m);
+    mt = first_m + r % gsz;
+    nt = r / gsz;
+}
+
+__device__ __forceinline__ void raise_timeout(volatile int *abort, unsigned *err) {
+    *abort = 1;
+    atomicMax(err, kDevErrTimeout);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <bool kRaw>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Control *ctl = reinterpret_cast<Control *>(smem + size_t(kStages) * kStageBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (p.M + BM - 1) / BM;
+    const int num_n = (p.N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nk = p.K / BK;
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&ctl->full[s]), 1);
+            mbar_init(smem_u32(&ctl->empty[s]), 1);
+        }
+        for (int a = 0; a < kAccBufs; ++a) {
+            mbar_init(smem_u32(&ctl->tmem_full[a]), 1);
+            mbar_init(smem_u32(&ctl->tmem_empty[a]), kEpilogueThreads);
+        }
+        mbar_init(smem_u32(&ctl->drain), 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    volatile int *abort = &ctl->abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_parity = 0;
+            bool ok = true;
+            if (!p.stall_producer) {
+                for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                    int mt, nt;
+                    tile_coords(tile, num_m, num_n, mt, nt);
+                    for (int kb = 0; kb < nk; ++kb) {
+                        const uint32_t empty = smem_u32(&ctl->empty[stage]);
+                        const uint32_t full = smem_u32(&ctl->full[stage]);
+                        if (!mbar_wait_bounded(empty, phase ^ 1u, limit, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(full, kStageBytes);
+                        const uint32_t a_dst = smem_u32(smem + size_t(stage) * kStageBytes);
+                        tma_load_2d(a_dst, &tmA, kb * BK, mt * BM, full);
+                        tma_load_2d(a_dst + kABytes, &tmB, kb * BK, nt * BN, full);
+                        issued |= 1u << stage;
+                        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            // Never leave a bulk copy in flight into shared memory: wait for
+            // the last copy issued into every stage to land.
+            for (int s = 0; s < kStages; ++s)
+                if (issued & (1u << s))
+                    if (!mbar_wait_bounded(smem_u32(&ctl->full[s]), (last_parity >> s) & 1u, limit,
+                                           nullptr))
+                        raise_timeout(abort, p.err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                if (!mbar_wait_bounded(smem_u32(&ctl->tmem_empty[acc]), acc_phase ^ 1u, limit,
+                                       abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + uint32_t(acc * BN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_src = smem_u32(smem + size_t(stage) * kStageBytes);
+                    const uint64_t adesc = smem_desc_sw128(a_src);
+                    const uint64_t bdesc = smem_desc_sw128(a_src + kABytes);
+#pragma unroll
+                    for (int k = 0; k < BK / kUmmaK; ++k) {
+                        // advance the start address by k * 32 bytes (>> 4)
+                        umma_i8(d, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), kIdesc,
+                                (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&ctl->empty[stage]));
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&ctl->tmem_full[acc]));
+                if (++acc == kAccBufs) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            // All MMAs issued by this thread complete before TMEM is freed.
+            umma_commit(smem_u32(&ctl->drain));
+            if (!mbar_wait_bounded(smem_u32(&ctl->drain), 0u, limit, nullptr))
+                raise_timeout(abort, p.err);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2-5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            int mt, nt;
+            tile_coords(tile, num_m, num_n, mt, nt);
+            if (!mbar_wait_bounded(smem_u32(&ctl->tmem_full[acc]), acc_phase, limit, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int row = mt * BM + quarter * 32 + lane;
+            const bool row_ok = row < p.M;
+            float sx = 0.0f;
+            if (!kRaw && row_ok) sx = p.s_x[row];
+            const uint32_t tbase =
+                tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
+                tmem_ld_wait();
+                const int n0 = nt * BN + c * 32;
+                if (!row_ok) continue;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int n = n0 + 8 * g;
+                    if (n >= p.N) break;
+                    if (kRaw) {
+                        int4 *dst = reinterpret_cast<int4 *>(p.acc + int64_t(row) * p.N + n);
+                        dst[0] = make_int4(int(r[8 * g + 0]), int(r[8 * g + 1]), int(r[8 * g + 2]),
+                                           int(r[8 * g + 3]));
+                        dst[1] = make_int4(int(r[8 * g + 4]), int(r[8 * g + 5]), int(r[8 * g + 6]),
+                                           int(r[8 * g + 7]));
+                    } else {
+                        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
+                        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n + 4));
+                        const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        float b[8];
+                        if (p.bias) {
+                            const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
+                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                b[2 * i] = __uint_as_float(bw[i] << 16);
+                                b[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) b[i] = 0.0f;
+                        }
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float v = __int2float_rn(int(r[8 * g + i]));
+                            v = __fmul_rn(v, sx);
+                            v = __fmul_rn(v, sw[i]);
+                            f[i] = __fadd_rn(v, b[i]);
+                        }
+                        uint4 out;
+                        out.x = bf16x2_rn(f[0], f[1]);
+                        out.y = bf16x2_rn(f[2], f[3]);
+                        out.z = bf16x2_rn(f[4], f[5]);
+                        out.w = bf16x2_rn(f[6], f[7]);
+                        *reinterpret_cast<uint4 *>(p.Y + int64_t(row) * p.N + n) = out;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
+            if (++acc == kAccBufs) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (!ok) raise_timeout(abort, p.err);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                           bool raw_i32, int num_sms, cudaStream_t stream) {
+    if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+    const int num_tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+    cudaError_t e;
+    if (raw_i32) {
+        e = cudaFuncSetAttribute(gemm_i8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        gemm_i8_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+    } else {
+        e = cudaFuncSetAttribute(gemm_i8_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        gemm_i8_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ck

@@ -1,0 +1,42 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace ck {
+
+// ---- fused ConvRot256 + per-row INT8 quantiser (quant_rotate.cu)
+
+// Rows of bf16 (bit patterns) with row stride ldx; rotate=false skips ConvRot.
+cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                   bool rotate, int8_t *Q, float *S, cudaStream_t stream);
+
+// Rows of fp32 with row stride K (offline weight preparation), always rotated.
+cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,
+                                  cudaStream_t stream);
+
+// ---- tcgen05 INT8 GEMM with fused epilogue (gemm_i8_tcgen05.cu)
+
+struct GemmParams {
+    const float *s_x;       // [M]
+    const float *s_w;       // [N]
+    const uint16_t *bias;   // [N] bf16 bits or nullptr
+    uint16_t *Y;            // [M, N] bf16 bits (epilogue mode)
+    int32_t *acc;           // [M, N] int32 (raw accumulator mode)
+    int M, N, K;
+    unsigned *err;          // device error word
+    uint64_t wait_limit_ns; // bound on every device-side wait
+    int stall_producer;     // test hook: TMA producer issues nothing
+};
+
+// Tile sizes of the GEMM (also used by the host to build the TMA boxes).
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 128;
+
+cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                           bool raw_i32, int num_sms, cudaStream_t stream);
+
+}  // namespace ck

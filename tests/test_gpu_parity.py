@@ -1,0 +1,291 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bar (ConvRot256 INT8 linear as defined in include/ck.h):
+  * INT8 codes, FP32 row scales and INT32 accumulators: bit-exact.
+  * BF16 outputs: within 1 bf16 ulp (the distance between the two bit
+    patterns on the ordered bf16 line); the kernel computes the epilogue with
+    the same fp32 operations in the same order, so 0 is expected.
+Inputs come from the seeded generators in ``workloads`` (shared by both
+sides); every expected value comes from ``oracle``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+BF16_ULP_TOL = 1
+
+
+@pytest.fixture(scope="module")
+def ck():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import int8_quantized_linear_convrot256_b200 as m
+
+    m.clear_device_error()
+    yield m
+    assert m.device_error() == m.CK_OK
+
+
+def bf16_ordered(bits: np.ndarray) -> np.ndarray:
+    """Map bf16 bit patterns to integers whose differences count ulps."""
+    b = bits.astype(np.int32)
+    return np.where(b & 0x8000, 0x8000 - b, b)
+
+
+def assert_bf16_close(got_bits: np.ndarray, ref_bits: np.ndarray, tol: int = BF16_ULP_TOL):
+    d = np.abs(bf16_ordered(got_bits) - bf16_ordered(ref_bits))
+    assert d.max(initial=0) <= tol, f"max bf16 ulp distance {d.max()} at {np.unravel_index(d.argmax(), d.shape)}"
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    t = t.cpu()
+    if t.dtype == torch.bfloat16:
+        return workloads.bf16_bits(t)
+    return t.numpy()
+
+
+def dev(t):
+    return t.cuda()
+
+
+# ------------------------------------------------------------------ quantiser
+
+
+QUANT_SHAPES = [(1, 256), (3, 512), (37, 768), (129, 5376), (7, 7168), (5, 28672),
+                (2, 32768), (3, 33024), (2, 132864), (300, 256), (1000, 512)]
+
+
+@pytest.mark.parametrize("M,K", QUANT_SHAPES)
+def test_quantize_rotate_bit_exact(ck, M, K):
+    cfg = workloads.custom(M, K, 8, seed=M * 7 + K)
+    X, _, _ = workloads.make_inputs(cfg)
+    Qx, s_x = ck.quantize_rotate_rowwise(dev(X))
+    rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=True)
+    assert np.array_equal(to_np(s_x).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(to_np(Qx), rq)
+
+
+@pytest.mark.parametrize("M,K", [(5, 256), (33, 1024), (4, 33024)])
+def test_quantize_norotate_bit_exact(ck, M, K):
+    cfg = workloads.custom(M, K, 8, seed=M + K)
+    X, _, _ = workloads.make_inputs(cfg)
+    for fn in (ck.quantize_int8_rowwise, ck.test_quantize_rowwise_norotate):
+        Qx, s_x = fn(dev(X))
+        rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=False)
+        assert np.array_equal(to_np(s_x).view(np.uint32), rs.view(np.uint32))
+        assert np.array_equal(to_np(Qx), rq)
+
+
+def test_quantize_row_stride(ck):
+    cfg = workloads.custom(19, 768, 8, seed=3)
+    X, _, _ = workloads.make_inputs(cfg)
+    wide = torch.full((19, 768 + 136), float("nan"), dtype=torch.bfloat16)
+    wide[:, :768] = X
+    Xv = dev(wide)[:, :768]
+    assert Xv.stride(0) == 904
+    Qx, s_x = ck.quantize_rotate_rowwise(Xv)
+    rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X))
+    assert np.array_equal(to_np(Qx), rq) and np.array_equal(to_np(s_x), rs)
+
+
+def test_quantize_special_rows(ck):
+    """Zero rows, ties (no rotation, s = 1), tiny rows whose scale is below
+    2^-120 (exact division path), huge and negative rows."""
+    K = 512
+    rows = np.zeros((8, K), np.float32)
+    rows[1, :16] = [127.0, -127.0, 0.5, 1.5, 2.5, 3.5, -0.5, -2.5, -3.5, 0.4921875, 126.5, -126.5,
+                    0.0, 7.25, -7.75, 100.5]
+    rng = np.random.default_rng(0)
+    rows[2] = rng.standard_normal(K) * 1e-38
+    rows[3] = rng.standard_normal(K) * 3e38 / 300
+    rows[4] = -np.abs(rng.standard_normal(K))
+    rows[5, 7] = 1e-40
+    rows[6] = rng.standard_normal(K) * 2.0 ** -110
+    rows[7] = 1.0
+    X = torch.from_numpy(rows).to(torch.bfloat16)
+    xb = workloads.bf16_bits(X)
+    for rot in (True, False):
+        fn = ck.quantize_rotate_rowwise if rot else ck.quantize_int8_rowwise
+        Qx, s_x = fn(dev(X))
+        rq, rs = oracle.quantize_rows_bf16(xb, rotate=rot)
+        assert np.array_equal(to_np(s_x).view(np.uint32), rs.view(np.uint32)), rot
+        assert np.array_equal(to_np(Qx), rq), rot
+
+
+def test_quantize_near_half_integers_take_exact_path(ck):
+    """Rows whose scale is a power of two (absmax = 127 * 2^e) and whose
+    values are (k + 0.5) * 2^e: every y / s is an exact tie, so the fast
+    reciprocal path must hand them to the exact division (ties to even)."""
+    K = 256
+    rng = np.random.default_rng(5)
+    M = 64
+    rows = np.zeros((M, K), np.float32)
+    for m in range(M):
+        e = int(rng.integers(-10, 11))
+        s = np.float32(2.0 ** e)
+        k = rng.integers(-126, 126, K).astype(np.float32) + np.float32(0.5)
+        rows[m] = k * s
+        rows[m, 0] = np.float32(127) * s
+    X = torch.from_numpy(rows).to(torch.bfloat16)
+    assert np.array_equal(X.float().numpy(), rows)  # exactly representable
+    Qx, s_x = ck.quantize_int8_rowwise(dev(X))
+    rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=False)
+    assert np.array_equal(to_np(Qx), rq) and np.array_equal(to_np(s_x), rs)
+    assert np.all(np.abs(rq[:, 1:].astype(np.int32)) % 2 == 0)  # ties went to even
+
+
+@pytest.mark.parametrize("N,K", [(8, 256), (264, 768), (520, 5376), (16, 33024)])
+def test_rotate_quant_weight_bit_exact(ck, N, K):
+    cfg = workloads.custom(1, K, N, seed=N + K)
+    _, W, _ = workloads.make_inputs(cfg)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    rq, rs = oracle.rotate_quant_weight(W.numpy())
+    assert np.array_equal(to_np(s_w).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(to_np(Qw), rq)
+
+
+# ------------------------------------------------------------------ GEMM
+
+
+GEMM_SHAPES = [(1, 8, 256), (3, 17 * 8, 256), (127, 256, 512), (128, 256, 512), (129, 264, 768),
+               (300, 520, 512), (257, 1032, 1024), (640, 512, 2048), (1, 256, 5376)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_i32_bit_exact(ck, M, N, K):
+    rng = np.random.default_rng(M * 31 + N * 7 + K)
+    a = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    b = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    acc = ck.test_int8_gemm_i32(dev(torch.from_numpy(a)), dev(torch.from_numpy(b)))
+    assert np.array_equal(to_np(acc), oracle.gemm_i32(a, b))
+
+
+def test_gemm_i32_extreme_codes(ck):
+    K = 28672
+    a = np.full((130, K), 127, np.int8)
+    a[1::2] = -127
+    b = np.full((16, K), 127, np.int8)
+    b[3] = -127
+    acc = to_np(ck.test_int8_gemm_i32(dev(torch.from_numpy(a)), dev(torch.from_numpy(b))))
+    assert np.array_equal(acc, oracle.gemm_i32(a, b))
+    assert acc[0, 0] == 462450688 and acc[1, 0] == -462450688
+
+
+# ------------------------------------------------------------------ whole linear
+
+
+def _oracle_linear(X, W, bias):
+    Qw, s_w = oracle.rotate_quant_weight(W.numpy())
+    bb = None if bias is None else workloads.bf16_bits(bias)
+    Y, Qx, s_x, acc = oracle.int8_linear(workloads.bf16_bits(X), Qw, s_w, bb)
+    return Y, Qw, s_w
+
+
+LINEAR_SHAPES = [(128, 512, 512), (1, 256, 8), (129, 768, 264), (255, 512, 520), (257, 1024, 256),
+                 (300, 5376, 512), (64, 28672, 264)]
+
+
+@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES)
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_int8_linear_matches_oracle(ck, M, K, N, with_bias):
+    cfg = workloads.custom(M, K, N, seed=M + K + N)
+    X, W, bias = workloads.make_inputs(cfg)
+    if not with_bias:
+        bias = None
+    Yr, Qw_r, s_w_r = _oracle_linear(X, W, bias)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    assert np.array_equal(to_np(Qw), Qw_r)
+    Y = ck.int8_linear(dev(X), Qw, s_w, None if bias is None else dev(bias))
+    assert_bf16_close(to_np(Y), Yr)
+
+
+def test_int8_gemm_rowscale_matches_oracle(ck):
+    cfg = workloads.custom(200, 1024, 264, seed=77)
+    X, W, bias = workloads.make_inputs(cfg)
+    Yr, Qw_r, s_w_r = _oracle_linear(X, W, bias)
+    Qx, s_x = ck.quantize_rotate_rowwise(dev(X))
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    Y = ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, dev(bias))
+    assert_bf16_close(to_np(Y), Yr)
+
+
+def test_empty_m_is_a_noop(ck):
+    Qw = torch.zeros((8, 256), dtype=torch.int8, device="cuda")
+    s_w = torch.ones(8, device="cuda")
+    X = torch.zeros((0, 256), dtype=torch.bfloat16, device="cuda")
+    Y = ck.int8_linear(X, Qw, s_w)
+    assert Y.shape == (0, 8)
+
+
+def test_row_split_invariance(ck):
+    """Outputs for M = 8193 in one launch equal those of the same rows split
+    into calls of 8192 + 1 and 4096 + 4096 + 1 (bit-exact)."""
+    cfg = workloads.custom(8193, 512, 264, seed=8193)
+    X, W, bias = workloads.make_inputs(cfg)
+    Xd, bd = dev(X), dev(bias)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    full = to_np(ck.int8_linear(Xd, Qw, s_w, bd))
+    for cuts in ([0, 8192, 8193], [0, 4096, 8192, 8193]):
+        parts = [to_np(ck.int8_linear(Xd[a:b], Qw, s_w, bd)) for a, b in zip(cuts[:-1], cuts[1:])]
+        assert np.array_equal(np.concatenate(parts), full)
+
+
+def test_dirty_workspace_and_output_are_overwritten(ck):
+    cfg = workloads.custom(130, 512, 264, seed=5)
+    X, W, bias = workloads.make_inputs(cfg)
+    Yr, _, _ = _oracle_linear(X, W, bias)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    ws = torch.full((ck.workspace_bytes(130, 512),), 0x5A, dtype=torch.uint8, device="cuda")
+    out = torch.full((130, 264), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ck.int8_linear(dev(X), Qw, s_w, dev(bias), out=out, workspace=ws)
+    assert_bf16_close(to_np(out), Yr)
+
+
+# ------------------------------------------------------------------ full-size configs
+
+
+def _sample_rows(M):
+    rows = {0, 1, 126, 127, 128, 129, M // 2, M - 129, M - 128, M - 2, M - 1}
+    rng = np.random.default_rng(M)
+    rows |= set(rng.integers(0, M, 24).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < M), np.int64)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", workloads.CONFIGS, ids=[c.name for c in workloads.CONFIGS])
+def test_full_size_config(ck, cfg):
+    """At the full sizes, in the launch configuration the benchmark times:
+    every code and row scale of activations and weights bit-exact; INT32
+    accumulators and BF16 outputs of sampled rows (tile edges and the ragged
+    last row included) against the oracle computed row by row."""
+    X, W, bias = workloads.make_inputs(cfg)
+    Xd, Wd, bd = dev(X), dev(W), dev(bias)
+    Qw, s_w = ck.rotate_quant_weight(Wd)
+    del Wd
+    rqw, rsw = oracle.rotate_quant_weight(W.numpy())
+    assert np.array_equal(to_np(s_w).view(np.uint32), rsw.view(np.uint32))
+    assert np.array_equal(to_np(Qw), rqw)
+    del W
+
+    ws = torch.empty((ck.workspace_bytes(cfg.M, cfg.K),), dtype=torch.uint8, device="cuda")
+    Y = ck.int8_linear(Xd, Qw, s_w, bd, workspace=ws)
+    torch.cuda.synchronize()
+    Qx = ws[: cfg.M * cfg.K].view(cfg.M, cfg.K).view(torch.int8)
+    off = (cfg.M * cfg.K + 255) // 256 * 256
+    s_x = ws[off: off + 4 * cfg.M].view(torch.float32)
+    rqx, rsx = oracle.quantize_rows_bf16(workloads.bf16_bits(X))
+    assert np.array_equal(to_np(s_x).view(np.uint32), rsx.view(np.uint32))
+    assert np.array_equal(to_np(Qx), rqx)
+
+    rows = _sample_rows(cfg.M)
+    Yr = oracle.linear_rows(rqx, rsx, rqw, rsw, workloads.bf16_bits(bias), rows)
+    Ys = to_np(Y[torch.from_numpy(rows).cuda()])
+    assert_bf16_close(Ys, Yr)
+
+    acc_rows = ck.test_int8_gemm_i32(Qx[torch.from_numpy(rows[:8]).cuda()].contiguous(), Qw)
+    assert np.array_equal(to_np(acc_rows), oracle.gemm_i32(rqx[rows[:8]], rqw))
