@@ -41,7 +41,7 @@ MAX_K = 132864
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m int8_quantized_linear_convrot256_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python int8_quantized_linear_convrot256_b200/build.py`"
         " (there is no CPU fallback)")
 
 _i64 = ctypes.c_int64

@@ -1,6 +1,8 @@
 """Builds libck.so in-tree with nvcc for sm_100a (B200) only.
 
-    python -m int8_quantized_linear_convrot256_b200.build [--force] [--verbose]
+    python int8_quantized_linear_convrot256_b200/build.py [--force] [--verbose]
+
+(run as a script: importing the package itself needs a built libck.so)
 
 Each .cu under csrc/ is compiled to an object under _build/, then linked into
 int8_quantized_linear_convrot256_b200/libck.so with the CUDA runtime linked
