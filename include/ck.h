@@ -159,6 +159,33 @@ ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t
                                 const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
                                 int64_t N, int64_t K, ck_stream_t stream);
 
+/* Size of the device array that ck_int8_linear_noalloc uses as its
+ * workspace: 32 MiB, enough for ck_int8_linear_workspace_bytes(M, K) of e.g.
+ * M = 4096, K = 8000 or M = 1024, K = 32512. */
+#define CK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * ck_int8_linear without a caller workspace, for callers that cannot allocate
+ * device memory (a plugin inside an engine that owns all device memory and
+ * gives it no workspace, code with a memory budget fixed at start-up, code
+ * that must not risk the device-wide synchronisation cudaFree can cause).
+ * The pages have no counterpart to this entry point; it exists for such
+ * callers only. Arguments and results are those of ck_int8_linear minus the
+ * workspace: the activation codes and row scales go to one file-scope device
+ * array of CK_NOALLOC_SCRATCH_BYTES instead, which every GPU that loads this
+ * part of the library holds until the process exits. Calls need
+ * ck_int8_linear_workspace_bytes(M, K) <= CK_NOALLOC_SCRATCH_BYTES, else
+ * CK_ERR_WORKSPACE is returned and nothing is launched. All calls on a device
+ * share the array (it keeps the last call's contents; each call rewrites all
+ * it reads, so nothing needs clearing), so calls whose work overlaps on the
+ * GPU race and give wrong results: order them. The first call on a device
+ * looks up the array's device address with that device current; make that
+ * first call before any stream capture. Allocates nothing.
+ */
+ck_status ck_int8_linear_noalloc(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
+                                 const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                                 ck_stream_t stream);
+
 /* A static, human-readable name for a status code. */
 const char *ck_status_string(ck_status status);
 

@@ -38,6 +38,7 @@ CK_ERR_ARCH = 5
 CK_ERR_CUDA = 6
 CK_ERR_DEVICE_TIMEOUT = 7
 MAX_K = 132864
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -57,6 +58,7 @@ _SIGS = {
     "ck_int8_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                              ctypes.c_size_t, _vp]),
     "ck_int8_gemm_rowscale": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
     "ck_clear_device_error": (_st, []),
@@ -195,6 +197,33 @@ def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
     _check(lib.ck_int8_linear(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out), M, N, K,
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)), "ck_int8_linear")
+    return out
+
+
+def int8_linear_noalloc(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                        bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """int8_linear for callers that cannot allocate device memory: the codes
+    and row scales go to the library's fixed 32 MiB device array instead of a
+    workspace (needs workspace_bytes(M, K) <= NOALLOC_SCRATCH_BYTES). Calls on
+    one device share that array, so they must not overlap on the GPU. ``out``
+    should be passed by such callers (otherwise this wrapper allocates it)."""
+    _need(X, "X", torch.bfloat16, 2)
+    _need(Qw, "Qw", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    M, K = X.shape
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_w.shape[0] != N or (bias is not None and bias.shape[0] != N):
+        raise ValueError("shape mismatch between X, Qw, s_w and bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_int8_linear_noalloc(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out),
+                                      M, N, K, _stream(stream)), "ck_int8_linear_noalloc")
     return out
 
 

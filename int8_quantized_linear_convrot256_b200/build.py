@@ -34,7 +34,7 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
 PER_FILE = {
     "quant_rotate.cu": ["-fmad=false"],
 }
-SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu"]
+SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "noalloc.cu"]
 HEADERS = ["ck_device.cuh", "internal.h", "libck.map"]
 
 
