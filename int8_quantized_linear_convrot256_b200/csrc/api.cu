@@ -98,12 +98,15 @@ ck_status make_tmap_i8(CUtensorMap *tm, const void *base, int64_t rows, int64_t 
 ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const float *s_w,
                    const ck_bf16 *bias, ck_bf16 *Y, int32_t *acc, int64_t M, int64_t N, int64_t K,
                    DeviceState *st, cudaStream_t stream) {
+    ck::GemmPlan plan{};
+    if (ck::plan_gemm(static_cast<int>(M), static_cast<int>(N), st->num_sms, &plan) != cudaSuccess)
+        return CK_ERR_CUDA;
     CUtensorMap tmA, tmB;
     std::memset(&tmA, 0, sizeof tmA);
     std::memset(&tmB, 0, sizeof tmB);
     ck_status s = make_tmap_i8(&tmA, Qx, M, K, ck::kGemmBM);
     if (s != CK_OK) return s;
-    s = make_tmap_i8(&tmB, Qw, N, K, ck::kGemmBN);
+    s = make_tmap_i8(&tmB, Qw, N, K, plan.b_box_rows);
     if (s != CK_OK) return s;
     ck::GemmParams p{};
     p.s_x = s_x;
@@ -123,7 +126,7 @@ ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const f
         t_stall_next = 0;
         t_stall_limit_ns = 0;
     }
-    cudaError_t e = ck::launch_gemm_i8(tmA, tmB, p, acc != nullptr, st->num_sms, stream);
+    cudaError_t e = ck::launch_gemm_i8(tmA, tmB, p, acc != nullptr, plan, stream);
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 

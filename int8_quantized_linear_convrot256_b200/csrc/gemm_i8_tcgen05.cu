@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "ck_device.cuh"
 #include "internal.h"
@@ -80,12 +81,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
            (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int &mt, int &nt) {
-    const int per_group = kGroupM * num_n;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int &mt, int &nt,
+                                            int group_m = kGroupM) {
+    const int per_group = group_m * num_n;
     const int g = tile / per_group;
     const int r = tile - g * per_group;
-    const int first_m = g * kGroupM;
-    const int gsz = min(kGroupM, num_m - first_m);
+    const int first_m = g * group_m;
+    const int gsz = min(group_m, num_m - first_m);
     mt = first_m + r % gsz;
     nt = r / gsz;
 }
@@ -99,6 +101,10 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
 }
+
+template <bool kRaw>
+__device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t tbase, int row,
+                                                   int n_tile0);
 
 template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -245,64 +251,9 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const int row = mt * BM + quarter * 32 + lane;
-            const bool row_ok = row < p.M;
-            float sx = 0.0f;
-            if (!kRaw && row_ok) sx = p.s_x[row];
             const uint32_t tbase =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
-                tmem_ld_wait();
-                const int n0 = nt * BN + c * 32;
-                if (!row_ok) continue;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int n = n0 + 8 * g;
-                    if (n >= p.N) break;
-                    if (kRaw) {
-                        int4 *dst = reinterpret_cast<int4 *>(p.acc + int64_t(row) * p.N + n);
-                        dst[0] = make_int4(int(r[8 * g + 0]), int(r[8 * g + 1]), int(r[8 * g + 2]),
-                                           int(r[8 * g + 3]));
-                        dst[1] = make_int4(int(r[8 * g + 4]), int(r[8 * g + 5]), int(r[8 * g + 6]),
-                                           int(r[8 * g + 7]));
-                    } else {
-                        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
-                        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n + 4));
-                        const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                        float b[8];
-                        if (p.bias) {
-                            const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
-                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                b[2 * i] = __uint_as_float(bw[i] << 16);
-                                b[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) b[i] = 0.0f;
-                        }
-                        float f[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float v = __int2float_rn(int(r[8 * g + i]));
-                            v = __fmul_rn(v, sx);
-                            v = __fmul_rn(v, sw[i]);
-                            f[i] = __fadd_rn(v, b[i]);
-                        }
-                        uint4 out;
-                        out.x = bf16x2_rn(f[0], f[1]);
-                        out.y = bf16x2_rn(f[2], f[3]);
-                        out.z = bf16x2_rn(f[4], f[5]);
-                        out.w = bf16x2_rn(f[6], f[7]);
-                        *reinterpret_cast<uint4 *>(p.Y + int64_t(row) * p.N + n) = out;
-                    }
-                }
-            }
+            store_accumulators<kRaw>(p, tbase, mt * BM + quarter * 32 + lane, nt * BN);
             tc_fence_before();
             mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
             if (++acc == kAccBufs) {
@@ -322,26 +273,403 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
+// ---------------------------------------------------------------- 2-SM variant
+//
+// A cluster of 2 CTAs on the two SMs of a TPC computes 256 x 256 output tiles
+// with tcgen05.mma.cta_group::2 (M = 256 split 128/128 across the pair, N =
+// 256 with B split 128/128). Each CTA loads only its own 128 rows of A and its
+// 128 rows of B per K-block (32 KB per stage, 6 stages), so each SM streams
+// 64 bytes of operands per MMA clock instead of 96. The even CTA (leader)
+// issues the MMAs; the TMA loads of both CTAs complete on the leader's "full"
+// barrier; the leader's commits arrive on "empty" and "tmem_full" barriers of
+// both CTAs (tcgen05.commit multicast; no TMA multicast anywhere). Each CTA's
+// epilogue drains its own TMEM (its 128 rows x 256 columns) and arrives on
+// the leader's "tmem_empty" barrier.
+constexpr int kPairRows = 128;
+constexpr int kPairBM = 2 * kPairRows;
+constexpr int kPairBN = 256;
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = kPairRows * BK;
+constexpr int kPairStageBytes = 2 * kPairRows * BK;
+constexpr int kPairGroupM = 8;
+constexpr uint32_t kPairEpilogueWarps = 8;  // 4 per CTA, one arrive each
+
+struct alignas(8) PairControl {
+    uint64_t full[kPairStages];
+    uint64_t empty[kPairStages];
+    uint64_t tmem_full[kAccBufs];
+    uint64_t tmem_empty[kAccBufs];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kPairSmemBytes = 1024 + size_t(kPairStages) * kPairStageBytes + sizeof(PairControl);
+
+constexpr uint32_t kPairIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
+                                (uint32_t(kPairBN >> 3) << 17) | (uint32_t(kPairBM >> 4) << 24);
+
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t cluster_addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+template <bool kRaw>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PairControl *ctl = reinterpret_cast<PairControl *>(smem + size_t(kPairStages) * kPairStageBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int num_m = (p.M + kPairBM - 1) / kPairBM;
+    const int num_n = (p.N + kPairBN - 1) / kPairBN;
+    const int num_tiles = num_m * num_n;
+    const int nk = p.K / BK;
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(smem_u32(&ctl->full[s]), 1);
+            mbar_init(smem_u32(&ctl->empty[s]), 1);
+        }
+        for (int a = 0; a < kAccBufs; ++a) {
+            mbar_init(smem_u32(&ctl->tmem_full[a]), 1);
+            mbar_init(smem_u32(&ctl->tmem_empty[a]), kPairEpilogueWarps);
+        }
+        mbar_init(smem_u32(&ctl->drain), 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&ctl->tmem_base), kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM address written
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    volatile int *abort = &ctl->abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const uint32_t leader_full0 = mapa_shared(smem_u32(&ctl->full[0]), 0);
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_parity = 0;
+            bool ok = true;
+            if (!p.stall_producer) {
+                for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+                    int mt, nt;
+                    tile_coords(tile, num_m, num_n, mt, nt, kPairGroupM);
+                    const int a_row = mt * kPairBM + int(rank) * kPairRows;
+                    const int b_row = nt * kPairBN + int(rank) * kPairRows;
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, limit,
+                                               abort)) {
+                            ok = false;
+                            break;
+                        }
+                        if (leader)
+                            mbar_arrive_expect_tx(smem_u32(&ctl->full[stage]), 2 * kPairStageBytes);
+                        const uint32_t dst = smem_u32(smem + size_t(stage) * kPairStageBytes);
+                        const uint32_t bar = leader_full0 + uint32_t(8 * stage);
+                        tma_load_2d_pair(dst, &tmA, kb * BK, a_row, bar);
+                        tma_load_2d_pair(dst + kPairABytes, &tmB, kb * BK, b_row, bar);
+                        issued |= 1u << stage;
+                        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                        if (++stage == kPairStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            // The leader's full barriers count the bytes of both CTAs: once the
+            // last phase of every used stage has completed, no copy of either
+            // CTA is still in flight.
+            if (leader)
+                for (int s = 0; s < kPairStages; ++s)
+                    if (issued & (1u << s))
+                        if (!mbar_wait_bounded(smem_u32(&ctl->full[s]), (last_parity >> s) & 1u,
+                                               limit, nullptr))
+                            raise_timeout(abort, p.err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && leader) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+                if (!mbar_wait_bounded(smem_u32(&ctl->tmem_empty[acc]), acc_phase ^ 1u, limit,
+                                       abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + uint32_t(acc * kPairBN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_src = smem_u32(smem + size_t(stage) * kPairStageBytes);
+                    const uint64_t adesc = smem_desc_sw128(a_src);
+                    const uint64_t bdesc = smem_desc_sw128(a_src + kPairABytes);
+#pragma unroll
+                    for (int k = 0; k < BK / kUmmaK; ++k)
+                        umma_i8_pair(d, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), kPairIdesc,
+                                     (kb | k) != 0 ? 1u : 0u);
+                    umma_commit_pair_mc(smem_u32(&ctl->empty[stage]), 0x3);
+                    if (++stage == kPairStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(smem_u32(&ctl->tmem_full[acc]), 0x3);
+                if (++acc == kAccBufs) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            umma_commit_pair_mc(smem_u32(&ctl->drain), 0x1);
+            if (!mbar_wait_bounded(smem_u32(&ctl->drain), 0u, limit, nullptr))
+                raise_timeout(abort, p.err);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2-5, both CTAs)
+        const int quarter = warp & 3;
+        const uint32_t leader_tmem_empty0 = mapa_shared(smem_u32(&ctl->tmem_empty[0]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+            int mt, nt;
+            tile_coords(tile, num_m, num_n, mt, nt, kPairGroupM);
+            if (!mbar_wait_bounded(smem_u32(&ctl->tmem_full[acc]), acc_phase, limit, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase =
+                tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * kPairBN);
+            store_accumulators<kRaw>(p, tbase,
+                                     mt * kPairBM + int(rank) * kPairRows + quarter * 32 + lane,
+                                     nt * kPairBN);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tmem_empty0 + uint32_t(8 * acc));
+            if (++acc == kAccBufs) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (!ok) raise_timeout(abort, p.err);
+    }
+
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    // After a timeout, give copies that may still be in flight (into this
+    // CTA's shared memory, or onto the leader's barriers) time to land
+    // before the pair's shared memory is released.
+    const int peer_abort = ld_shared_cluster_s32(mapa_shared(smem_u32(&ctl->abort), rank ^ 1u));
+    if (*abort || peer_abort) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+    __syncwarp();
+    cluster_sync_all();
+}
+
+// Epilogue of one 256-column accumulator row block: this warp's 32 TMEM lanes
+// (rows), 8 chunks of 32 columns. tcgen05.ld is warp-collective, so every
+// lane takes part even when its row is past M; stores are clipped at M and N.
+template <bool kRaw>
+__device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t tbase, int row,
+                                                   int n_tile0) {
+    const bool row_ok = row < p.M;
+    float sx = 0.0f;
+    if (!kRaw && row_ok) sx = p.s_x[row];
+#pragma unroll 1
+    for (int c = 0; c < 256 / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
+        tmem_ld_wait();
+        const int n0 = n_tile0 + c * 32;
+        if (!row_ok) continue;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int n = n0 + 8 * g;
+            if (n >= p.N) break;
+            if (kRaw) {
+                int4 *dst = reinterpret_cast<int4 *>(p.acc + int64_t(row) * p.N + n);
+                dst[0] = make_int4(int(r[8 * g + 0]), int(r[8 * g + 1]), int(r[8 * g + 2]),
+                                   int(r[8 * g + 3]));
+                dst[1] = make_int4(int(r[8 * g + 4]), int(r[8 * g + 5]), int(r[8 * g + 6]),
+                                   int(r[8 * g + 7]));
+            } else {
+                const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
+                const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n + 4));
+                const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float b[8];
+                if (p.bias) {
+                    const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
+                    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        b[2 * i] = __uint_as_float(bw[i] << 16);
+                        b[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) b[i] = 0.0f;
+                }
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float v = __int2float_rn(int(r[8 * g + i]));
+                    v = __fmul_rn(v, sx);
+                    v = __fmul_rn(v, sw[i]);
+                    f[i] = __fadd_rn(v, b[i]);
+                }
+                uint4 out;
+                out.x = bf16x2_rn(f[0], f[1]);
+                out.y = bf16x2_rn(f[2], f[3]);
+                out.z = bf16x2_rn(f[4], f[5]);
+                out.w = bf16x2_rn(f[6], f[7]);
+                *reinterpret_cast<uint4 *>(p.Y + int64_t(row) * p.N + n) = out;
+            }
+        }
+    }
+}
+
 }  // namespace
 
-cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                           bool raw_i32, int num_sms, cudaStream_t stream) {
-    if (p.M <= 0 || p.N <= 0) return cudaSuccess;
-    const int num_tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
-    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_plan_mutex;
+int g_max_pairs[kMaxDevices];  // co-resident clusters of the pair kernel; 0 = not queried
+bool g_attrs_set[kMaxDevices];
+
+cudaError_t set_attributes() {
     cudaError_t e;
-    if (raw_i32) {
-        e = cudaFuncSetAttribute(gemm_i8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(kSmemBytes));
+    if ((e = cudaFuncSetAttribute(gemm_i8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(kSmemBytes))) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(gemm_i8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(kSmemBytes))) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(gemm_i8_pair_kernel<false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(kPairSmemBytes))) != cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(gemm_i8_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(kPairSmemBytes));
+}
+
+// Number of 2-CTA clusters of the pair kernel that fit on the device at once.
+cudaError_t max_active_pairs(int dev, int *out) {
+    std::lock_guard<std::mutex> lock(g_plan_mutex);
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!g_attrs_set[dev]) {
+        cudaError_t e = set_attributes();
         if (e != cudaSuccess) return e;
-        gemm_i8_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
-    } else {
-        e = cudaFuncSetAttribute(gemm_i8_kernel<false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-        if (e != cudaSuccess) return e;
-        gemm_i8_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+        g_attrs_set[dev] = true;
     }
-    return cudaGetLastError();
+    if (g_max_pairs[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kPairSmemBytes;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel<false>, &cfg);
+        if (e != cudaSuccess) return e;
+        g_max_pairs[dev] = n > 0 ? n : -1;
+    }
+    *out = g_max_pairs[dev] > 0 ? g_max_pairs[dev] : 0;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t plan_gemm(int M, int N, int num_sms, GemmPlan *plan) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int pairs = 0;
+    e = max_active_pairs(dev, &pairs);
+    if (e != cudaSuccess) return e;
+    plan->pair = M > kGemmBM && pairs > 0;
+    if (plan->pair) {
+        const int tiles = ((M + kPairBM - 1) / kPairBM) * ((N + kPairBN - 1) / kPairBN);
+        plan->b_box_rows = kPairRows;
+        plan->grid = 2 * (tiles < pairs ? tiles : pairs);
+    } else {
+        const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+        plan->b_box_rows = BN;
+        plan->grid = tiles < num_sms ? tiles : num_sms;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                           bool raw_i32, const GemmPlan &plan, cudaStream_t stream) {
+    if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+    if (!plan.pair) {
+        if (raw_i32)
+            gemm_i8_kernel<true><<<plan.grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+        else
+            gemm_i8_kernel<false><<<plan.grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(plan.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (raw_i32) return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<true>, tmA, tmB, p);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<false>, tmA, tmB, p);
 }
 
 }  // namespace ck

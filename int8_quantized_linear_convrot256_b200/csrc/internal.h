@@ -36,7 +36,19 @@ constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
 
+// Which GEMM variant runs for an M x N output, and its grid: the 2-SM
+// (cta_group::2, 256 x 256 tiles per CTA pair) kernel when M > 128 and pairs
+// fit on the device, else the 1-SM 128 x 256 kernel. A's TMA box is always
+// kGemmBM rows; B's box is b_box_rows rows.
+struct GemmPlan {
+    bool pair;
+    int b_box_rows;
+    int grid;
+};
+
+cudaError_t plan_gemm(int M, int N, int num_sms, GemmPlan *plan);
+
 cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                           bool raw_i32, int num_sms, cudaStream_t stream);
+                           bool raw_i32, const GemmPlan &plan, cudaStream_t stream);
 
 }  // namespace ck
