@@ -144,8 +144,8 @@ ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8
     DeviceState *st = nullptr;
     s = device_state(&st);
     if (s != CK_OK) return s;
-    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, Qx, s_x,
-                                               reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, Qx, s_x, st->err,
+                                               st->num_sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
@@ -228,7 +228,7 @@ ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const 
     float *s_x = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                            round256(size_t(M) * size_t(K)));
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, true, Qx, s_x, cs);
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, true, Qx, s_x, st->err, st->num_sms, cs);
     if (e != cudaSuccess) return CK_ERR_CUDA;
     return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
 }

@@ -6,37 +6,51 @@
 // FP32 row scales; ComfyUI-AppleSilicon-FP8 README row 17: rotate online,
 // then quantise per row):
 //   every 256-block of a row -> 8 fp32 butterfly stages h = 1, 2, ..., 128,
-//   then * 1/16; s = absmax(row) / 127; q = round-half-even(y / s) clamped to
-//   [-127, 127]; a zero row gives s = 0 and q = 0.
+//   then * 1/16 (y); s = absmax(y) / 127; q = round-half-even(y / s) clamped
+//   to [-127, 127]; a zero row gives s = 0 and q = 0.
 //
 // Design (HBM-bound: 2 B read + 1 B written per element, 4 B per row):
 //  * One quad (4 consecutive lanes) owns one 256-block; each lane keeps 64
-//    values in registers. Element e of the block sits in lane (e >> 3) & 3 of
-//    the quad, register ((e >> 5) << 3) | (e & 7). Lane t therefore loads 8
-//    contiguous values at e = 8t + 32j (j = 0..7): 16-byte loads, and each
-//    quad reads 64 contiguous bytes per load instruction.
-//  * Butterfly stages on element bits 0, 1, 2, 5, 6, 7 pair registers of the
-//    same lane; stages on bits 3 and 4 (h = 8, 16) pair lanes t and t ^ 1,
-//    t ^ 2 of the quad through one shuffle per value. Stages run in the order
-//    h = 1, 2, 4, ..., 128 and each is one IEEE add or subtract per value,
-//    so the result is bit-identical to the sequential definition.
-//  * The whole row stays in registers of one CTA (rows_per_cta rows of
-//    K/256 quads each); the row absmax is reduced through a shared-memory
-//    atomicMax on the fp32 bit pattern (non-negative floats order like their
-//    bits), so X is read from HBM exactly once. K > 32768 takes a two-pass
-//    variant that re-reads the (L2-resident) row instead.
+//    values in registers as 32 float2 pairs. Element e of the block sits in
+//    lane (e >> 3) & 3 of the quad; within the lane, pair j holds elements
+//    with e bit 0 = 0/1, j bit 0 = e bit 1, bit 1 = e bit 2, bits 2-4 = e
+//    bits 5-7. Lane t therefore loads 8 contiguous values at e = 8t + 32i
+//    (i = 0..7): 16-byte loads, each quad reading 64 contiguous bytes.
+//  * Butterfly stages h = 1, 2, ..., 128 run in that order; each is one IEEE
+//    add or subtract per value (a - c as fma(c, -1, a): one rounding of the
+//    exact difference). h = 1 pairs the two halves of a float2 (scalar ops);
+//    h = 2, 4, 32, 64, 128 pair whole float2s (packed add.f32x2 / fma.f32x2);
+//    h = 8, 16 pair lanes t ^ 1, t ^ 2 of the quad through shuffles and one
+//    packed fma(+-1, v, partner). Results are bit-identical to the
+//    sequential definition.
+//  * The exact * 1/16 is folded into the scale: with z = 16 y (the butterfly
+//    output), amax_y = amax_z / 16 and s = fl(amax_z / 127) / 16 exactly, and
+//    fl(y / s) = fl(z / fl(amax_z / 127)), as long as nothing is subnormal:
+//    rows with amax_z >= 2^-93 take this path (values with |z| < 2^-122, whose
+//    y would be subnormal, give code 0 either way because |z / s| < 2^-22).
+//    Smaller rows follow the definition step by step (y = fl(z / 16), then the
+//    exact division).
 //  * Division: q needs round-half-even of the IEEE quotient fl(y / s). With
-//    r = fl(1/s) and t = fl(y * r), |t - y/s| < 2^-16 and |fl(y/s) - y/s| <=
-//    2^-17 when |y/s| < 128 (always: |y| <= absmax and s = fl(absmax/127)).
-//    So if t is farther than 2^-14 from every half-integer, rint(t) equals
-//    rint(fl(y / s)). Values closer than that (about 1 in 8000) and rows with
-//    s < 2^-120 take the exact path rint(__fdiv_rn(y, s)). rint(t) itself uses
-//    t + 1.5 * 2^23, whose low byte is then the two's-complement code; no
-//    clamp is needed on the fast path because |y / s| <= 127 * (1 + 2^-23).
+//    d the divisor, r = fl(1/d) and t = fl(z * r), |t - z/d| < 2^-16 and
+//    |fl(z/d) - z/d| <= 2^-17 because |z/d| <= 127 (1 + 2^-23). So if t is
+//    farther than 2^-14 from every half-integer, rint(t) = rint(fl(z/d)).
+//    Groups of 8 values that contain a closer one (about 1 in 1000 groups)
+//    take rint(__fdiv_rn(z, d)). rint(t) itself is t + 1.5 * 2^23, whose low
+//    byte is the two's-complement code; no clamp is needed on that path.
+//  * The whole row stays in registers of one CTA (rows_per_cta rows x K/256
+//    quads); the row absmax is reduced through a shared-memory atomicMax on
+//    the fp32 bit pattern, so X is read from HBM exactly once. BF16 rows are
+//    staged into shared memory by 1-D bulk copies (cp.async.bulk) one row
+//    group ahead of the compute, in a persistent grid, so HBM always has a
+//    full row group per CTA in flight. K > 32768 takes a two-pass variant
+//    (rows re-read from L2); fp32 weights (offline) take direct loads.
 //  * No FMA contraction: every operation is an explicit _rn intrinsic.
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "ck_device.cuh"
 #include "internal.h"
@@ -45,97 +59,174 @@ namespace ck {
 namespace {
 
 constexpr int kBlock = 256;
-constexpr int kVals = 64;  // values of a block held by one lane
+constexpr int kPairs = 32;  // float2 pairs per lane per block (64 values)
 constexpr int kMaxThreads = 512;
 constexpr int kMaxRowsPerCta = kMaxThreads / 4;
-constexpr int kTwoPassQuads = 128;  // quads per row in the two-pass variant
-constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23
-constexpr float kNearHalf = 0.49993896484375f;     // 0.5 - 2^-14
+constexpr int kTwoPassQuads = 128;                   // quads per row in the two-pass variant
+constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
+constexpr float kNearHalf = 0.49993896484375f;       // 0.5 - 2^-14
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
+constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
+constexpr size_t kBulkSmemBudget = 112 * 1024;       // per-CTA staging budget (2 buffers)
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
-    return __ldcs(reinterpret_cast<const uint4 *>(p));
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b with one rounding: b * (-1) is exact, then the sum is rounded once.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
-// Load lane t's 64 values of one block: base points at element 8t of the block.
-__device__ __forceinline__ void load_block(const uint16_t *base, float (&v)[kVals]) {
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float2 widen_bf16x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// Lane t's 64 values of one block; base points at element 8t of the block.
+__device__ __forceinline__ void load_block(const uint16_t *base, float2 (&P)[kPairs]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint4 u = ld_stream_v4(base + 32 * j);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int i = 0; i < 8; ++i) {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(base + 32 * i));
+        P[4 * i + 0] = widen_bf16x2(u.x);
+        P[4 * i + 1] = widen_bf16x2(u.y);
+        P[4 * i + 2] = widen_bf16x2(u.z);
+        P[4 * i + 3] = widen_bf16x2(u.w);
+    }
+}
+
+__device__ __forceinline__ void load_block(const float *base, float2 (&P)[kPairs]) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[8 * j + 2 * i] = __uint_as_float(w[i] << 16);
-            v[8 * j + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int i = 0; i < 8; ++i) {
+        const float4 a = __ldcs(reinterpret_cast<const float4 *>(base + 32 * i));
+        const float4 b = __ldcs(reinterpret_cast<const float4 *>(base + 32 * i + 4));
+        P[4 * i + 0] = make_float2(a.x, a.y);
+        P[4 * i + 1] = make_float2(a.z, a.w);
+        P[4 * i + 2] = make_float2(b.x, b.y);
+        P[4 * i + 3] = make_float2(b.z, b.w);
+    }
+}
+
+__device__ __forceinline__ void load_block_smem(uint32_t saddr, float2 (&P)[kPairs]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t x, y, z, w;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                     : "r"(saddr + 64u * i));
+        P[4 * i + 0] = widen_bf16x2(x);
+        P[4 * i + 1] = widen_bf16x2(y);
+        P[4 * i + 2] = widen_bf16x2(z);
+        P[4 * i + 3] = widen_bf16x2(w);
+    }
+}
+
+__device__ __forceinline__ void zero_block(float2 (&P)[kPairs]) {
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) P[j] = make_float2(0.0f, 0.0f);
+}
+
+// h = 1: the two halves of every pair.
+__device__ __forceinline__ void stage_in_pair(float2 (&P)[kPairs]) {
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        const float a = P[j].x;
+        const float c = P[j].y;
+        P[j] = make_float2(__fadd_rn(a, c), __fsub_rn(a, c));
+    }
+}
+
+// Pairs j and j + J (J = 1, 2, 4, 8, 16).
+template <int J>
+__device__ __forceinline__ void stage_pairs(float2 (&P)[kPairs]) {
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        if ((j & J) == 0) {
+            const float2 a = P[j];
+            const float2 c = P[j + J];
+            P[j] = add2(a, c);
+            P[j + J] = sub2(a, c);
         }
     }
 }
 
-__device__ __forceinline__ void load_block(const float *base, float (&v)[kVals]) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float4 a = __ldcs(reinterpret_cast<const float4 *>(base + 32 * j));
-        const float4 b = __ldcs(reinterpret_cast<const float4 *>(base + 32 * j + 4));
-        v[8 * j + 0] = a.x; v[8 * j + 1] = a.y; v[8 * j + 2] = a.z; v[8 * j + 3] = a.w;
-        v[8 * j + 4] = b.x; v[8 * j + 5] = b.y; v[8 * j + 6] = b.z; v[8 * j + 7] = b.w;
-    }
-}
-
-// Butterfly between registers r and r + R (R = 1, 2, 4, 8, 16, 32).
-template <int R>
-__device__ __forceinline__ void stage_regs(float (&v)[kVals]) {
-#pragma unroll
-    for (int r = 0; r < kVals; ++r) {
-        if ((r & R) == 0) {
-            const float a = v[r];
-            const float c = v[r + R];
-            v[r] = __fadd_rn(a, c);
-            v[r + R] = __fsub_rn(a, c);
-        }
-    }
-}
-
-// Butterfly between lanes t and t ^ L of the quad (L = 1, 2). The lane with
-// the bit clear holds a and computes a + c; the other holds c and computes
-// a - c = fma(-1, c, a), a single rounding, the same value as the subtraction.
+// Lanes t and t ^ L of the quad (L = 1, 2): the lane with the bit clear holds
+// a and computes a + c; the other holds c and computes a - c = fma(-1, c, a).
 template <int L>
-__device__ __forceinline__ void stage_lanes(float (&v)[kVals], int t) {
-    const float sg = (t & L) ? -1.0f : 1.0f;
+__device__ __forceinline__ void stage_lanes(float2 (&P)[kPairs], int t) {
+    const float s = (t & L) ? -1.0f : 1.0f;
+    const float2 sg = make_float2(s, s);
 #pragma unroll
-    for (int r = 0; r < kVals; ++r) {
-        const float p = __shfl_xor_sync(0xFFFFFFFFu, v[r], L);
-        v[r] = __fmaf_rn(sg, v[r], p);
+    for (int j = 0; j < kPairs; ++j) {
+        const float2 p = make_float2(__shfl_xor_sync(0xFFFFFFFFu, P[j].x, L),
+                                     __shfl_xor_sync(0xFFFFFFFFu, P[j].y, L));
+        P[j] = __ffma2_rn(sg, P[j], p);
     }
 }
 
-// ConvRot256 of the block spread over the quad: stages h = 1..128 in order.
-__device__ __forceinline__ void rotate_block(float (&v)[kVals], int t) {
-    stage_regs<1>(v);    // h = 1
-    stage_regs<2>(v);    // h = 2
-    stage_regs<4>(v);    // h = 4
-    stage_lanes<1>(v, t);  // h = 8
-    stage_lanes<2>(v, t);  // h = 16
-    stage_regs<8>(v);    // h = 32
-    stage_regs<16>(v);   // h = 64
-    stage_regs<32>(v);   // h = 128
-#pragma unroll
-    for (int r = 0; r < kVals; ++r) v[r] = __fmul_rn(v[r], 0.0625f);
+// The 8 butterfly stages of ConvRot256, without the final * 1/16 (z = 16 y).
+__device__ __forceinline__ void butterflies(float2 (&P)[kPairs], int t) {
+    stage_in_pair(P);    // h = 1
+    stage_pairs<1>(P);   // h = 2
+    stage_pairs<2>(P);   // h = 4
+    stage_lanes<1>(P, t);  // h = 8
+    stage_lanes<2>(P, t);  // h = 16
+    stage_pairs<4>(P);   // h = 32
+    stage_pairs<8>(P);   // h = 64
+    stage_pairs<16>(P);  // h = 128
 }
 
-__device__ __forceinline__ float quad_absmax(const float (&v)[kVals]) {
+__device__ __forceinline__ float quad_absmax(const float2 (&P)[kPairs]) {
     float m = 0.0f;
 #pragma unroll
-    for (int r = 0; r < kVals; ++r) m = fmaxf(m, fabsf(v[r]));
+    for (int j = 0; j < kPairs; ++j) m = max3(m, fabsf(P[j].x), fabsf(P[j].y));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     return m;
 }
 
-// Exact path: the code as the definition states it, returned as the bit
+// How a row is quantised, from its absmax (of z for rotated rows).
+struct RowQuant {
+    float s;      // the row scale to store (the definition's s)
+    float div;    // divisor applied to the held values
+    float rc;     // fl(1 / div) when fast
+    bool fast;    // reciprocal path with the near-half-integer fallback
+    bool scale16; // exact path must first form y = fl(z / 16)
+};
+
+template <bool kRotate>
+__device__ __forceinline__ RowQuant row_quant(float amax) {
+    RowQuant r;
+    if (kRotate) {
+        if (amax >= kMinFoldAmax) {
+            r.div = __fdiv_rn(amax, 127.0f);
+            r.s = __fmul_rn(r.div, 0.0625f);
+            r.fast = true;
+            r.scale16 = false;
+        } else {
+            r.s = __fdiv_rn(__fmul_rn(amax, 0.0625f), 127.0f);
+            r.div = r.s;
+            r.fast = false;
+            r.scale16 = true;
+        }
+    } else {
+        r.s = __fdiv_rn(amax, 127.0f);
+        r.div = r.s;
+        r.fast = r.s >= kMinFastScale;
+        r.scale16 = false;
+    }
+    r.rc = r.fast ? __frcp_rn(r.div) : 0.0f;
+    return r;
+}
+
+// Exact path for one value, as the definition states it; returns the bit
 // pattern of 1.5 * 2^23 + q (low byte = q in two's complement).
-__device__ __forceinline__ uint32_t code_exact(float y, float s) {
-    if (s == 0.0f) return __float_as_uint(kMagic);
-    float q = rintf(__fdiv_rn(y, s));
+__device__ __forceinline__ uint32_t code_exact(float z, const RowQuant &rq) {
+    if (rq.div == 0.0f) return __float_as_uint(kMagic);
+    const float y = rq.scale16 ? __fmul_rn(z, 0.0625f) : z;
+    float q = rintf(__fdiv_rn(y, rq.div));
     q = fminf(fmaxf(q, -127.0f), 127.0f);
     return __float_as_uint(__fadd_rn(q, kMagic));
 }
@@ -146,35 +237,66 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
     return __byte_perm(ab, cd, 0x5410);
 }
 
-// Quantise lane t's 64 values with row scale s and store the codes: register
-// group j holds elements 8t + 32j .. +7, stored as 8 contiguous bytes.
-__device__ __forceinline__ void quantize_store(const float (&v)[kVals], float s, int8_t *qbase) {
-    const bool fast = s >= kMinFastScale;
-    const float rc = fast ? __frcp_rn(s) : 0.0f;
+// Quantise lane t's 64 values and store the codes: group i (pairs 4i..4i+3)
+// holds elements 8t + 32i .. +7, stored as 8 contiguous bytes. The fast path
+// stores every group without branching and records which groups hold a value
+// near a half-integer; those (rare) groups are then recomputed exactly and
+// stored again.
+__device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int i,
+                                                  const RowQuant &rq, int8_t *qbase) {
+    uint32_t u[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int k = 0; k < 4; ++k) {
+        u[2 * k] = code_exact(P[4 * i + k].x, rq);
+        u[2 * k + 1] = code_exact(P[4 * i + k].y, rq);
+    }
+    uint2 out;
+    out.x = pack4(u[0], u[1], u[2], u[3]);
+    out.y = pack4(u[4], u[5], u[6], u[7]);
+    *reinterpret_cast<uint2 *>(qbase + 32 * i) = out;
+}
+
+__device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const RowQuant &rq,
+                                               int8_t *qbase) {
+    if (!rq.fast) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) store_group_exact(P, i, rq, qbase);
+        return;
+    }
+    const float2 rc2 = make_float2(rq.rc, rq.rc);
+    const float2 magic2 = make_float2(kMagic, kMagic);
+    const float2 nmagic2 = make_float2(-kMagic, -kMagic);
+    uint32_t redo = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
         uint32_t u[8];
         float dmax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float t = __fmul_rn(v[8 * j + i], rc);
-            const float m = __fadd_rn(t, kMagic);
-            const float rt = __fsub_rn(m, kMagic);
-            dmax = fmaxf(dmax, fabsf(__fsub_rn(t, rt)));
-            u[i] = __float_as_uint(m);
+        for (int k = 0; k < 4; ++k) {
+            const float2 t = __fmul2_rn(P[4 * i + k], rc2);
+            const float2 m = add2(t, magic2);
+            const float2 rt = add2(m, nmagic2);
+            const float2 d = sub2(t, rt);
+            dmax = max3(dmax, fabsf(d.x), fabsf(d.y));
+            u[2 * k] = __float_as_uint(m.x);
+            u[2 * k + 1] = __float_as_uint(m.y);
         }
-        if (!fast || dmax >= kNearHalf) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = code_exact(v[8 * j + i], s);
-        }
+        redo |= uint32_t(dmax >= kNearHalf) << i;
         uint2 out;
         out.x = pack4(u[0], u[1], u[2], u[3]);
         out.y = pack4(u[4], u[5], u[6], u[7]);
-        *reinterpret_cast<uint2 *>(qbase + 32 * j) = out;
+        *reinterpret_cast<uint2 *>(qbase + 32 * i) = out;
+    }
+    if (redo) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (redo & (1u << i)) store_group_exact(P, i, rq, qbase);
     }
 }
 
-// Single pass: CTA = rows_per_cta rows x (K/256) quads, whole rows in registers.
+// ------------------------------------------------------------------ kernels
+
+// Single pass with direct loads: CTA = rows_per_cta rows x (K/256) quads.
 template <bool kRotate, typename TIn>
 __global__ void __launch_bounds__(kMaxThreads, 1)
 quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
@@ -191,24 +313,116 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     const int col0 = blk * kBlock + 8 * t;
 
     if (tid < rows_per_cta) s_amax[tid] = 0u;
-
-    float v[kVals];
-    if (active) {
-        load_block(X + row * ldx + col0, v);
-    } else {
-#pragma unroll
-        for (int r = 0; r < kVals; ++r) v[r] = 0.0f;
-    }
-    if (kRotate) rotate_block(v, t);
-    const float m = quad_absmax(v);
+    float2 P[kPairs];
+    if (active)
+        load_block(X + row * ldx + col0, P);
+    else
+        zero_block(P);
+    if (kRotate) butterflies(P, t);
+    const float m = quad_absmax(P);
     __syncthreads();  // s_amax initialised
     if (active && t == 0) atomicMax(&s_amax[row_local], __float_as_uint(m));
     __syncthreads();
     if (!active) return;
-    const float amax = __uint_as_float(s_amax[row_local]);
-    const float s = __fdiv_rn(amax, 127.0f);
-    if (blk == 0 && t == 0) S[row] = s;
-    quantize_store(v, s, Q + row * static_cast<int64_t>(K) + col0);
+    const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax[row_local]));
+    if (blk == 0 && t == 0) S[row] = rq.s;
+    quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0);
+}
+
+// Persistent single pass for BF16 rows: row groups are staged into shared
+// memory with cp.async.bulk two groups ahead (2 buffers). One CTA barrier per
+// group: after it, every thread has read its values out of the buffer (so the
+// buffer can be refilled) and the row absmax is complete. The absmax slots are
+// triple-buffered so a slot is cleared one full barrier before its next use.
+template <bool kRotate>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
+                       int rows_per_cta, int8_t *__restrict__ Q, float *__restrict__ S,
+                       unsigned *err, uint64_t limit_ns) {
+    extern __shared__ __align__(128) uint8_t stage_raw[];
+    __shared__ unsigned s_amax[3][kMaxRowsPerCta];
+    __shared__ __align__(8) uint64_t full[2];
+    const int tid = threadIdx.x;
+    const int t = tid & 3;
+    const int quad = tid >> 2;
+    const int nb = K >> 8;
+    const int R = rows_per_cta;
+    const int row_local = quad / nb;
+    const int blk = quad - row_local * nb;
+    const int col0 = blk * kBlock + 8 * t;
+    const int64_t ngroups = (M + R - 1) / R;
+    const uint32_t row_bytes = uint32_t(K) * 2u;
+    const uint32_t buf0 = smem_u32(stage_raw);
+    const uint32_t buf_bytes = uint32_t(R) * row_bytes;
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 3 * kMaxRowsPerCta; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
+    __syncthreads();
+
+    // Thread 0: stage the rows of group g into buffer b.
+    auto issue = [&](int64_t g, int b) {
+        const int64_t r0 = g * R;
+        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
+        const uint32_t bar = smem_u32(&full[b]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
+        for (int r = 0; r < n; ++r) {
+            const uint16_t *src = X + (r0 + r) * ldx;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(buf0 + uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes),
+                "l"(reinterpret_cast<uint64_t>(src)), "r"(row_bytes), "r"(bar)
+                : "memory");
+        }
+    };
+
+    const int64_t g0 = blockIdx.x;
+    const int64_t step = gridDim.x;
+    if (tid == 0) {
+        if (g0 < ngroups) issue(g0, 0);
+        if (g0 + step < ngroups) issue(g0 + step, 1);
+    }
+    int slot = 0;  // i % 3
+    for (int i = 0; g0 + i * step < ngroups; ++i) {
+        const int64_t g = g0 + i * step;
+        const int b = i & 1;
+        const bool ok = mbar_wait_bounded(smem_u32(&full[b]), uint32_t(i >> 1) & 1u, limit_ns,
+                                          nullptr);
+        const int64_t row = g * R + row_local;
+        const bool active = ok && row_local < R && row < M;
+        float2 P[kPairs];
+        if (active)
+            load_block_smem(buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
+                                uint32_t(col0) * 2u,
+                            P);
+        else
+            zero_block(P);
+        if (kRotate) butterflies(P, t);
+        const float m = quad_absmax(P);
+        if (active && t == 0) atomicMax(&s_amax[slot][row_local], __float_as_uint(m));
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicMax(err, kDevErrTimeout);
+            // let a late copy land before the CTA's shared memory is released
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000ull) {
+            }
+            break;
+        }
+        // Buffer b has been read by every thread: refill it two groups ahead.
+        if (tid == 0 && g + 2 * step < ngroups) issue(g + 2 * step, b);
+        const int clear = slot == 0 ? 2 : slot - 1;  // (i + 2) % 3
+        if (tid < R) s_amax[clear][tid] = 0u;
+        if (active) {
+            const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax[slot][row_local]));
+            if (blk == 0 && t == 0) S[row] = rq.s;
+            quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0);
+        }
+        slot = slot == 2 ? 0 : slot + 1;
+    }
 }
 
 // Two passes for long rows (K > 32768): one CTA per row, 128 quads; pass 1
@@ -229,44 +443,39 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
     float m = 0.0f;
     for (int b0 = 0; b0 < nb; b0 += kTwoPassQuads) {
         const int blk = b0 + quad;
-        float v[kVals];
-        if (blk < nb) {
-            load_block(xrow + blk * kBlock + 8 * t, v);
-        } else {
-#pragma unroll
-            for (int r = 0; r < kVals; ++r) v[r] = 0.0f;
-        }
-        if (kRotate) rotate_block(v, t);
-        m = fmaxf(m, quad_absmax(v));
+        float2 P[kPairs];
+        if (blk < nb)
+            load_block(xrow + blk * kBlock + 8 * t, P);
+        else
+            zero_block(P);
+        if (kRotate) butterflies(P, t);
+        m = fmaxf(m, quad_absmax(P));
     }
     __syncthreads();
     if (t == 0) atomicMax(&s_amax, __float_as_uint(m));
     __syncthreads();
-    const float amax = __uint_as_float(s_amax);
-    const float s = __fdiv_rn(amax, 127.0f);
-    if (tid == 0) S[row] = s;
+    const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax));
+    if (tid == 0) S[row] = rq.s;
     for (int b0 = 0; b0 < nb; b0 += kTwoPassQuads) {
         const int blk = b0 + quad;
-        float v[kVals];
-        if (blk < nb) {
-            load_block(xrow + blk * kBlock + 8 * t, v);
-        } else {
-#pragma unroll
-            for (int r = 0; r < kVals; ++r) v[r] = 0.0f;
-        }
-        if (kRotate) rotate_block(v, t);
-        if (blk < nb) quantize_store(v, s, Q + row * static_cast<int64_t>(K) + blk * kBlock + 8 * t);
+        float2 P[kPairs];
+        if (blk < nb)
+            load_block(xrow + blk * kBlock + 8 * t, P);
+        else
+            zero_block(P);
+        if (kRotate) butterflies(P, t);
+        if (blk < nb) quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + blk * kBlock + 8 * t);
     }
 }
 
-// Rows per CTA for the single-pass kernel: the CTA has 4 * nb * R useful
-// threads rounded up to whole warps; pick the R with the fewest idle lanes,
-// then the CTA size closest to 256 threads.
-int pick_rows_per_cta(int nb, int *threads_out) {
+// Rows per CTA: the CTA has 4 * nb * R useful threads rounded up to whole
+// warps; pick the R with the fewest idle lanes, then the CTA size closest to
+// 256 threads, with at most max_rows rows.
+int pick_rows_per_cta(int nb, int max_rows, int *threads_out) {
     int best_r = 1, best_t = ((4 * nb + 31) / 32) * 32;
     double best_waste = 2.0;
     int best_dist = 1 << 30;
-    for (int r = 1; 4 * nb * r <= kMaxThreads; ++r) {
+    for (int r = 1; r <= max_rows && 4 * nb * r <= kMaxThreads; ++r) {
         const int used = 4 * nb * r;
         const int threads = ((used + 31) / 32) * 32;
         if (threads > kMaxThreads) break;
@@ -283,14 +492,65 @@ int pick_rows_per_cta(int nb, int *threads_out) {
     return best_r;
 }
 
+std::mutex g_occ_mutex;
+// (device, rotate, threads, smem) -> CTAs of the bulk kernel per SM
+std::map<std::tuple<int, int, int, size_t>, int> g_bulk_occupancy;
+
+template <bool kRotate>
+cudaError_t bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
+    std::lock_guard<std::mutex> lock(g_occ_mutex);
+    const auto key = std::make_tuple(dev, kRotate ? 1 : 0, threads, smem);
+    auto it = g_bulk_occupancy.find(key);
+    if (it != g_bulk_occupancy.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel<kRotate>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(kBulkSmemBudget));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_bulk_kernel<kRotate>,
+                                                      threads, smem);
+    if (e != cudaSuccess) return e;
+    g_bulk_occupancy[key] = per_sm;
+    *out = per_sm;
+    return cudaSuccess;
+}
+
+template <bool kRotate>
+cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
+                        unsigned *err, int num_sms, cudaStream_t stream, bool *launched) {
+    *launched = false;
+    const int nb = static_cast<int>(K / kBlock);
+    const int max_rows = static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2));
+    if (max_rows < 1 || 4 * nb > kMaxThreads) return cudaSuccess;
+    int threads = 0;
+    const int rows = pick_rows_per_cta(nb, max_rows, &threads);
+    const size_t smem = 2 * size_t(rows) * size_t(K) * 2;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = bulk_blocks_per_sm<kRotate>(dev, threads, smem, &per_sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaSuccess;
+    const int64_t groups = (M + rows - 1) / rows;
+    const int64_t cap = int64_t(per_sm) * num_sms;
+    const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
+    quant_rows_bulk_kernel<kRotate><<<grid, threads, smem, stream>>>(
+        X, M, static_cast<int>(K), ldx, rows, Q, S, err, kDefaultWaitLimitNs);
+    *launched = true;
+    return cudaGetLastError();
+}
+
 template <bool kRotate, typename TIn>
-cudaError_t launch_rows(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
-                        cudaStream_t stream) {
-    if (M <= 0) return cudaSuccess;
+cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
+                          cudaStream_t stream) {
     const int nb = static_cast<int>(K / kBlock);
     if (4 * nb <= kMaxThreads) {
         int threads = 0;
-        const int rows = pick_rows_per_cta(nb, &threads);
+        const int rows = pick_rows_per_cta(nb, kMaxRowsPerCta, &threads);
         const int64_t grid = (M + rows - 1) / rows;
         quant_rows_kernel<kRotate, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
             X, M, static_cast<int>(K), ldx, rows, Q, S);
@@ -305,14 +565,22 @@ cudaError_t launch_rows(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_t 
 }  // namespace
 
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   bool rotate, int8_t *Q, float *S, cudaStream_t stream) {
-    return rotate ? launch_rows<true>(X, M, K, ldx, Q, S, stream)
-                  : launch_rows<false>(X, M, K, ldx, Q, S, stream);
+                                   bool rotate, int8_t *Q, float *S, unsigned *err, int num_sms,
+                                   cudaStream_t stream) {
+    if (M <= 0) return cudaSuccess;
+    bool launched = false;
+    cudaError_t e =
+        rotate ? launch_bulk<true>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched)
+               : launch_bulk<false>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+    return rotate ? launch_direct<true>(X, M, K, ldx, Q, S, stream)
+                  : launch_direct<false>(X, M, K, ldx, Q, S, stream);
 }
 
 cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,
                                   cudaStream_t stream) {
-    return launch_rows<true>(W, N, K, K, Q, S, stream);
+    if (N <= 0) return cudaSuccess;
+    return launch_direct<true>(W, N, K, K, Q, S, stream);
 }
 
 }  // namespace ck
