@@ -59,6 +59,31 @@ def peaks():
                 "source": "fallback"}
 
 
+# ---------------------------------------------------------------- ranks
+
+
+def shard_rows(M: int, rank: int, world: int):
+    """Contiguous, balanced rows [lo, hi) of an M-row batch owned by `rank`
+    when the rows are split over `world` ranks (strong scaling). Rows of the
+    linear are independent, so no collective is needed on the data path."""
+    base, rem = divmod(M, world)
+    lo = rank * base + min(rank, rem)
+    return lo, lo + base + (1 if rank < rem else 0)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (timings are
+    reported as the slowest rank's). A no-op without a process group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -193,10 +218,12 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
-def config_dict(cfg, world):
+def config_dict(cfg, world, scaling="weak"):
+    par = (f"replicas x{world}: every rank runs the whole batch" if scaling == "weak"
+           else f"rows split over {world} ranks")
     return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "seed": cfg.seed,
             "x_dist": cfg.x_dist, "outlier_channels": cfg.n_outlier,
-            "parallelism": f"replicas x{world} (rows independent, no collective)",
+            "parallelism": par + " (rows are independent: no collective on the data path)",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); X is also larger than L2",
             "weights": "rotated + quantised once before timing (offline)"}
 
@@ -215,11 +242,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     P = peaks()
 
     X, W, bias = workloads.make_inputs(cfg)
+    if args.scaling == "strong":
+        lo, hi = shard_rows(cfg.M, rank, world)
+        X = X[lo:hi].contiguous()
     Xd = X.to(dev)
     bd = bias.to(dev)
     Qw, s_w = ck.rotate_quant_weight(W.to(dev))
     Wcpu = W
-    M, N, K = cfg.M, cfg.N, cfg.K
+    M, N, K = X.shape[0], cfg.N, cfg.K
     Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
     s_x = torch.empty((M,), dtype=torch.float32, device=dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -267,18 +297,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     ms_step = sum(s_ms) / len(s_ms)
     ms_q = sum(q_ms) / len(q_ms)
     ms_g = sum(g_ms) / len(g_ms)
-    if world > 1:
-        t = torch.tensor([ms_step, ms_q, ms_g], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_q, ms_g = t.tolist()
+    ms_step, ms_q, ms_g = max_over_ranks([ms_step, ms_q, ms_g], dev)
 
     # ---- end to end through the public composite call, host buffers
     if args.no_e2e:
         ms_e2e = float("nan")
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
-    ops = 2.0 * M * N * K
-    return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, ops,
+    return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
                   clocks, t_wall0, t_wall1)
 
 
@@ -310,18 +336,18 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = t.item()
-    return ms_e2e
+    return max_over_ranks([ms_e2e], dev)[0]
 
 
-def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, ops, clocks,
+def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
            t_wall0, t_wall1):
-    M, N, K = cfg.M, cfg.N, cfg.K
-    value = world * ops / (ms_step / 1e3) / 1e12
-    e2e_value = world * ops / (ms_e2e / 1e3) / 1e12
+    # per-rank work: the full batch (weak, replicas) or this rank's row shard
+    # (strong); the job's total is world x per-rank (weak) or the whole batch
+    M, N, K = X.shape[0], cfg.N, cfg.K
+    ops = 2.0 * M * N * K
+    job_ops = world * ops if args.scaling == "weak" else 2.0 * cfg.M * N * K
+    value = job_ops / (ms_step / 1e3) / 1e12
+    e2e_value = job_ops / (ms_e2e / 1e3) / 1e12
     gemm_tops = ops / (ms_g / 1e3) / 1e12
     q_bytes = 3.0 * M * K + 4.0 * M
     q_gbs = q_bytes / (ms_q / 1e3) / 1e9
@@ -353,10 +379,10 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": (value / world) / (ops / (page_ms / 1e3) / 1e12) if page_ms else None,
+            "scaling": args.scaling,
+            "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
             "dtype": "int8", "data": "synthetic", "impl": "ours",
-            "config": config_dict(cfg, world),
+            "config": config_dict(cfg, world, args.scaling),
             "roofline": {"kernel": "gemm_i8_kernel (tcgen05 kind::i8 + fused epilogue)",
                          "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
@@ -385,6 +411,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=workloads.HEADLINE.name, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="weak: every rank runs the whole batch (replicas); strong: the "
+                         "batch's rows are split over the ranks")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
