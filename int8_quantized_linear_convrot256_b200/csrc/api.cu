@@ -95,6 +95,20 @@ ck_status make_tmap_i8(CUtensorMap *tm, const void *base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS ? CK_OK : CK_ERR_CUDA;
 }
 
+// Row-major [M, N] bf16 output, box = 32 columns x 32 rows, 64-byte swizzle.
+ck_status make_tmap_y(CUtensorMap *tm, const void *base, int64_t M, int64_t N) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(ck::kGemmYBoxCols),
+                         static_cast<cuuint32_t>(ck::kGemmYBoxRows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CK_OK : CK_ERR_CUDA;
+}
+
 ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const float *s_w,
                    const ck_bf16 *bias, ck_bf16 *Y, int32_t *acc, int64_t M, int64_t N, int64_t K,
                    DeviceState *st, cudaStream_t stream) {
@@ -108,6 +122,12 @@ ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const f
     if (s != CK_OK) return s;
     s = make_tmap_i8(&tmB, Qw, N, K, plan.b_box_rows);
     if (s != CK_OK) return s;
+    CUtensorMap tmY;
+    std::memset(&tmY, 0, sizeof tmY);
+    if (Y != nullptr) {
+        s = make_tmap_y(&tmY, Y, M, N);
+        if (s != CK_OK) return s;
+    }
     ck::GemmParams p{};
     p.s_x = s_x;
     p.s_w = s_w;
@@ -126,7 +146,7 @@ ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const f
         t_stall_next = 0;
         t_stall_limit_ns = 0;
     }
-    cudaError_t e = ck::launch_gemm_i8(tmA, tmB, p, acc != nullptr, plan, stream);
+    cudaError_t e = ck::launch_gemm_i8(tmA, tmB, tmY, p, acc != nullptr, plan, stream);
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 

@@ -105,6 +105,10 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 template <bool kRaw>
 __device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t tbase, int row,
                                                    int n_tile0);
+__device__ __forceinline__ void store_accumulators_tma(const GemmParams &p,
+                                                       const CUtensorMap *tmY, uint32_t tbase,
+                                                       int row0, int lane, int n_tile0,
+                                                       uint32_t stage_buf, int &chunk_count);
 
 template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -304,7 +308,9 @@ struct alignas(8) PairControl {
     int abort;
 };
 
-constexpr size_t kPairSmemBytes = 1024 + size_t(kPairStages) * kPairStageBytes + sizeof(PairControl);
+constexpr int kEpiStageBytes = 4 * 2 * 2048;  // 4 epilogue warps x 2 buffers x 2 KB
+constexpr size_t kPairSmemBytes =
+    1024 + size_t(kPairStages) * kPairStageBytes + kEpiStageBytes + sizeof(PairControl);
 
 constexpr uint32_t kPairIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
                                 (uint32_t(kPairBN >> 3) << 17) | (uint32_t(kPairBM >> 4) << 24);
@@ -318,11 +324,12 @@ __device__ __forceinline__ int ld_shared_cluster_s32(uint32_t cluster_addr) {
 template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    PairControl *ctl = reinterpret_cast<PairControl *>(smem + size_t(kPairStages) * kPairStageBytes);
+    uint8_t *epi_stage = smem + size_t(kPairStages) * kPairStageBytes;
+    PairControl *ctl = reinterpret_cast<PairControl *>(epi_stage + kEpiStageBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -352,6 +359,7 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (!kRaw) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(&ctl->tmem_base), kTmemCols);
@@ -458,6 +466,8 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ------------------------------------------------ epilogue (warps 2-5, both CTAs)
         const int quarter = warp & 3;
         const uint32_t leader_tmem_empty0 = mapa_shared(smem_u32(&ctl->tmem_empty[0]), 0);
+        const uint32_t stage_buf = smem_u32(epi_stage) + uint32_t(warp - 2) * 4096u;
+        int chunk_count = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
@@ -471,9 +481,12 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * kPairBN);
-            store_accumulators<kRaw>(p, tbase,
-                                     mt * kPairBM + int(rank) * kPairRows + quarter * 32 + lane,
-                                     nt * kPairBN);
+            const int row0 = mt * kPairBM + int(rank) * kPairRows + quarter * 32;
+            if (kRaw)
+                store_accumulators<true>(p, tbase, row0 + lane, nt * kPairBN);
+            else
+                store_accumulators_tma(p, &tmY, tbase, row0, lane, nt * kPairBN, stage_buf,
+                                       chunk_count);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tmem_empty0 + uint32_t(8 * acc));
@@ -483,6 +496,9 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
         }
         if (!ok) raise_timeout(abort, p.err);
+        // every bulk store issued by this warp has completed before exit
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -504,6 +520,83 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     __syncwarp();
     cluster_sync_all();
+}
+
+// Epilogue of one 256-column accumulator row block written through shared
+// memory and TMA stores: each 32-column chunk of the warp's 32 rows (2 KB of
+// bf16) goes into one of two staging buffers of the warp, laid out as the
+// TMA box {32 columns, 32 rows} with the 64-byte swizzle (16-byte piece k of
+// row r sits at piece k ^ ((r >> 1) & 3)), which keeps the 32 lanes' shared
+// stores free of bank conflicts; lane 0 then issues the bulk tensor store.
+// The store clips rows past M and columns past N.
+__device__ __forceinline__ void store_accumulators_tma(const GemmParams &p,
+                                                       const CUtensorMap *tmY, uint32_t tbase,
+                                                       int row0, int lane, int n_tile0,
+                                                       uint32_t stage_buf, int &chunk_count) {
+    const int row = row0 + lane;
+    const bool row_ok = row < p.M;
+    const bool warp_rows_ok = row0 < p.M;
+    const float sx = row_ok ? p.s_x[row] : 0.0f;
+    const uint32_t swz = uint32_t((lane >> 1) & 3);
+#pragma unroll 1
+    for (int c = 0; c < 256 / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
+        tmem_ld_wait();
+        const int n0 = n_tile0 + c * 32;
+        if (!warp_rows_ok || n0 >= p.N) continue;  // warp-uniform
+        const uint32_t buf = stage_buf + uint32_t(chunk_count & 1) * 2048u;
+        // the bulk store that last read this buffer (two chunks ago) is done
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int n = n0 + 8 * g;
+            uint4 out = make_uint4(0u, 0u, 0u, 0u);
+            if (n < p.N) {
+                const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
+                const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n + 4));
+                const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float b[8];
+                if (p.bias) {
+                    const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
+                    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        b[2 * i] = __uint_as_float(bw[i] << 16);
+                        b[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) b[i] = 0.0f;
+                }
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float v = __int2float_rn(int(r[8 * g + i]));
+                    v = __fmul_rn(v, sx);
+                    v = __fmul_rn(v, sw[i]);
+                    f[i] = __fadd_rn(v, b[i]);
+                }
+                out.x = bf16x2_rn(f[0], f[1]);
+                out.y = bf16x2_rn(f[2], f[3]);
+                out.z = bf16x2_rn(f[4], f[5]);
+                out.w = bf16x2_rn(f[6], f[7]);
+            }
+            const uint32_t dst = buf + uint32_t(lane) * 64u + ((uint32_t(g) ^ swz) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out.x),
+                         "r"(out.y), "r"(out.z), "r"(out.w)
+                         : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, n0, row0, buf);
+            bulk_commit_group();
+        }
+        ++chunk_count;
+    }
 }
 
 // Epilogue of one 256-column accumulator row block: this warp's 32 TMEM lanes
@@ -646,8 +739,9 @@ cudaError_t plan_gemm(int M, int N, int num_sms, GemmPlan *plan) {
     return cudaSuccess;
 }
 
-cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                           bool raw_i32, const GemmPlan &plan, cudaStream_t stream) {
+cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmY,
+                           const GemmParams &p, bool raw_i32, const GemmPlan &plan,
+                           cudaStream_t stream) {
     if (p.M <= 0 || p.N <= 0) return cudaSuccess;
     if (!plan.pair) {
         if (raw_i32)
@@ -668,8 +762,8 @@ cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (raw_i32) return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<true>, tmA, tmB, p);
-    return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<false>, tmA, tmB, p);
+    if (raw_i32) return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<true>, tmA, tmB, tmY, p);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<false>, tmA, tmB, tmY, p);
 }
 
 }  // namespace ck

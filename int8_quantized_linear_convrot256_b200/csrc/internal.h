@@ -50,7 +50,13 @@ struct GemmPlan {
 
 cudaError_t plan_gemm(int M, int N, int num_sms, GemmPlan *plan);
 
-cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                           bool raw_i32, const GemmPlan &plan, cudaStream_t stream);
+// tmY: bf16 [M, N] output, box {kGemmYBoxCols, kGemmYBoxRows}, 64-byte
+// swizzle (used by the 2-SM kernel's epilogue; ignored in raw mode).
+constexpr int kGemmYBoxCols = 32;
+constexpr int kGemmYBoxRows = 32;
+
+cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmY,
+                           const GemmParams &p, bool raw_i32, const GemmPlan &plan,
+                           cudaStream_t stream);
 
 }  // namespace ck

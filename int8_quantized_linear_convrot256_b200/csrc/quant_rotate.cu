@@ -18,7 +18,8 @@
 //    (i = 0..7): 16-byte loads, each quad reading 64 contiguous bytes.
 //  * Butterfly stages h = 1, 2, ..., 128 run in that order; each is one IEEE
 //    add or subtract per value (a - c as fma(c, -1, a): one rounding of the
-//    exact difference). h = 1 pairs the two halves of a float2 (scalar ops);
+//    exact difference). h = 1 pairs the two halves of a float2 (scalar ops;
+//    in the staged kernel it is fused with the widening, add/sub.f32.bf16);
 //    h = 2, 4, 32, 64, 128 pair whole float2s (packed add.f32x2 / fma.f32x2);
 //    h = 8, 16 pair lanes t ^ 1, t ^ 2 of the quad through shuffles and one
 //    packed fma(+-1, v, partner). Results are bit-identical to the
@@ -109,6 +110,32 @@ __device__ __forceinline__ void load_block(const float *base, float2 (&P)[kPairs
     }
 }
 
+// Widening fused with the h = 1 butterfly for the two bf16 of one word:
+// add.f32.bf16 / sub.f32.bf16 widen their bf16 operand exactly and round the
+// fp32 sum once, giving fl(a + c) and fl(a - c) as the sequential definition
+// does.
+__device__ __forceinline__ float2 widen_stage1(uint32_t w) {
+    float s, d;
+    const float c = __uint_as_float(w & 0xFFFF0000u);
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %3;\n\tsub.rn.f32.bf16 %1, lo, %3;\n\t}"
+        : "=f"(s), "=f"(d) : "r"(w), "f"(c));
+    return make_float2(s, d);
+}
+// Shared-memory load with the h = 1 stage already applied.
+__device__ __forceinline__ void load_block_smem_s1(uint32_t saddr, float2 (&P)[kPairs]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t x, y, z, w;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                     : "r"(saddr + 64u * i));
+        P[4 * i + 0] = widen_stage1(x);
+        P[4 * i + 1] = widen_stage1(y);
+        P[4 * i + 2] = widen_stage1(z);
+        P[4 * i + 3] = widen_stage1(w);
+    }
+}
 __device__ __forceinline__ void load_block_smem(uint32_t saddr, float2 (&P)[kPairs]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -166,9 +193,11 @@ __device__ __forceinline__ void stage_lanes(float2 (&P)[kPairs], int t) {
     }
 }
 
-// The 8 butterfly stages of ConvRot256, without the final * 1/16 (z = 16 y).
+// The 8 butterfly stages of ConvRot256, without the final * 1/16 (z = 16 y);
+// kStage1Done when h = 1 was applied while loading.
+template <bool kStage1Done = false>
 __device__ __forceinline__ void butterflies(float2 (&P)[kPairs], int t) {
-    stage_in_pair(P);    // h = 1
+    if (!kStage1Done) stage_in_pair(P);    // h = 1
     stage_pairs<1>(P);   // h = 2
     stage_pairs<2>(P);   // h = 4
     stage_lanes<1>(P, t);  // h = 8
@@ -179,9 +208,11 @@ __device__ __forceinline__ void butterflies(float2 (&P)[kPairs], int t) {
 }
 
 __device__ __forceinline__ float quad_absmax(const float2 (&P)[kPairs]) {
-    float m = 0.0f;
+    // four independent chains keep the reduction's dependency depth short
+    float mm[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) m = max3(m, fabsf(P[j].x), fabsf(P[j].y));
+    for (int j = 0; j < kPairs; ++j) mm[j & 3] = max3(mm[j & 3], fabsf(P[j].x), fabsf(P[j].y));
+    float m = fmaxf(max3(mm[0], mm[1], mm[2]), mm[3]);
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     return m;
@@ -395,13 +426,14 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const int64_t row = g * R + row_local;
         const bool active = ok && row_local < R && row < M;
         float2 P[kPairs];
-        if (active)
-            load_block_smem(buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
-                                uint32_t(col0) * 2u,
-                            P);
-        else
-            zero_block(P);
-        if (kRotate) butterflies(P, t);
+        const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
+                            uint32_t(col0) * 2u;
+        if (kRotate) {
+            if (active) load_block_smem_s1(sa, P); else zero_block(P);
+            butterflies<true>(P, t);
+        } else {
+            if (active) load_block_smem(sa, P); else zero_block(P);
+        }
         const float m = quad_absmax(P);
         if (active && t == 0) atomicMax(&s_amax[slot][row_local], __float_as_uint(m));
         if (__syncthreads_or(!ok)) {
