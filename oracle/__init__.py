@@ -73,6 +73,13 @@ def lib():
             L.oracle_quant_row.restype = None
             L.oracle_quantize_rows_bf16.argtypes = [u16p, i64, i64, i64, ctypes.c_int, i8p, f32p]
             L.oracle_quantize_rows_bf16.restype = ctypes.c_int
+            L.oracle_quantize_rows_bf16_act.argtypes = [u16p, i64, i64, i64, ctypes.c_int,
+                                                        ctypes.c_int, i8p, f32p]
+            L.oracle_quantize_rows_bf16_act.restype = ctypes.c_int
+            L.oracle_exp.argtypes = [ctypes.c_float]
+            L.oracle_exp.restype = ctypes.c_float
+            L.oracle_act.argtypes = [ctypes.c_int, ctypes.c_float]
+            L.oracle_act.restype = ctypes.c_float
             L.oracle_rotate_quant_weight.argtypes = [f32p, i64, i64, i8p, f32p]
             L.oracle_rotate_quant_weight.restype = ctypes.c_int
             L.oracle_gemm_i32.argtypes = [i8p, i8p, i64, i64, i64, i32p]
@@ -144,17 +151,38 @@ def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
     return q, s
 
 
-def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = None):
+ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu_tanh": 3}
+
+
+def exp(x) -> np.ndarray:
+    """The oracle's own fp32 e^x (used by the activations), element-wise."""
+    x = np.asarray(x, dtype=np.float32)
+    L = lib()
+    return np.array([L.oracle_exp(float(v)) for v in x.reshape(-1)], np.float32).reshape(x.shape)
+
+
+def act(name: str, x) -> np.ndarray:
+    """fp32 activation (before the bf16 rounding), element-wise."""
+    x = np.asarray(x, dtype=np.float32)
+    L = lib()
+    a = ACTS[name]
+    return np.array([L.oracle_act(a, float(v)) for v in x.reshape(-1)], np.float32).reshape(x.shape)
+
+
+def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = None,
+                       act: str = "none"):
     """quantize_and_rotate_rowwise (rotate=True) or quantize_int8_rowwise
-    (rotate=False) on BF16 rows. ``X_bits`` is uint16 [M, ldx]; the first K
-    columns of each row are used (K defaults to ldx)."""
+    (rotate=False) on BF16 rows, optionally after an input activation
+    (``act`` in ACTS). ``X_bits`` is uint16 [M, ldx]; the first K columns of
+    each row are used (K defaults to ldx)."""
     X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
     M, ld = X_bits.shape
     K = ld if K is None else K
     Qx = np.empty((M, K), np.int8)
     s_x = np.empty(M, np.float32)
-    rc = lib().oracle_quantize_rows_bf16(_ptr(X_bits, ctypes.c_uint16), M, K, ld, int(rotate),
-                                         _ptr(Qx, ctypes.c_int8), _ptr(s_x, ctypes.c_float))
+    rc = lib().oracle_quantize_rows_bf16_act(_ptr(X_bits, ctypes.c_uint16), M, K, ld, int(rotate),
+                                             ACTS[act], _ptr(Qx, ctypes.c_int8),
+                                             _ptr(s_x, ctypes.c_float))
     if rc:
         raise ValueError(f"oracle_quantize_rows_bf16 failed ({rc}): K={K} must be a multiple of 256")
     return Qx, s_x
@@ -219,9 +247,9 @@ def linear_rows(Qx, s_x, Qw, s_w, bias_bits, rows) -> np.ndarray:
     return Y
 
 
-def int8_linear(X_bits, Qw, s_w, bias_bits=None):
-    """The whole forward: quantize_and_rotate_rowwise on X, INT32 GEMM, epilogue.
-    Returns (Y bits [M,N], Qx, s_x, acc)."""
-    Qx, s_x = quantize_rows_bf16(X_bits, rotate=True)
+def int8_linear(X_bits, Qw, s_w, bias_bits=None, act: str = "none"):
+    """The whole forward: quantize_and_rotate_rowwise on X (after the input
+    activation ``act``), INT32 GEMM, epilogue. Returns (Y bits [M,N], Qx, s_x, acc)."""
+    Qx, s_x = quantize_rows_bf16(X_bits, rotate=True, act=act)
     acc = gemm_i32(Qx, Qw)
     return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc

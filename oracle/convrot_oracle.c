@@ -64,6 +64,82 @@ uint16_t oracle_f32_to_bf16_rne(float f) {
     return (uint16_t)kept;
 }
 
+/* ---------------------------------------------------------------- input_act
+ * comfy-kitchen 0.2.40, "HIP backend": int8_linear(input_act=...) applies an
+ * activation to the linear's input inside the quantiser's load, so
+ * linear(act(proj(x))) never stores act's output. The pages do not list the
+ * activations nor their formulas; the readings taken: relu, silu
+ * x / (1 + e^-x) and the tanh form of gelu
+ * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), computed in fp32 on the
+ * widened bf16 input and rounded to bf16 (the precision an unfused bf16
+ * activation would store) before the rotation. The gelu is evaluated as
+ * x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3), which equals
+ * 0.5 x (1 + tanh(u)) and has no cancellation where tanh(u) is near -1.
+ *
+ * e^x: Cody-Waite reduction x = n ln2 + r with ln2 split in a 16-bit head
+ * (n * head is exact for |n| < 256) and a tail, a degree-7 Taylor polynomial
+ * of e^r (|r| <= ln2/2, truncation error below 2^-27) in Horner form with
+ * separate IEEE multiplies and adds, then an exact scaling by 2^n (two steps
+ * when 2^n is subnormal). */
+#define ACT_NONE 0
+#define ACT_RELU 1
+#define ACT_SILU 2
+#define ACT_GELU_TANH 3
+
+static float pow2i(int k) { /* 2^k for -126 <= k <= 127, exact */
+    uint32_t u = (uint32_t)(k + 127) << 23;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+float oracle_exp(float x) {
+    if (x > 88.8f)
+        return INFINITY;
+    if (x < -104.0f)
+        return 0.0f;
+    const float log2e = 1.442695f;
+    const float ln2_hi = 0.693145751953125f;
+    const float ln2_lo = 1.4286068e-06f;
+    float n = nearbyintf(x * log2e);
+    float r = x - n * ln2_hi;
+    r = r - n * ln2_lo;
+    float p = 1.984127e-04f; /* 1/7!, 1/6!, ... rounded to fp32 */
+    p = p * r + 1.3888889e-03f;
+    p = p * r + 8.333334e-03f;
+    p = p * r + 4.1666668e-02f;
+    p = p * r + 1.6666667e-01f;
+    p = p * r + 0.5f;
+    p = p * r + 1.0f;
+    p = p * r + 1.0f;
+    int k = (int)n;
+    if (k > 127)
+        return (p * pow2i(127)) * pow2i(k - 127);
+    if (k < -126)
+        return (p * pow2i(k + 100)) * pow2i(-100);
+    return p * pow2i(k);
+}
+
+float oracle_act(int act, float x) {
+    switch (act) {
+    case ACT_RELU:
+        return x > 0.0f ? x : 0.0f;
+    case ACT_SILU: {
+        float e = oracle_exp(-x);
+        return x / (1.0f + e);
+    }
+    case ACT_GELU_TANH: {
+        float x3 = (x * x) * x;
+        float inner = x + 0.044715f * x3;
+        float u = 7.978846e-01f * inner; /* sqrt(2/pi) */
+        float e = oracle_exp(-2.0f * u);
+        return x / (1.0f + e);
+    }
+    default:
+        return x;
+    }
+}
+
 /* ConvRot256 on one block of 256 values, in place. */
 void oracle_rot256(float *v) {
     for (int h = 1; h < ROT_N; h <<= 1) {
@@ -108,8 +184,17 @@ void oracle_quant_row(const float *y, int64_t K, int8_t *q, float *s_out) {
 /* quantize_and_rotate_rowwise on BF16 rows: widen, ConvRot256 every 256-block
  * of the row, then quantise the whole rotated row. X has row stride ldx
  * (elements). rotate == 0 skips the rotation (plain quantize_int8_rowwise). */
+int oracle_quantize_rows_bf16_act(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                  int rotate, int act, int8_t *Qx, float *s_x);
+
 int oracle_quantize_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                               int rotate, int8_t *Qx, float *s_x) {
+    return oracle_quantize_rows_bf16_act(X, M, K, ldx, rotate, ACT_NONE, Qx, s_x);
+}
+
+/* The same, with the input activation applied first (ACT_NONE: none). */
+int oracle_quantize_rows_bf16_act(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                  int rotate, int act, int8_t *Qx, float *s_x) {
     if (K % ROT_N != 0 || ldx < K)
         return 1;
     int err = 0;
@@ -123,8 +208,12 @@ int oracle_quantize_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t l
 #pragma omp for schedule(static)
             for (int64_t m = 0; m < M; ++m) {
                 const uint16_t *row = X + m * ldx;
-                for (int64_t k = 0; k < K; ++k)
-                    buf[k] = oracle_bf16_to_f32(row[k]);
+                for (int64_t k = 0; k < K; ++k) {
+                    float v = oracle_bf16_to_f32(row[k]);
+                    if (act != ACT_NONE)
+                        v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));
+                    buf[k] = v;
+                }
                 if (rotate)
                     for (int64_t b = 0; b < K; b += ROT_N)
                         oracle_rot256(buf + b);

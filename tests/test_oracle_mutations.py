@@ -29,6 +29,12 @@ MUTATIONS = {
     "epilogue_bias_dropped": ("    f = f + b;\n", "    (void)b;\n"),
     "bf16_truncates": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (rest >= 0x8000u)"),
+    "gelu_cubic_coefficient": ("float inner = x + 0.044715f * x3;", "float inner = x + 0.04715f * x3;"),
+    "silu_wrong_sign": ("float e = oracle_exp(-x);", "float e = oracle_exp(x);"),
+    "exp_drops_a_term": ("p = p * r + 1.6666667e-01f;", "p = p * r + 0.0f;"),
+    "exp_reduction_head_only": ("r = r - n * ln2_lo;", "r = r - 0.0f;"),
+    "act_not_rounded_to_bf16": ("v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));",
+                                "v = oracle_act(act, v);"),
 }
 
 
@@ -44,6 +50,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
                           stderr=subprocess.DEVNULL)
     env = dict(os.environ, CONVROT_ORACLE_LIB=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_act_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
