@@ -154,14 +154,14 @@ class ClockSampler:
 # ---------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float):
+def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float, act: str = "none"):
     """Time the oracle on a bounded sample of rows (quantise + linear rows).
     Returns (TOPS, rows, seconds, threads)."""
     import oracle
 
     def run(rows):
         t = time.perf_counter()
-        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows])
+        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows], act=act)
         oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
         return time.perf_counter() - t
 
@@ -190,14 +190,14 @@ def run_reference(args, cfg, rank, world):
     total_budget = 150.0
     per_step = total_budget / max(1, args.steps + args.warmup)
     t_probe = time.perf_counter()
-    Qx, s_x = oracle.quantize_rows_bf16(X_bits[:4])
+    Qx, s_x = oracle.quantize_rows_bf16(X_bits[:4], act=args.act)
     oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(4))
     t_row = (time.perf_counter() - t_probe) / 4
     rows = int(max(1, min(cfg.M, per_step / max(t_row, 1e-9))))
     times = []
     for i in range(args.warmup + args.steps):
         t = time.perf_counter()
-        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows])
+        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows], act=args.act)
         oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
         dt = time.perf_counter() - t
         if i >= args.warmup:
@@ -209,7 +209,7 @@ def run_reference(args, cfg, rank, world):
     line = {"metric": METRIC, "value": tops, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic", "impl": "reference",
-            "config": config_dict(cfg, world),
+            "config": config_dict(cfg, world, "weak", args.act),
             "cpu_baseline": {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": tops, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -218,14 +218,15 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
-def config_dict(cfg, world, scaling="weak"):
+def config_dict(cfg, world, scaling="weak", act="none"):
     par = (f"replicas x{world}: every rank runs the whole batch" if scaling == "weak"
            else f"rows split over {world} ranks")
     return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "seed": cfg.seed,
             "x_dist": cfg.x_dist, "outlier_channels": cfg.n_outlier,
             "parallelism": par + " (rows are independent: no collective on the data path)",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); X is also larger than L2",
-            "weights": "rotated + quantised once before timing (offline)"}
+            "weights": "rotated + quantised once before timing (offline)",
+            "input_act": act}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -258,8 +259,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     ck.clear_device_error()
 
+    def quantize():
+        if args.act == "none":
+            ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        else:
+            ck.quantize_rotate_rowwise_act(Xd, args.act, Qx, s_x)
+
     def step():
-        ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        quantize()
         ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
 
     for _ in range(args.warmup):
@@ -278,7 +285,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        quantize()
         ev[i][1].record(stream)
         ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
         ev[i][2].record(stream)
@@ -321,7 +328,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
     e2e_steps = max(1, min(args.steps, 10))
     for _ in range(2):
         Xd2.copy_(X_host, non_blocking=True)
-        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws)
+        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws, input_act=args.act)
         Y_host.copy_(Y, non_blocking=True)
     torch.cuda.synchronize()
     if world > 1:
@@ -331,7 +338,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
     e0.record(stream)
     for _ in range(e2e_steps):
         Xd2.copy_(X_host, non_blocking=True)
-        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws)
+        ck.int8_linear(Xd2, Qw, s_w, bd, out=Y, workspace=ws, input_act=args.act)
         Y_host.copy_(Y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -371,7 +378,8 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
 
             Qw_o, s_w_o = oracle.rotate_quant_weight(Wcpu.numpy())
             tops, rows, dt, cores = oracle_sample(cfg, X_bits, Qw_o, s_w_o,
-                                                  workloads.bf16_bits(bias), args.cpu_seconds)
+                                                  workloads.bf16_bits(bias), args.cpu_seconds,
+                                                  args.act)
             cpu = {"value": tops, "unit": UNIT, "cores": cores, "kind": "oracle",
                    "sample": f"{rows} of {cfg.M} rows (rotate+quantise and all {cfg.N} outputs of "
                              f"those rows) in {dt:.1f} s, plain C oracle, OpenMP over rows"}
@@ -382,7 +390,7 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
             "scaling": args.scaling,
             "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
             "dtype": "int8", "data": "synthetic", "impl": "ours",
-            "config": config_dict(cfg, world, args.scaling),
+            "config": config_dict(cfg, world, args.scaling, args.act),
             "roofline": {"kernel": "gemm_i8_kernel (tcgen05 kind::i8 + fused epilogue)",
                          "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
@@ -414,6 +422,8 @@ def main(argv=None):
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: every rank runs the whole batch (replicas); strong: the "
                          "batch's rows are split over the ranks")
+    ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
+                    help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",

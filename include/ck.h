@@ -120,6 +120,29 @@ ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int
 ck_status ck_quantize_int8_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Qx, float *s_x, ck_stream_t stream);
 
+/* Input activations for the *_act entry points (applied to the bf16 input in
+ * fp32, rounded to bf16, then rotated and quantised). */
+typedef enum ck_act {
+    CK_ACT_NONE = 0,
+    CK_ACT_RELU = 1,      /* max(x, 0) */
+    CK_ACT_SILU = 2,      /* x / (1 + e^-x) */
+    CK_ACT_GELU_TANH = 3  /* 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) */
+} ck_act;
+
+/*
+ * quantize_and_rotate_rowwise with an input activation (comfy-kitchen 0.2.40,
+ * "HIP backend": int8_linear(input_act=...) folds the activation into the
+ * fused ConvRot quantiser's load, so act(x) is never written to memory).
+ * Each element becomes bf16_rne(act(float(x))) before ConvRot256; act is a
+ * ck_act value (CK_ERR_INVALID_VALUE otherwise). The list of activations and
+ * their formulas are a reading: the page names the argument only. e^x is the
+ * library's own (Cody-Waite reduction + degree-7 Taylor polynomial, every
+ * step one IEEE operation), accurate to a few ulp. Other arguments as for
+ * ck_quantize_rotate_rowwise.
+ */
+ck_status ck_quantize_rotate_rowwise_act(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                         int act, int8_t *Qx, float *s_x, ck_stream_t stream);
+
 /*
  * Bytes of device workspace ck_int8_linear needs for M rows of K features:
  * the INT8 codes (M*K bytes) and the row scales (4*M bytes), each part
@@ -148,6 +171,16 @@ size_t ck_int8_linear_workspace_bytes(int64_t M, int64_t K);
 ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
                          const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
                          void *workspace, size_t workspace_bytes, ck_stream_t stream);
+
+/*
+ * ck_int8_linear with an input activation: Y = linear(act(X)) with act
+ * applied inside the quantiser's load (see ck_quantize_rotate_rowwise_act).
+ * CK_ACT_NONE gives exactly ck_int8_linear.
+ */
+ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_t *Qw,
+                             const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                             int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                             ck_stream_t stream);
 
 /*
  * The GEMM and fused epilogue alone, on activations already quantised (by

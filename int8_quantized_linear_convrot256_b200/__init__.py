@@ -38,6 +38,7 @@ CK_ERR_ARCH = 5
 CK_ERR_CUDA = 6
 CK_ERR_DEVICE_TIMEOUT = 7
 MAX_K = 132864
+ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu_tanh": 3}
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 if not os.path.exists(LIB_PATH):
@@ -58,6 +59,9 @@ _SIGS = {
     "ck_int8_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                              ctypes.c_size_t, _vp]),
     "ck_int8_gemm_rowscale": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_quantize_rotate_rowwise_act": (_st, [_vp, _i64, _i64, _i64, _st, _vp, _vp, _vp]),
+    "ck_int8_linear_act": (_st, [_vp, _i64, _st, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                 ctypes.c_size_t, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
@@ -157,6 +161,14 @@ def quantize_rotate_rowwise(X: torch.Tensor, Qx=None, s_x=None, stream=None):
     return _quant(lib.ck_quantize_rotate_rowwise, "ck_quantize_rotate_rowwise", X, Qx, s_x, stream)
 
 
+def quantize_rotate_rowwise_act(X: torch.Tensor, act: str, Qx=None, s_x=None, stream=None):
+    """quantize_and_rotate_rowwise after an input activation ("none", "relu",
+    "silu", "gelu_tanh"), applied inside the quantiser's load."""
+    a = ACTS[act]
+    return _quant(lambda *args: lib.ck_quantize_rotate_rowwise_act(*args[:4], a, *args[4:]),
+                  "ck_quantize_rotate_rowwise_act", X, Qx, s_x, stream)
+
+
 def quantize_int8_rowwise(X: torch.Tensor, Qx=None, s_x=None, stream=None):
     """quantize_int8_rowwise: per-row INT8 of bf16 X [M, K] without rotation."""
     return _quant(lib.ck_quantize_int8_rowwise, "ck_quantize_int8_rowwise", X, Qx, s_x, stream)
@@ -172,8 +184,11 @@ test_quantize_rowwise_norotate.__test__ = False
 
 def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
                 bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Y[M, N] = bf16(((int8 GEMM of rotate+quantised X with Qw) * s_x) * s_w + bias)."""
+                workspace: torch.Tensor | None = None, stream=None,
+                input_act: str = "none") -> torch.Tensor:
+    """Y[M, N] = bf16(((int8 GEMM of rotate+quantised act(X) with Qw) * s_x) * s_w + bias).
+    ``input_act`` ("none", "relu", "silu", "gelu_tanh") is applied inside the
+    quantiser's load (ck_int8_linear_act); "none" calls ck_int8_linear."""
     _need(X, "X", torch.bfloat16, 2)
     _need(Qw, "Qw", torch.int8, 2)
     _rows_contiguous(Qw, "Qw")
@@ -194,9 +209,14 @@ def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
     ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
-    _check(lib.ck_int8_linear(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out), M, N, K,
-                              _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              _stream(stream)), "ck_int8_linear")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if input_act == "none":
+        _check(lib.ck_int8_linear(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out), M, N,
+                                  K, _ptr(workspace), ws_bytes, _stream(stream)), "ck_int8_linear")
+    else:
+        _check(lib.ck_int8_linear_act(_ptr(X), ldx, ACTS[input_act], _ptr(Qw), _ptr(s_w),
+                                      _ptr(bias), _ptr(out), M, N, K, _ptr(workspace), ws_bytes,
+                                      _stream(stream)), "ck_int8_linear_act")
     return out
 
 

@@ -151,8 +151,8 @@ ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const f
 }
 
 ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8_t *Qx,
-                       float *s_x, bool rotate, ck_stream_t stream) {
-    if (M < 0) return CK_ERR_INVALID_VALUE;
+                       float *s_x, bool rotate, int act, ck_stream_t stream) {
+    if (M < 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
     ck_status s = check_k(K);
     if (s == CK_ERR_INVALID_VALUE) return s;
     if (ldx < K && K > 0) return CK_ERR_INVALID_VALUE;
@@ -164,7 +164,7 @@ ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8
     DeviceState *st = nullptr;
     s = device_state(&st);
     if (s != CK_OK) return s;
-    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, Qx, s_x, st->err,
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, act, Qx, s_x, st->err,
                                                st->num_sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
@@ -207,17 +207,22 @@ ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Q
 
 ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                      int8_t *Qx, float *s_x, ck_stream_t stream) {
-    return quant_common(X, M, K, ldx, Qx, s_x, true, stream);
+    return quant_common(X, M, K, ldx, Qx, s_x, true, CK_ACT_NONE, stream);
+}
+
+ck_status ck_quantize_rotate_rowwise_act(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                         int act, int8_t *Qx, float *s_x, ck_stream_t stream) {
+    return quant_common(X, M, K, ldx, Qx, s_x, true, act, stream);
 }
 
 ck_status ck_quantize_int8_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Qx, float *s_x, ck_stream_t stream) {
-    return quant_common(X, M, K, ldx, Qx, s_x, false, stream);
+    return quant_common(X, M, K, ldx, Qx, s_x, false, CK_ACT_NONE, stream);
 }
 
 ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                             int8_t *Qx, float *s_x, ck_stream_t stream) {
-    return quant_common(X, M, K, ldx, Qx, s_x, false, stream);
+    return quant_common(X, M, K, ldx, Qx, s_x, false, CK_ACT_NONE, stream);
 }
 
 size_t ck_int8_linear_workspace_bytes(int64_t M, int64_t K) {
@@ -225,10 +230,11 @@ size_t ck_int8_linear_workspace_bytes(int64_t M, int64_t K) {
     return round256(size_t(M) * size_t(K)) + round256(size_t(M) * 4);
 }
 
-ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
-                         const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
-                         void *workspace, size_t workspace_bytes, ck_stream_t stream) {
-    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_t *Qw,
+                             const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                             int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                             ck_stream_t stream) {
+    if (M < 0 || N < 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
     ck_status s = check_k(K);
     if (s == CK_ERR_INVALID_VALUE) return s;
     if (ldx < K) return CK_ERR_INVALID_VALUE;
@@ -248,9 +254,17 @@ ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const 
     float *s_x = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                            round256(size_t(M) * size_t(K)));
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, true, Qx, s_x, st->err, st->num_sms, cs);
+    cudaError_t e =
+        ck::launch_quant_rows_bf16(X, M, K, ldx, true, act, Qx, s_x, st->err, st->num_sms, cs);
     if (e != cudaSuccess) return CK_ERR_CUDA;
     return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
+}
+
+ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
+                         const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                         void *workspace, size_t workspace_bytes, ck_stream_t stream) {
+    return ck_int8_linear_act(X, ldx, CK_ACT_NONE, Qw, s_w, bias, Y, M, N, K, workspace,
+                              workspace_bytes, stream);
 }
 
 ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t *Qw,

@@ -11,9 +11,11 @@ namespace ck {
 
 // Rows of bf16 (bit patterns) with row stride ldx; rotate=false skips ConvRot.
 // err is the device error word (bounded waits of the staged variant).
+// act: input activation applied before the rotation (0 none, 1 relu, 2 silu,
+// 3 tanh-form gelu); only with rotate.
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   bool rotate, int8_t *Q, float *S, unsigned *err, int num_sms,
-                                   cudaStream_t stream);
+                                   bool rotate, int act, int8_t *Q, float *S, unsigned *err,
+                                   int num_sms, cudaStream_t stream);
 
 // Rows of fp32 with row stride K (offline weight preparation), always rotated.
 cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,

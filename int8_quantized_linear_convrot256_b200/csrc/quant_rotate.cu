@@ -46,6 +46,7 @@
 //    full row group per CTA in flight. K > 32768 takes a two-pass variant
 //    (rows re-read from L2); fp32 weights (offline) take direct loads.
 //  * No FMA contraction: every operation is an explicit _rn intrinsic.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -86,18 +87,137 @@ __device__ __forceinline__ float2 widen_bf16x2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+// ------------------------------------------------------------------ input_act
+// int8_linear(input_act=...) (comfy-kitchen 0.2.40, "HIP backend"): the
+// activation is applied to the widened bf16 input, in fp32, and rounded to
+// bf16 before the rotation. relu; silu x / (1 + e^-x); gelu (tanh form)
+// 0.5 x (1 + tanh(u)) = x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3).
+// e^x: Cody-Waite reduction x = n ln2 + r (ln2 = 16-bit head + tail),
+// degree-7 Taylor polynomial of e^r in Horner form, exact scaling by 2^n;
+// every step is one IEEE operation (fused multiply-adds where the definition
+// has them), so CPU and GPU agree bit for bit.
+constexpr int kActNone = 0;
+constexpr int kActRelu = 1;
+constexpr int kActSilu = 2;
+constexpr int kActGeluTanh = 3;
+
+// e^x of two values, branch-free: n = rint(x log2 e) by adding and removing
+// 1.5 * 2^23 (round-to-nearest-even, |x log2 e| < 2^22 in range), k = n from
+// the sum's bits; r = x - n ln2 (two fused steps, 16-bit head + tail);
+// degree-7 Taylor polynomial of e^r by fused Horner steps (packed
+// fma.f32x2); then p * 2^k as (p * 2^a) * 2^b with a = floor(k/2),
+// b = ceil(k/2): p * 2^a is exact and normal (p >= 0.7, a >= -75), so the
+// result is p * 2^k rounded once, as the definition's scaling gives for every
+// k in range. Outside [-104, 88.8] the definition's limits (0, +inf) are
+// selected.
+__device__ __forceinline__ float2 act_exp2(float2 x) {
+    const float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float2 m = __fadd2_rn(__fmul2_rn(x, make_float2(1.442695f, 1.442695f)),
+                                make_float2(kRound, kRound));
+    const float2 n = __fadd2_rn(m, make_float2(-kRound, -kRound));
+    const float2 mn = make_float2(-n.x, -n.y);
+    float2 r = __ffma2_rn(mn, make_float2(0.693145751953125f, 0.693145751953125f), x);
+    r = __ffma2_rn(mn, make_float2(1.4286068e-06f, 1.4286068e-06f), r);
+    float2 p = make_float2(1.984127e-04f, 1.984127e-04f);  // 1/7!, 1/6!, ..., 1, 1 in fp32
+    p = __ffma2_rn(p, r, make_float2(1.3888889e-03f, 1.3888889e-03f));
+    p = __ffma2_rn(p, r, make_float2(8.333334e-03f, 8.333334e-03f));
+    p = __ffma2_rn(p, r, make_float2(4.1666668e-02f, 4.1666668e-02f));
+    p = __ffma2_rn(p, r, make_float2(1.6666667e-01f, 1.6666667e-01f));
+    p = __ffma2_rn(p, r, make_float2(0.5f, 0.5f));
+    p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+    p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+    const int kx = int(__float_as_uint(m.x) - __float_as_uint(kRound));
+    const int ky = int(__float_as_uint(m.y) - __float_as_uint(kRound));
+    // k = a + b with a = floor(k/2), b = ceil(k/2), both in [-75, 64]; each
+    // factor is built from k alone
+    const float2 s1 = make_float2(__uint_as_float(uint32_t((kx >> 1) + 127) << 23),
+                                  __uint_as_float(uint32_t((ky >> 1) + 127) << 23));
+    const float2 s2 = make_float2(__uint_as_float(uint32_t(((kx + 1) >> 1) + 127) << 23),
+                                  __uint_as_float(uint32_t(((ky + 1) >> 1) + 127) << 23));
+    float2 e = __fmul2_rn(__fmul2_rn(p, s1), s2);
+    const float inf = __uint_as_float(0x7F800000u);
+    e.x = x.x > 88.8f ? inf : (x.x < -104.0f ? 0.0f : e.x);
+    e.y = x.y > 88.8f ? inf : (x.y < -104.0f ? 0.0f : e.y);
+    return e;
+}
+
+// x / d where only bf16_rne of the quotient is used: a reciprocal
+// approximation (error <= 1 ulp) times x is within 2 fp32 ulps of the
+// correctly rounded quotient, so its bf16 rounding is the same unless it
+// lies within a few ulps of a bf16 rounding midpoint (the low 16 bits near
+// 0x8000) or d is huge; `exact` is set for those, and the caller then redoes
+// the value with the IEEE division.
+__device__ __forceinline__ float div_for_bf16(float x, float d, bool &exact) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(d));
+    const float q = __fmul_rn(x, r);
+    const uint32_t lo = __float_as_uint(q) & 0xFFFFu;
+    exact = exact || (lo - 0x7FF8u <= 16u) || (d > 1.0e36f);
+    return q;
+}
+
+// Denominator 1 + e^v of silu (v = -x) and of the tanh-form gelu (v = -2u).
+template <int kAct>
+__device__ __forceinline__ float2 act_denominator(float2 x) {
+    float2 v;
+    if (kAct == kActSilu) {
+        v = make_float2(-x.x, -x.y);
+    } else {
+        const float2 x3 = __fmul2_rn(__fmul2_rn(x, x), x);
+        const float2 inner = __ffma2_rn(make_float2(0.044715f, 0.044715f), x3, x);
+        const float2 u = __fmul2_rn(make_float2(7.978846e-01f, 7.978846e-01f), inner);
+        v = __fmul2_rn(make_float2(-2.0f, -2.0f), u);
+    }
+    return __fadd2_rn(make_float2(1.0f, 1.0f), act_exp2(v));
+}
+
+// bf16x2 word -> activation of both values -> bf16x2 word (round to nearest
+// even). `exact` is raised when a quotient needs the IEEE division; then
+// act_bf16x2_exact gives the word.
+template <int kAct>
+__device__ __forceinline__ uint32_t act_bf16x2(uint32_t w, bool &exact) {
+    if (kAct == kActNone) return w;
+    const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    float2 a;
+    if (kAct == kActRelu) {
+        a = make_float2(x.x > 0.0f ? x.x : 0.0f, x.y > 0.0f ? x.y : 0.0f);
+    } else {
+        const float2 d = act_denominator<kAct>(x);
+        a = make_float2(div_for_bf16(x.x, d.x, exact), div_for_bf16(x.y, d.y, exact));
+    }
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a.x, a.y);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <int kAct>
+__device__ __noinline__ uint32_t act_bf16x2_exact(uint32_t w) {
+    const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    const float2 d = act_denominator<kAct>(x);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(__fdiv_rn(x.x, d.x), __fdiv_rn(x.y, d.y));
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <int kAct>
+__device__ __forceinline__ uint32_t act_bf16x2(uint32_t w) {
+    bool exact = false;
+    const uint32_t r = act_bf16x2<kAct>(w, exact);
+    return exact ? act_bf16x2_exact<kAct>(w) : r;
+}
+
 // Lane t's 64 values of one block; base points at element 8t of the block.
+template <int kAct = kActNone>
 __device__ __forceinline__ void load_block(const uint16_t *base, float2 (&P)[kPairs]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(base + 32 * i));
-        P[4 * i + 0] = widen_bf16x2(u.x);
-        P[4 * i + 1] = widen_bf16x2(u.y);
-        P[4 * i + 2] = widen_bf16x2(u.z);
-        P[4 * i + 3] = widen_bf16x2(u.w);
+        P[4 * i + 0] = widen_bf16x2(act_bf16x2<kAct>(u.x));
+        P[4 * i + 1] = widen_bf16x2(act_bf16x2<kAct>(u.y));
+        P[4 * i + 2] = widen_bf16x2(act_bf16x2<kAct>(u.z));
+        P[4 * i + 3] = widen_bf16x2(act_bf16x2<kAct>(u.w));
     }
 }
 
+template <int kAct = kActNone>
 __device__ __forceinline__ void load_block(const float *base, float2 (&P)[kPairs]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -122,7 +242,36 @@ __device__ __forceinline__ float2 widen_stage1(uint32_t w) {
         : "=f"(s), "=f"(d) : "r"(w), "f"(c));
     return make_float2(s, d);
 }
-// Shared-memory load with the h = 1 stage already applied.
+// Applies the input activation in place to this lane's 64 staged bf16 values
+// (8 chunks of 16 bytes at saddr + 64 i, read and written only by this lane).
+// A rolled loop keeps one copy of the activation code in the kernel.
+template <int kAct>
+__device__ __forceinline__ void act_in_smem(uint32_t saddr) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        uint32_t x, y, z, w;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                     : "r"(saddr + 64u * i));
+        bool exact = false;
+        uint32_t ax = act_bf16x2<kAct>(x, exact);
+        uint32_t ay = act_bf16x2<kAct>(y, exact);
+        uint32_t az = act_bf16x2<kAct>(z, exact);
+        uint32_t aw = act_bf16x2<kAct>(w, exact);
+        if (exact) {
+            ax = act_bf16x2_exact<kAct>(x);
+            ay = act_bf16x2_exact<kAct>(y);
+            az = act_bf16x2_exact<kAct>(z);
+            aw = act_bf16x2_exact<kAct>(w);
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr + 64u * i), "r"(ax),
+                     "r"(ay), "r"(az), "r"(aw)
+                     : "memory");
+    }
+}
+
+// Shared-memory load (input activation applied) with the h = 1 stage done.
+template <int kAct>
 __device__ __forceinline__ void load_block_smem_s1(uint32_t saddr, float2 (&P)[kPairs]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -130,10 +279,10 @@ __device__ __forceinline__ void load_block_smem_s1(uint32_t saddr, float2 (&P)[k
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
                      : "r"(saddr + 64u * i));
-        P[4 * i + 0] = widen_stage1(x);
-        P[4 * i + 1] = widen_stage1(y);
-        P[4 * i + 2] = widen_stage1(z);
-        P[4 * i + 3] = widen_stage1(w);
+        P[4 * i + 0] = widen_stage1(act_bf16x2<kAct>(x));
+        P[4 * i + 1] = widen_stage1(act_bf16x2<kAct>(y));
+        P[4 * i + 2] = widen_stage1(act_bf16x2<kAct>(z));
+        P[4 * i + 3] = widen_stage1(act_bf16x2<kAct>(w));
     }
 }
 __device__ __forceinline__ void load_block_smem(uint32_t saddr, float2 (&P)[kPairs]) {
@@ -328,7 +477,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const 
 // ------------------------------------------------------------------ kernels
 
 // Single pass with direct loads: CTA = rows_per_cta rows x (K/256) quads.
-template <bool kRotate, typename TIn>
+template <bool kRotate, int kAct, typename TIn>
 __global__ void __launch_bounds__(kMaxThreads, 1)
 quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
                   int8_t *__restrict__ Q, float *__restrict__ S) {
@@ -346,7 +495,7 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     if (tid < rows_per_cta) s_amax[tid] = 0u;
     float2 P[kPairs];
     if (active)
-        load_block(X + row * ldx + col0, P);
+        load_block<kAct>(X + row * ldx + col0, P);
     else
         zero_block(P);
     if (kRotate) butterflies(P, t);
@@ -365,7 +514,7 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
 // group: after it, every thread has read its values out of the buffer (so the
 // buffer can be refilled) and the row absmax is complete. The absmax slots are
 // triple-buffered so a slot is cleared one full barrier before its next use.
-template <bool kRotate>
+template <bool kRotate, int kAct>
 __global__ void __launch_bounds__(kMaxThreads, 1)
 quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
                        int rows_per_cta, int8_t *__restrict__ Q, float *__restrict__ S,
@@ -429,7 +578,12 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
                             uint32_t(col0) * 2u;
         if (kRotate) {
-            if (active) load_block_smem_s1(sa, P); else zero_block(P);
+            if (active) {
+                if (kAct != kActNone) act_in_smem<kAct>(sa);
+                load_block_smem_s1<kActNone>(sa, P);
+            } else {
+                zero_block(P);
+            }
             butterflies<true>(P, t);
         } else {
             if (active) load_block_smem(sa, P); else zero_block(P);
@@ -460,7 +614,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
 // Two passes for long rows (K > 32768): one CTA per row, 128 quads; pass 1
 // rotates every block and reduces the absmax, pass 2 reloads (from L2),
 // rotates again and quantises.
-template <bool kRotate, typename TIn>
+template <bool kRotate, int kAct, typename TIn>
 __global__ void __launch_bounds__(kTwoPassQuads * 4, 1)
 quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx,
                            int8_t *__restrict__ Q, float *__restrict__ S) {
@@ -477,7 +631,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
         const int blk = b0 + quad;
         float2 P[kPairs];
         if (blk < nb)
-            load_block(xrow + blk * kBlock + 8 * t, P);
+            load_block<kAct>(xrow + blk * kBlock + 8 * t, P);
         else
             zero_block(P);
         if (kRotate) butterflies(P, t);
@@ -492,7 +646,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
         const int blk = b0 + quad;
         float2 P[kPairs];
         if (blk < nb)
-            load_block(xrow + blk * kBlock + 8 * t, P);
+            load_block<kAct>(xrow + blk * kBlock + 8 * t, P);
         else
             zero_block(P);
         if (kRotate) butterflies(P, t);
@@ -528,21 +682,21 @@ std::mutex g_occ_mutex;
 // (device, rotate, threads, smem) -> CTAs of the bulk kernel per SM
 std::map<std::tuple<int, int, int, size_t>, int> g_bulk_occupancy;
 
-template <bool kRotate>
+template <bool kRotate, int kAct>
 cudaError_t bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
     std::lock_guard<std::mutex> lock(g_occ_mutex);
-    const auto key = std::make_tuple(dev, kRotate ? 1 : 0, threads, smem);
+    const auto key = std::make_tuple(dev, (kRotate ? 1 : 0) + 2 * kAct, threads, smem);
     auto it = g_bulk_occupancy.find(key);
     if (it != g_bulk_occupancy.end()) {
         *out = it->second;
         return cudaSuccess;
     }
-    cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel<kRotate>,
+    cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel<kRotate, kAct>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kBulkSmemBudget));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_bulk_kernel<kRotate>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_bulk_kernel<kRotate, kAct>,
                                                       threads, smem);
     if (e != cudaSuccess) return e;
     g_bulk_occupancy[key] = per_sm;
@@ -550,7 +704,7 @@ cudaError_t bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
     return cudaSuccess;
 }
 
-template <bool kRotate>
+template <bool kRotate, int kAct>
 cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
                         unsigned *err, int num_sms, cudaStream_t stream, bool *launched) {
     *launched = false;
@@ -564,19 +718,19 @@ cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, in
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = bulk_blocks_per_sm<kRotate>(dev, threads, smem, &per_sm);
+    e = bulk_blocks_per_sm<kRotate, kAct>(dev, threads, smem, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaSuccess;
     const int64_t groups = (M + rows - 1) / rows;
     const int64_t cap = int64_t(per_sm) * num_sms;
     const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
-    quant_rows_bulk_kernel<kRotate><<<grid, threads, smem, stream>>>(
+    quant_rows_bulk_kernel<kRotate, kAct><<<grid, threads, smem, stream>>>(
         X, M, static_cast<int>(K), ldx, rows, Q, S, err, kDefaultWaitLimitNs);
     *launched = true;
     return cudaGetLastError();
 }
 
-template <bool kRotate, typename TIn>
+template <bool kRotate, int kAct, typename TIn>
 cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
                           cudaStream_t stream) {
     const int nb = static_cast<int>(K / kBlock);
@@ -584,35 +738,45 @@ cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_
         int threads = 0;
         const int rows = pick_rows_per_cta(nb, kMaxRowsPerCta, &threads);
         const int64_t grid = (M + rows - 1) / rows;
-        quant_rows_kernel<kRotate, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
+        quant_rows_kernel<kRotate, kAct, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
             X, M, static_cast<int>(K), ldx, rows, Q, S);
     } else {
-        quant_rows_two_pass_kernel<kRotate, TIn>
+        quant_rows_two_pass_kernel<kRotate, kAct, TIn>
             <<<static_cast<unsigned>(M), kTwoPassQuads * 4, 0, stream>>>(
                 X, M, static_cast<int>(K), ldx, Q, S);
     }
     return cudaGetLastError();
 }
 
+template <bool kRotate, int kAct>
+cudaError_t launch_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
+                        unsigned *err, int num_sms, cudaStream_t stream) {
+    bool launched = false;
+    cudaError_t e = launch_bulk<kRotate, kAct>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+    return launch_direct<kRotate, kAct>(X, M, K, ldx, Q, S, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   bool rotate, int8_t *Q, float *S, unsigned *err, int num_sms,
-                                   cudaStream_t stream) {
+                                   bool rotate, int act, int8_t *Q, float *S, unsigned *err,
+                                   int num_sms, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
-    bool launched = false;
-    cudaError_t e =
-        rotate ? launch_bulk<true>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched)
-               : launch_bulk<false>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched);
-    if (e != cudaSuccess || launched) return e;
-    return rotate ? launch_direct<true>(X, M, K, ldx, Q, S, stream)
-                  : launch_direct<false>(X, M, K, ldx, Q, S, stream);
+    if (!rotate) return launch_bf16<false, kActNone>(X, M, K, ldx, Q, S, err, num_sms, stream);
+    switch (act) {
+        case kActRelu: return launch_bf16<true, kActRelu>(X, M, K, ldx, Q, S, err, num_sms, stream);
+        case kActSilu: return launch_bf16<true, kActSilu>(X, M, K, ldx, Q, S, err, num_sms, stream);
+        case kActGeluTanh:
+            return launch_bf16<true, kActGeluTanh>(X, M, K, ldx, Q, S, err, num_sms, stream);
+        default: return launch_bf16<true, kActNone>(X, M, K, ldx, Q, S, err, num_sms, stream);
+    }
 }
 
 cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,
                                   cudaStream_t stream) {
     if (N <= 0) return cudaSuccess;
-    return launch_direct<true>(W, N, K, K, Q, S, stream);
+    return launch_direct<true, kActNone>(W, N, K, K, Q, S, stream);
 }
 
 }  // namespace ck

@@ -77,10 +77,10 @@ uint16_t oracle_f32_to_bf16_rne(float f) {
  * 0.5 x (1 + tanh(u)) and has no cancellation where tanh(u) is near -1.
  *
  * e^x: Cody-Waite reduction x = n ln2 + r with ln2 split in a 16-bit head
- * (n * head is exact for |n| < 256) and a tail, a degree-7 Taylor polynomial
- * of e^r (|r| <= ln2/2, truncation error below 2^-27) in Horner form with
- * separate IEEE multiplies and adds, then an exact scaling by 2^n (two steps
- * when 2^n is subnormal). */
+ * and a tail, each reduction step one fused multiply-add (fmaf: one IEEE
+ * rounding), a degree-7 Taylor polynomial of e^r (|r| <= ln2/2, truncation
+ * error below 2^-27) in Horner form with fused multiply-adds, then an exact
+ * scaling by 2^n (two steps when 2^n is subnormal). */
 #define ACT_NONE 0
 #define ACT_RELU 1
 #define ACT_SILU 2
@@ -102,16 +102,16 @@ float oracle_exp(float x) {
     const float ln2_hi = 0.693145751953125f;
     const float ln2_lo = 1.4286068e-06f;
     float n = nearbyintf(x * log2e);
-    float r = x - n * ln2_hi;
-    r = r - n * ln2_lo;
+    float r = fmaf(-n, ln2_hi, x);
+    r = fmaf(-n, ln2_lo, r);
     float p = 1.984127e-04f; /* 1/7!, 1/6!, ... rounded to fp32 */
-    p = p * r + 1.3888889e-03f;
-    p = p * r + 8.333334e-03f;
-    p = p * r + 4.1666668e-02f;
-    p = p * r + 1.6666667e-01f;
-    p = p * r + 0.5f;
-    p = p * r + 1.0f;
-    p = p * r + 1.0f;
+    p = fmaf(p, r, 1.3888889e-03f);
+    p = fmaf(p, r, 8.333334e-03f);
+    p = fmaf(p, r, 4.1666668e-02f);
+    p = fmaf(p, r, 1.6666667e-01f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
     int k = (int)n;
     if (k > 127)
         return (p * pow2i(127)) * pow2i(k - 127);
@@ -130,7 +130,7 @@ float oracle_act(int act, float x) {
     }
     case ACT_GELU_TANH: {
         float x3 = (x * x) * x;
-        float inner = x + 0.044715f * x3;
+        float inner = fmaf(0.044715f, x3, x);
         float u = 7.978846e-01f * inner; /* sqrt(2/pi) */
         float e = oracle_exp(-2.0f * u);
         return x / (1.0f + e);

@@ -289,3 +289,40 @@ def test_full_size_config(ck, cfg):
 
     acc_rows = ck.test_int8_gemm_i32(Qx[torch.from_numpy(rows[:8]).cuda()].contiguous(), Qw)
     assert np.array_equal(to_np(acc_rows), oracle.gemm_i32(rqx[rows[:8]], rqw))
+
+
+# ------------------------------------------------------------------ input activation
+
+
+def _act_inputs(M, K, seed):
+    cfg = workloads.custom(M, K, 8, seed=seed)
+    X, _, _ = workloads.make_inputs(cfg)
+    x = X.float()
+    x[:, 3] = torch.linspace(-120.0, 120.0, M)  # exp over- and underflow ranges
+    x[::5, 7] = -1.0e4
+    x[1::7, 9] = 3.0e4
+    x[::3] *= 3.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("act", ["relu", "silu", "gelu_tanh"])
+@pytest.mark.parametrize("M,K", [(37, 768), (130, 5376), (9, 28672), (2, 32768), (3, 33024)])
+def test_quantize_rotate_act_bit_exact(ck, act, M, K):
+    X = _act_inputs(M, K, seed=M + K)
+    Qx, s_x = ck.quantize_rotate_rowwise_act(dev(X), act)
+    rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=True, act=act)
+    assert np.array_equal(to_np(s_x).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(to_np(Qx), rq)
+
+
+@pytest.mark.parametrize("act", ["none", "relu", "silu", "gelu_tanh"])
+def test_int8_linear_act_matches_oracle(ck, act):
+    M, K, N = 300, 1024, 264
+    cfg = workloads.custom(M, K, N, seed=31)
+    _, W, bias = workloads.make_inputs(cfg)
+    X = _act_inputs(M, K, seed=32)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    rqw, rsw = oracle.rotate_quant_weight(W.numpy())
+    Y = ck.int8_linear(dev(X), Qw, s_w, dev(bias), input_act=act)
+    Yr = oracle.int8_linear(workloads.bf16_bits(X), rqw, rsw, workloads.bf16_bits(bias), act=act)[0]
+    assert_bf16_close(to_np(Y), Yr)
