@@ -76,6 +76,16 @@ def lib():
             L.oracle_quantize_rows_bf16_act.argtypes = [u16p, i64, i64, i64, ctypes.c_int,
                                                         ctypes.c_int, i8p, f32p]
             L.oracle_quantize_rows_bf16_act.restype = ctypes.c_int
+            L.oracle_quantize_rows_bf16_q.argtypes = [u16p, i64, i64, i64, ctypes.c_int,
+                                                      ctypes.c_int, ctypes.c_float, i8p, f32p]
+            L.oracle_quantize_rows_bf16_q.restype = ctypes.c_int
+            L.oracle_quant_row_q.argtypes = [f32p, i64, ctypes.c_float, i8p, f32p]
+            L.oracle_quant_row_q.restype = None
+            u8p = _P(ctypes.c_uint8)
+            L.oracle_rotate_quant_weight_int4.argtypes = [f32p, i64, i64, u8p, f32p]
+            L.oracle_rotate_quant_weight_int4.restype = ctypes.c_int
+            L.oracle_unpack_int4.argtypes = [u8p, i64, i64, i8p]
+            L.oracle_unpack_int4.restype = None
             L.oracle_exp.argtypes = [ctypes.c_float]
             L.oracle_exp.restype = ctypes.c_float
             L.oracle_act.argtypes = [ctypes.c_int, ctypes.c_float]
@@ -133,8 +143,9 @@ def rot256(v) -> np.ndarray:
     return flat.reshape(a.shape)
 
 
-def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
-    """Per-row symmetric INT8 quantisation of fp32 rows [R, K] (no rotation)."""
+def quant_rows(y, qmax: float = 127.0) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row symmetric quantisation of fp32 rows [R, K] (no rotation) to
+    codes in [-qmax, qmax] (127: INT8, 7: signed INT4 in int8 storage)."""
     y = np.ascontiguousarray(y, dtype=np.float32)
     y2 = y.reshape(-1, y.shape[-1])
     R, K = y2.shape
@@ -145,8 +156,8 @@ def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
         row = np.ascontiguousarray(y2[r])
         qr = np.empty(K, np.int8)
         sr = np.empty(1, np.float32)
-        L.oracle_quant_row(_ptr(row, ctypes.c_float), K, _ptr(qr, ctypes.c_int8),
-                           _ptr(sr, ctypes.c_float))
+        L.oracle_quant_row_q(_ptr(row, ctypes.c_float), K, float(qmax), _ptr(qr, ctypes.c_int8),
+                             _ptr(sr, ctypes.c_float))
         q[r], s[r] = qr, sr[0]
     return q, s
 
@@ -170,7 +181,7 @@ def act(name: str, x) -> np.ndarray:
 
 
 def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = None,
-                       act: str = "none"):
+                       act: str = "none", qmax: float = 127.0):
     """quantize_and_rotate_rowwise (rotate=True) or quantize_int8_rowwise
     (rotate=False) on BF16 rows, optionally after an input activation
     (``act`` in ACTS). ``X_bits`` is uint16 [M, ldx]; the first K columns of
@@ -180,9 +191,9 @@ def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = 
     K = ld if K is None else K
     Qx = np.empty((M, K), np.int8)
     s_x = np.empty(M, np.float32)
-    rc = lib().oracle_quantize_rows_bf16_act(_ptr(X_bits, ctypes.c_uint16), M, K, ld, int(rotate),
-                                             ACTS[act], _ptr(Qx, ctypes.c_int8),
-                                             _ptr(s_x, ctypes.c_float))
+    rc = lib().oracle_quantize_rows_bf16_q(_ptr(X_bits, ctypes.c_uint16), M, K, ld, int(rotate),
+                                           ACTS[act], float(qmax), _ptr(Qx, ctypes.c_int8),
+                                           _ptr(s_x, ctypes.c_float))
     if rc:
         raise ValueError(f"oracle_quantize_rows_bf16 failed ({rc}): K={K} must be a multiple of 256")
     return Qx, s_x
@@ -199,6 +210,39 @@ def rotate_quant_weight(W) -> tuple[np.ndarray, np.ndarray]:
     if rc:
         raise ValueError(f"oracle_rotate_quant_weight failed ({rc})")
     return Qw, s_w
+
+
+def rotate_quant_weight_int4(W) -> tuple[np.ndarray, np.ndarray]:
+    """convrot_w4a4_linear's weight preparation: ConvRot256, per-row signed INT4
+    (s = absmax / 7), two codes per byte (element 2j in the low nibble).
+    Returns (Qw4 uint8 [N, K/2], s_w fp32 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Qw4 = np.empty((N, K // 2), np.uint8)
+    s_w = np.empty(N, np.float32)
+    rc = lib().oracle_rotate_quant_weight_int4(_ptr(W, ctypes.c_float), N, K,
+                                               _ptr(Qw4, ctypes.c_uint8), _ptr(s_w, ctypes.c_float))
+    if rc:
+        raise ValueError(f"oracle_rotate_quant_weight_int4 failed ({rc})")
+    return Qw4, s_w
+
+
+def unpack_int4(Q4: np.ndarray) -> np.ndarray:
+    """Packed INT4 [rows, K/2] -> int8 codes [rows, K]."""
+    Q4 = np.ascontiguousarray(Q4, dtype=np.uint8)
+    rows, half = Q4.shape
+    Q8 = np.empty((rows, 2 * half), np.int8)
+    lib().oracle_unpack_int4(_ptr(Q4, ctypes.c_uint8), rows, 2 * half, _ptr(Q8, ctypes.c_int8))
+    return Q8
+
+
+def convrot_w4a4_linear(X_bits, Qw4, s_w, bias_bits=None):
+    """convrot_w4a4_linear: ConvRot256 + per-row signed INT4 codes of X (in int8
+    storage), the packed INT4 weights unpacked to int8, INT32 GEMM, the same
+    epilogue as int8_linear. Returns (Y bits, Qx, s_x, acc)."""
+    Qx, s_x = quantize_rows_bf16(X_bits, rotate=True, qmax=7.0)
+    acc = gemm_i32(Qx, unpack_int4(Qw4))
+    return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc
 
 
 def gemm_i32(Qx: np.ndarray, Qw: np.ndarray) -> np.ndarray:

@@ -156,15 +156,24 @@ void oracle_rot256(float *v) {
         v[i] = v[i] * 0.0625f;
 }
 
+/* Dynamic symmetric per-row quantisation of one row y[0..K) to codes in
+ * [-qmax, qmax]: qmax = 127 for INT8, 7 for signed INT4 (codes kept in int8
+ * storage). */
+void oracle_quant_row_q(const float *y, int64_t K, float qmax, int8_t *q, float *s_out);
+
 /* Dynamic symmetric per-row INT8 quantisation of one row y[0..K). */
 void oracle_quant_row(const float *y, int64_t K, int8_t *q, float *s_out) {
+    oracle_quant_row_q(y, K, 127.0f, q, s_out);
+}
+
+void oracle_quant_row_q(const float *y, int64_t K, float qmax, int8_t *q, float *s_out) {
     float amax = 0.0f;
     for (int64_t k = 0; k < K; ++k) {
         float a = fabsf(y[k]);
         if (a > amax)
             amax = a;
     }
-    float s = amax / 127.0f;
+    float s = amax / qmax;
     *s_out = s;
     if (amax == 0.0f) {
         memset(q, 0, (size_t)K);
@@ -173,10 +182,10 @@ void oracle_quant_row(const float *y, int64_t K, int8_t *q, float *s_out) {
     for (int64_t k = 0; k < K; ++k) {
         float t = y[k] / s;
         float r = nearbyintf(t); /* default rounding mode: ties to even */
-        if (r > 127.0f)
-            r = 127.0f;
-        if (r < -127.0f)
-            r = -127.0f;
+        if (r > qmax)
+            r = qmax;
+        if (r < -qmax)
+            r = -qmax;
         q[k] = (int8_t)r;
     }
 }
@@ -192,9 +201,18 @@ int oracle_quantize_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t l
     return oracle_quantize_rows_bf16_act(X, M, K, ldx, rotate, ACT_NONE, Qx, s_x);
 }
 
+int oracle_quantize_rows_bf16_q(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                int rotate, int act, float qmax, int8_t *Qx, float *s_x);
+
 /* The same, with the input activation applied first (ACT_NONE: none). */
 int oracle_quantize_rows_bf16_act(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                   int rotate, int act, int8_t *Qx, float *s_x) {
+    return oracle_quantize_rows_bf16_q(X, M, K, ldx, rotate, act, 127.0f, Qx, s_x);
+}
+
+/* ... and with codes in [-qmax, qmax] (7: convrot_w4a4_linear's INT4). */
+int oracle_quantize_rows_bf16_q(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                int rotate, int act, float qmax, int8_t *Qx, float *s_x) {
     if (K % ROT_N != 0 || ldx < K)
         return 1;
     int err = 0;
@@ -217,7 +235,7 @@ int oracle_quantize_rows_bf16_act(const uint16_t *X, int64_t M, int64_t K, int64
                 if (rotate)
                     for (int64_t b = 0; b < K; b += ROT_N)
                         oracle_rot256(buf + b);
-                oracle_quant_row(buf, K, Qx + m * K, s_x + m);
+                oracle_quant_row_q(buf, K, qmax, Qx + m * K, s_x + m);
             }
             free(buf);
         }
@@ -249,6 +267,51 @@ int oracle_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw,
         }
     }
     return err;
+}
+
+/* convrot_w4a4_linear's weights (comfy-kitchen 0.2.40, "Huawei Ascend
+ * backend": ConvRot then signed INT4 quantisation; packed weights are
+ * unpacked to INT8 for INT32 accumulation): each fp32 row rotated, quantised
+ * to [-7, 7] with s = absmax / 7, then packed two codes per byte, element 2j
+ * in the low nibble and 2j + 1 in the high nibble, each nibble the 4-bit
+ * two's complement of its code (the packing order is a reading). */
+int oracle_rotate_quant_weight_int4(const float *W, int64_t N, int64_t K, uint8_t *Qw4,
+                                    float *s_w) {
+    if (K % ROT_N != 0)
+        return 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        float *buf = (float *)malloc((size_t)K * sizeof(float));
+        int8_t *q = (int8_t *)malloc((size_t)K);
+        if (!buf || !q) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t n = 0; n < N; ++n) {
+                memcpy(buf, W + n * K, (size_t)K * sizeof(float));
+                for (int64_t b = 0; b < K; b += ROT_N)
+                    oracle_rot256(buf + b);
+                oracle_quant_row_q(buf, K, 7.0f, q, s_w + n);
+                for (int64_t j = 0; j < K / 2; ++j)
+                    Qw4[n * (K / 2) + j] =
+                        (uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));
+            }
+        }
+        free(buf);
+        free(q);
+    }
+    return err;
+}
+
+/* Packed INT4 [rows, K/2] -> int8 codes [rows, K] (sign-extended nibbles). */
+void oracle_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8) {
+    for (int64_t i = 0; i < rows * (K / 2); ++i) {
+        int lo = Q4[i] & 0xF, hi = Q4[i] >> 4;
+        Q8[2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+        Q8[2 * i + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+    }
 }
 
 /* acc[m][n] = sum_k Qx[m][k] * Qw[n][k], exact in int32 while K * 127^2 < 2^31. */

@@ -22,17 +22,21 @@ MUTATIONS = {
     "round_half_away": ("float r = nearbyintf(t);", "float r = roundf(t);"),
     "truncate": ("float r = nearbyintf(t);", "float r = truncf(t);"),
     "max_without_abs": ("float a = fabsf(y[k]);", "float a = y[k];"),
-    "scale_over_128": ("float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+    "scale_over_qmax_plus_1": ("float s = amax / qmax;", "float s = amax / (qmax + 1.0f);"),
     "gemm_transposed_weight": ("const int8_t *b = Qw + n * K;\n            int32_t s = 0;\n            for (int64_t k = 0; k < K; ++k)\n                s += (int32_t)a[k] * (int32_t)b[k];\n            acc[m * N + n] = s;",
                                "int32_t s = 0;\n            for (int64_t k = 0; k < K; ++k)\n                s += (int32_t)a[k] * (int32_t)Qw[(k % N) * K + (n % K)];\n            acc[m * N + n] = s;"),
     "epilogue_drops_weight_scale": ("    f = f * sw;\n", "    (void)sw;\n"),
     "epilogue_bias_dropped": ("    f = f + b;\n", "    (void)b;\n"),
     "bf16_truncates": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (rest >= 0x8000u)"),
-    "gelu_cubic_coefficient": ("float inner = x + 0.044715f * x3;", "float inner = x + 0.04715f * x3;"),
+    "gelu_cubic_coefficient": ("float inner = fmaf(0.044715f, x3, x);", "float inner = fmaf(0.04715f, x3, x);"),
     "silu_wrong_sign": ("float e = oracle_exp(-x);", "float e = oracle_exp(x);"),
-    "exp_drops_a_term": ("p = p * r + 1.6666667e-01f;", "p = p * r + 0.0f;"),
-    "exp_reduction_head_only": ("r = r - n * ln2_lo;", "r = r - 0.0f;"),
+    "exp_drops_a_term": ("p = fmaf(p, r, 1.6666667e-01f);", "p = fmaf(p, r, 0.0f);"),
+    "exp_reduction_head_only": ("r = fmaf(-n, ln2_lo, r);", "r = r - 0.0f;"),
+    "int4_qmax_8": ("oracle_quant_row_q(buf, K, 7.0f, q, s_w + n);", "oracle_quant_row_q(buf, K, 8.0f, q, s_w + n);"),
+    "int4_nibbles_swapped": ("(uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));",
+                             "(uint8_t)(((uint8_t)q[2 * j + 1] & 0xFu) | (((uint8_t)q[2 * j] & 0xFu) << 4));"),
+    "int4_unpack_no_sign": ("Q8[2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);", "Q8[2 * i] = (int8_t)lo;"),
     "act_not_rounded_to_bf16": ("v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));",
                                 "v = oracle_act(act, v);"),
 }
@@ -51,6 +55,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     env = dict(os.environ, CONVROT_ORACLE_LIB=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_act_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_act_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_w4a4_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
