@@ -218,7 +218,7 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
-def config_dict(cfg, world, scaling="weak", act="none"):
+def config_dict(cfg, world, scaling="weak", act="none", path="int8"):
     par = (f"replicas x{world}: every rank runs the whole batch" if scaling == "weak"
            else f"rows split over {world} ranks")
     return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "seed": cfg.seed,
@@ -226,7 +226,7 @@ def config_dict(cfg, world, scaling="weak", act="none"):
             "parallelism": par + " (rows are independent: no collective on the data path)",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); X is also larger than L2",
             "weights": "rotated + quantised once before timing (offline)",
-            "input_act": act}
+            "input_act": act, "path": path}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -248,7 +248,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         X = X[lo:hi].contiguous()
     Xd = X.to(dev)
     bd = bias.to(dev)
-    Qw, s_w = ck.rotate_quant_weight(W.to(dev))
+    if args.path == "w4a4":
+        Qw4, s_w = ck.rotate_quant_weight_int4(W.to(dev))
+        Qw = torch.empty((cfg.N, cfg.K), dtype=torch.int8, device=dev)
+    else:
+        Qw, s_w = ck.rotate_quant_weight(W.to(dev))
     Wcpu = W
     M, N, K = X.shape[0], cfg.N, cfg.K
     Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
@@ -260,7 +264,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     ck.clear_device_error()
 
     def quantize():
-        if args.act == "none":
+        # convrot_w4a4_linear: INT4 codes of X, then the packed weights unpacked
+        if args.path == "w4a4":
+            ck.quantize_rotate_rowwise_int4(Xd, Qx, s_x)
+            ck.unpack_int4(Qw4, out=Qw)
+        elif args.act == "none":
             ck.quantize_rotate_rowwise(Xd, Qx, s_x)
         else:
             ck.quantize_rotate_rowwise_act(Xd, args.act, Qx, s_x)
@@ -307,7 +315,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     ms_step, ms_q, ms_g = max_over_ranks([ms_step, ms_q, ms_g], dev)
 
     # ---- end to end through the public composite call, host buffers
-    if args.no_e2e:
+    if args.no_e2e or args.path == "w4a4":
         ms_e2e = float("nan")
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
@@ -390,7 +398,7 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
             "scaling": args.scaling,
             "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
             "dtype": "int8", "data": "synthetic", "impl": "ours",
-            "config": config_dict(cfg, world, args.scaling, args.act),
+            "config": config_dict(cfg, world, args.scaling, args.act, args.path),
             "roofline": {"kernel": "gemm_i8_kernel (tcgen05 kind::i8 + fused epilogue)",
                          "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
@@ -403,10 +411,10 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                           "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
                           "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},
             "cpu_baseline": cpu,
-            "e2e": None if args.no_e2e else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
+            "e2e": None if (args.no_e2e or args.path == "w4a4") else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
                     "call": "ck_int8_linear with X copied from pinned host memory and Y copied back"},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (3 if args.path == "w4a4" else 2) * args.steps,
             "clocks": clocks.summary(t_wall0, t_wall1),
         }
     return line
@@ -422,6 +430,9 @@ def main(argv=None):
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: every rank runs the whole batch (replicas); strong: the "
                          "batch's rows are split over the ranks")
+    ap.add_argument("--path", default="int8", choices=["int8", "w4a4"],
+                    help="int8: int8_linear; w4a4: convrot_w4a4_linear (INT4 codes, packed "
+                         "INT4 weights unpacked per step)")
     ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -183,6 +183,42 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
                              ck_stream_t stream);
 
 /*
+ * convrot_w4a4_linear (comfy-kitchen 0.2.40, "Huawei Ascend backend": ConvRot
+ * then signed INT4 quantisation of both operands; activation codes stay in
+ * INT8 storage; packed weights are unpacked to INT8 for INT32 accumulation;
+ * the result is scaled like int8_linear's). Readings: s = absmax / 7, codes
+ * round-half-even(y / s) clamped to [-7, 7]; two weight codes per byte,
+ * element 2j in the low nibble of byte j, each nibble 4-bit two's complement.
+ */
+
+/* Offline: ConvRot256 + per-row signed INT4 of fp32 W [N, K] (16-B aligned).
+ * Qw4 [N, K/2] bytes (16-B aligned), s_w [N] fp32 (16-B aligned). */
+ck_status ck_rotate_quant_weight_int4(const float *W, int64_t N, int64_t K, uint8_t *Qw4,
+                                      float *s_w, ck_stream_t stream);
+
+/* Packed INT4 [N, K/2] -> int8 codes [N, K] (both 16-B aligned). */
+ck_status ck_unpack_int4(const uint8_t *Qw4, int64_t N, int64_t K, int8_t *Qw, ck_stream_t stream);
+
+/* ConvRot256 + per-row signed INT4 codes (in int8 storage, [-7, 7]) of bf16
+ * X; arguments as for ck_quantize_rotate_rowwise. */
+ck_status ck_quantize_rotate_rowwise_int4(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                          int8_t *Qx, float *s_x, ck_stream_t stream);
+
+/* Workspace of ck_convrot_w4a4_linear: activation codes (M*K), row scales
+ * (4*M) and the unpacked weights (N*K), each part rounded up to 256 bytes. */
+size_t ck_convrot_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Y = bf16(((INT32 GEMM of the INT4 codes of rotated X with the unpacked
+ * weights) * s_x) * s_w + bias): the INT4 quantiser, the unpack kernel and
+ * the INT8 tcgen05 GEMM on `stream`. Arguments as for ck_int8_linear, with
+ * Qw4 [N, K/2] packed codes (16-B aligned) and the workspace sized by
+ * ck_convrot_w4a4_linear_workspace_bytes (256-B aligned). */
+ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw4,
+                                 const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                                 int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                                 ck_stream_t stream);
+
+/*
  * The GEMM and fused epilogue alone, on activations already quantised (by
  * ck_quantize_rotate_rowwise):
  *   Qx [M, K] int8 (16-B aligned), s_x [M] fp32 (4-B aligned), Qw/s_w/bias/Y as

@@ -62,6 +62,12 @@ _SIGS = {
     "ck_quantize_rotate_rowwise_act": (_st, [_vp, _i64, _i64, _i64, _st, _vp, _vp, _vp]),
     "ck_int8_linear_act": (_st, [_vp, _i64, _st, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                  ctypes.c_size_t, _vp]),
+    "ck_rotate_quant_weight_int4": (_st, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "ck_unpack_int4": (_st, [_vp, _i64, _i64, _vp, _vp]),
+    "ck_quantize_rotate_rowwise_int4": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ck_convrot_w4a4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "ck_convrot_w4a4_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                     ctypes.c_size_t, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
@@ -244,6 +250,76 @@ def int8_linear_noalloc(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
     ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
     _check(lib.ck_int8_linear_noalloc(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out),
                                       M, N, K, _stream(stream)), "ck_int8_linear_noalloc")
+    return out
+
+
+def rotate_quant_weight_int4(W: torch.Tensor, Qw4: torch.Tensor | None = None,
+                             s_w: torch.Tensor | None = None, stream=None):
+    """Offline: ConvRot256 + per-row signed INT4 of fp32 W [N, K], packed two
+    codes per byte. Returns (Qw4 uint8 [N, K/2], s_w fp32 [N])."""
+    _need(W, "W", torch.float32, 2)
+    _rows_contiguous(W, "W")
+    N, K = W.shape
+    if Qw4 is None:
+        Qw4 = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    if s_w is None:
+        s_w = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _need(Qw4, "Qw4", torch.uint8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    _check(lib.ck_rotate_quant_weight_int4(_ptr(W), N, K, _ptr(Qw4), _ptr(s_w), _stream(stream)),
+           "ck_rotate_quant_weight_int4")
+    return Qw4, s_w
+
+
+def unpack_int4(Qw4: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Packed INT4 [N, K/2] -> int8 codes [N, K]."""
+    _need(Qw4, "Qw4", torch.uint8, 2)
+    _rows_contiguous(Qw4, "Qw4")
+    N, K = Qw4.shape[0], 2 * Qw4.shape[1]
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.int8, device=Qw4.device)
+    _need(out, "out", torch.int8, 2)
+    _check(lib.ck_unpack_int4(_ptr(Qw4), N, K, _ptr(out), _stream(stream)), "ck_unpack_int4")
+    return out
+
+
+def quantize_rotate_rowwise_int4(X: torch.Tensor, Qx=None, s_x=None, stream=None):
+    """ConvRot256 + per-row signed INT4 codes (int8 storage, [-7, 7]) of bf16 X."""
+    return _quant(lib.ck_quantize_rotate_rowwise_int4, "ck_quantize_rotate_rowwise_int4", X, Qx,
+                  s_x, stream)
+
+
+def w4a4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.ck_convrot_w4a4_linear_workspace_bytes(M, N, K))
+
+
+def convrot_w4a4_linear(X: torch.Tensor, Qw4: torch.Tensor, s_w: torch.Tensor,
+                        bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """convrot_w4a4_linear: INT4 codes of rotated X times the unpacked INT4
+    weights, INT32 accumulation, int8_linear's epilogue."""
+    _need(X, "X", torch.bfloat16, 2)
+    _need(Qw4, "Qw4", torch.uint8, 2)
+    _rows_contiguous(Qw4, "Qw4")
+    _need(s_w, "s_w", torch.float32, 1)
+    M, K = X.shape
+    N = Qw4.shape[0]
+    if 2 * Qw4.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch between X, Qw4 and s_w")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    need = w4a4_workspace_bytes(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_convrot_w4a4_linear(_ptr(X), ldx, _ptr(Qw4), _ptr(s_w), _ptr(bias), _ptr(out),
+                                      M, N, K, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream)), "ck_convrot_w4a4_linear")
     return out
 
 

@@ -151,7 +151,7 @@ ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const f
 }
 
 ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8_t *Qx,
-                       float *s_x, bool rotate, int act, ck_stream_t stream) {
+                       float *s_x, bool rotate, int act, ck_stream_t stream, int qmax = 127) {
     if (M < 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
     ck_status s = check_k(K);
     if (s == CK_ERR_INVALID_VALUE) return s;
@@ -164,7 +164,7 @@ ck_status quant_common(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx, int8
     DeviceState *st = nullptr;
     s = device_state(&st);
     if (s != CK_OK) return s;
-    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, act, Qx, s_x, st->err,
+    cudaError_t e = ck::launch_quant_rows_bf16(X, M, K, ldx, rotate, act, qmax, Qx, s_x, st->err,
                                                st->num_sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
@@ -183,12 +183,8 @@ ck_status gemm_args(const int8_t *Qx, const int8_t *Qw, const void *Y, int64_t M
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-}  // namespace
-
-extern "C" {
-
-ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw, float *s_w,
-                                 ck_stream_t stream) {
+ck_status weight_common(const float *W, int64_t N, int64_t K, void *Qw, float *s_w, bool int4,
+                        ck_stream_t stream) {
     if (N < 0) return CK_ERR_INVALID_VALUE;
     ck_status s = check_k(K);
     if (s == CK_ERR_INVALID_VALUE) return s;
@@ -200,9 +196,51 @@ ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Q
     DeviceState *st = nullptr;
     s = device_state(&st);
     if (s != CK_OK) return s;
-    cudaError_t e =
-        ck::launch_quant_rows_f32(W, N, K, Qw, s_w, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = ck::launch_quant_rows_f32(W, N, K, int4, static_cast<int8_t *>(Qw), s_w,
+                                              reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ck_status ck_rotate_quant_weight(const float *W, int64_t N, int64_t K, int8_t *Qw, float *s_w,
+                                 ck_stream_t stream) {
+    return weight_common(W, N, K, Qw, s_w, false, stream);
+}
+
+ck_status ck_rotate_quant_weight_int4(const float *W, int64_t N, int64_t K, uint8_t *Qw4,
+                                      float *s_w, ck_stream_t stream) {
+    return weight_common(W, N, K, Qw4, s_w, true, stream);
+}
+
+ck_status ck_unpack_int4(const uint8_t *Qw4, int64_t N, int64_t K, int8_t *Qw, ck_stream_t stream) {
+    if (N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (N > 0 && (!Qw4 || !Qw)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return CK_OK;
+    if (!aligned16(Qw4) || !aligned16(Qw)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_unpack_int4(Qw4, N, K, Qw, st->num_sms,
+                                           reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status ck_quantize_rotate_rowwise_int4(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                          int8_t *Qx, float *s_x, ck_stream_t stream) {
+    return quant_common(X, M, K, ldx, Qx, s_x, true, CK_ACT_NONE, stream, 7);
+}
+
+size_t ck_convrot_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return round256(size_t(M) * size_t(K)) + round256(size_t(M) * 4) +
+           round256(size_t(N) * size_t(K));
 }
 
 ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
@@ -255,7 +293,7 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
                                            round256(size_t(M) * size_t(K)));
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e =
-        ck::launch_quant_rows_bf16(X, M, K, ldx, true, act, Qx, s_x, st->err, st->num_sms, cs);
+        ck::launch_quant_rows_bf16(X, M, K, ldx, true, act, 127, Qx, s_x, st->err, st->num_sms, cs);
     if (e != cudaSuccess) return CK_ERR_CUDA;
     return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
 }
@@ -265,6 +303,40 @@ ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const 
                          void *workspace, size_t workspace_bytes, ck_stream_t stream) {
     return ck_int8_linear_act(X, ldx, CK_ACT_NONE, Qw, s_w, bias, Y, M, N, K, workspace,
                               workspace_bytes, stream);
+}
+
+ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw4,
+                                 const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
+                                 int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                                 ck_stream_t stream) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && N > 0 && (!X || !Qw4 || !s_w || !Y || !workspace)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Qw4) || !aligned16(s_w) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CK_ERR_MISALIGNED;
+    if (workspace_bytes < ck_convrot_w4a4_linear_workspace_bytes(M, N, K)) return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    int8_t *Qx = reinterpret_cast<int8_t *>(base);
+    float *s_x = reinterpret_cast<float *>(base + round256(size_t(M) * size_t(K)));
+    int8_t *Qw = reinterpret_cast<int8_t *>(base + round256(size_t(M) * size_t(K)) +
+                                            round256(size_t(M) * 4));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e =
+        ck::launch_quant_rows_bf16(X, M, K, ldx, true, CK_ACT_NONE, 7, Qx, s_x, st->err, st->num_sms, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    e = ck::launch_unpack_int4(Qw4, N, K, Qw, st->num_sms, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
 }
 
 ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t *Qw,

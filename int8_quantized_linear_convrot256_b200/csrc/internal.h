@@ -12,14 +12,20 @@ namespace ck {
 // Rows of bf16 (bit patterns) with row stride ldx; rotate=false skips ConvRot.
 // err is the device error word (bounded waits of the staged variant).
 // act: input activation applied before the rotation (0 none, 1 relu, 2 silu,
-// 3 tanh-form gelu); only with rotate.
+// 3 tanh-form gelu); only with rotate. qmax: 127 (INT8 codes) or 7 (signed
+// INT4 codes in int8 storage, rotate only, no act).
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   bool rotate, int act, int8_t *Q, float *S, unsigned *err,
-                                   int num_sms, cudaStream_t stream);
+                                   bool rotate, int act, int qmax, int8_t *Q, float *S,
+                                   unsigned *err, int num_sms, cudaStream_t stream);
 
-// Rows of fp32 with row stride K (offline weight preparation), always rotated.
-cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,
-                                  cudaStream_t stream);
+// Rows of fp32 with row stride K (offline weight preparation), always rotated;
+// int4_packed: signed INT4 codes packed two per byte into Q [N, K/2].
+cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int4_packed,
+                                  int8_t *Q, float *S, cudaStream_t stream);
+
+// Packed signed INT4 [rows, K/2] -> int8 [rows, K].
+cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8,
+                               int num_sms, cudaStream_t stream);
 
 // ---- tcgen05 INT8 GEMM with fused epilogue (gemm_i8_tcgen05.cu)
 

@@ -374,25 +374,30 @@ struct RowQuant {
     float rc;     // fl(1 / div) when fast
     bool fast;    // reciprocal path with the near-half-integer fallback
     bool scale16; // exact path must first form y = fl(z / 16)
+    float qmax;   // codes lie in [-qmax, qmax]
 };
 
-template <bool kRotate>
+// kQ = 127: INT8 codes; kQ = 7: signed INT4 codes (convrot_w4a4_linear). The
+// reciprocal fast path's bound holds a fortiori for |z / d| <= 7.
+template <bool kRotate, int kQ = 127>
 __device__ __forceinline__ RowQuant row_quant(float amax) {
     RowQuant r;
+    const float qmax = float(kQ);
+    r.qmax = qmax;
     if (kRotate) {
         if (amax >= kMinFoldAmax) {
-            r.div = __fdiv_rn(amax, 127.0f);
+            r.div = __fdiv_rn(amax, qmax);
             r.s = __fmul_rn(r.div, 0.0625f);
             r.fast = true;
             r.scale16 = false;
         } else {
-            r.s = __fdiv_rn(__fmul_rn(amax, 0.0625f), 127.0f);
+            r.s = __fdiv_rn(__fmul_rn(amax, 0.0625f), qmax);
             r.div = r.s;
             r.fast = false;
             r.scale16 = true;
         }
     } else {
-        r.s = __fdiv_rn(amax, 127.0f);
+        r.s = __fdiv_rn(amax, qmax);
         r.div = r.s;
         r.fast = r.s >= kMinFastScale;
         r.scale16 = false;
@@ -407,7 +412,7 @@ __device__ __forceinline__ uint32_t code_exact(float z, const RowQuant &rq) {
     if (rq.div == 0.0f) return __float_as_uint(kMagic);
     const float y = rq.scale16 ? __fmul_rn(z, 0.0625f) : z;
     float q = rintf(__fdiv_rn(y, rq.div));
-    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    q = fminf(fmaxf(q, -rq.qmax), rq.qmax);
     return __float_as_uint(__fadd_rn(q, kMagic));
 }
 
@@ -417,11 +422,29 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
     return __byte_perm(ab, cd, 0x5410);
 }
 
+// Stores the 8 codes of group i: 8 int8 bytes at qbase + 32 i, or (kPack4)
+// 8 signed nibbles in one 32-bit word at qbase + 16 i, element 2j in the low
+// nibble of byte j. qbase already points at this lane's first element (or
+// its packed byte).
+template <bool kPack4>
+__device__ __forceinline__ void store_group(const uint32_t (&u)[8], int i, int8_t *qbase) {
+    const uint32_t lo = pack4(u[0], u[1], u[2], u[3]);
+    const uint32_t hi = pack4(u[4], u[5], u[6], u[7]);
+    if (!kPack4) {
+        *reinterpret_cast<uint2 *>(qbase + 32 * i) = make_uint2(lo, hi);
+    } else {
+        const uint32_t a = lo & 0x0F0F0F0Fu, b = hi & 0x0F0F0F0Fu;
+        const uint32_t a2 = a | (a >> 4), b2 = b | (b >> 4);  // byte pairs -> one byte each
+        *reinterpret_cast<uint32_t *>(qbase + 16 * i) = __byte_perm(a2, b2, 0x6420);
+    }
+}
+
 // Quantise lane t's 64 values and store the codes: group i (pairs 4i..4i+3)
 // holds elements 8t + 32i .. +7, stored as 8 contiguous bytes. The fast path
 // stores every group without branching and records which groups hold a value
 // near a half-integer; those (rare) groups are then recomputed exactly and
 // stored again.
+template <bool kPack4>
 __device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int i,
                                                   const RowQuant &rq, int8_t *qbase) {
     uint32_t u[8];
@@ -430,17 +453,15 @@ __device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int
         u[2 * k] = code_exact(P[4 * i + k].x, rq);
         u[2 * k + 1] = code_exact(P[4 * i + k].y, rq);
     }
-    uint2 out;
-    out.x = pack4(u[0], u[1], u[2], u[3]);
-    out.y = pack4(u[4], u[5], u[6], u[7]);
-    *reinterpret_cast<uint2 *>(qbase + 32 * i) = out;
+    store_group<kPack4>(u, i, qbase);
 }
 
+template <bool kPack4 = false>
 __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const RowQuant &rq,
                                                int8_t *qbase) {
     if (!rq.fast) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) store_group_exact(P, i, rq, qbase);
+        for (int i = 0; i < 8; ++i) store_group_exact<kPack4>(P, i, rq, qbase);
         return;
     }
     const float2 rc2 = make_float2(rq.rc, rq.rc);
@@ -462,22 +483,19 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const 
             u[2 * k + 1] = __float_as_uint(m.y);
         }
         redo |= uint32_t(dmax >= kNearHalf) << i;
-        uint2 out;
-        out.x = pack4(u[0], u[1], u[2], u[3]);
-        out.y = pack4(u[4], u[5], u[6], u[7]);
-        *reinterpret_cast<uint2 *>(qbase + 32 * i) = out;
+        store_group<kPack4>(u, i, qbase);
     }
     if (redo) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            if (redo & (1u << i)) store_group_exact(P, i, rq, qbase);
+            if (redo & (1u << i)) store_group_exact<kPack4>(P, i, rq, qbase);
     }
 }
 
 // ------------------------------------------------------------------ kernels
 
 // Single pass with direct loads: CTA = rows_per_cta rows x (K/256) quads.
-template <bool kRotate, int kAct, typename TIn>
+template <bool kRotate, int kAct, int kQ, bool kPack4, typename TIn>
 __global__ void __launch_bounds__(kMaxThreads, 1)
 quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
                   int8_t *__restrict__ Q, float *__restrict__ S) {
@@ -504,9 +522,12 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     if (active && t == 0) atomicMax(&s_amax[row_local], __float_as_uint(m));
     __syncthreads();
     if (!active) return;
-    const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax[row_local]));
+    const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[row_local]));
     if (blk == 0 && t == 0) S[row] = rq.s;
-    quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0);
+    if (kPack4)
+        quantize_store<true>(P, rq, Q + row * static_cast<int64_t>(K / 2) + col0 / 2);
+    else
+        quantize_store<false>(P, rq, Q + row * static_cast<int64_t>(K) + col0);
 }
 
 // Persistent single pass for BF16 rows: row groups are staged into shared
@@ -514,7 +535,7 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
 // group: after it, every thread has read its values out of the buffer (so the
 // buffer can be refilled) and the row absmax is complete. The absmax slots are
 // triple-buffered so a slot is cleared one full barrier before its next use.
-template <bool kRotate, int kAct>
+template <bool kRotate, int kAct, int kQ>
 __global__ void __launch_bounds__(kMaxThreads, 1)
 quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
                        int rows_per_cta, int8_t *__restrict__ Q, float *__restrict__ S,
@@ -603,7 +624,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const int clear = slot == 0 ? 2 : slot - 1;  // (i + 2) % 3
         if (tid < R) s_amax[clear][tid] = 0u;
         if (active) {
-            const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax[slot][row_local]));
+            const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[slot][row_local]));
             if (blk == 0 && t == 0) S[row] = rq.s;
             quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0);
         }
@@ -614,7 +635,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
 // Two passes for long rows (K > 32768): one CTA per row, 128 quads; pass 1
 // rotates every block and reduces the absmax, pass 2 reloads (from L2),
 // rotates again and quantises.
-template <bool kRotate, int kAct, typename TIn>
+template <bool kRotate, int kAct, int kQ, bool kPack4, typename TIn>
 __global__ void __launch_bounds__(kTwoPassQuads * 4, 1)
 quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx,
                            int8_t *__restrict__ Q, float *__restrict__ S) {
@@ -640,7 +661,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
     __syncthreads();
     if (t == 0) atomicMax(&s_amax, __float_as_uint(m));
     __syncthreads();
-    const RowQuant rq = row_quant<kRotate>(__uint_as_float(s_amax));
+    const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax));
     if (tid == 0) S[row] = rq.s;
     for (int b0 = 0; b0 < nb; b0 += kTwoPassQuads) {
         const int blk = b0 + quad;
@@ -650,7 +671,13 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
         else
             zero_block(P);
         if (kRotate) butterflies(P, t);
-        if (blk < nb) quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + blk * kBlock + 8 * t);
+        if (blk < nb) {
+            if (kPack4)
+                quantize_store<true>(P, rq, Q + row * static_cast<int64_t>(K / 2) +
+                                                (blk * kBlock + 8 * t) / 2);
+            else
+                quantize_store<false>(P, rq, Q + row * static_cast<int64_t>(K) + blk * kBlock + 8 * t);
+        }
     }
 }
 
@@ -682,21 +709,21 @@ std::mutex g_occ_mutex;
 // (device, rotate, threads, smem) -> CTAs of the bulk kernel per SM
 std::map<std::tuple<int, int, int, size_t>, int> g_bulk_occupancy;
 
-template <bool kRotate, int kAct>
+template <bool kRotate, int kAct, int kQ>
 cudaError_t bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
     std::lock_guard<std::mutex> lock(g_occ_mutex);
-    const auto key = std::make_tuple(dev, (kRotate ? 1 : 0) + 2 * kAct, threads, smem);
+    const auto key = std::make_tuple(dev, (kRotate ? 1 : 0) + 2 * kAct + 16 * kQ, threads, smem);
     auto it = g_bulk_occupancy.find(key);
     if (it != g_bulk_occupancy.end()) {
         *out = it->second;
         return cudaSuccess;
     }
-    cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel<kRotate, kAct>,
+    cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel<kRotate, kAct, kQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kBulkSmemBudget));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_bulk_kernel<kRotate, kAct>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_bulk_kernel<kRotate, kAct, kQ>,
                                                       threads, smem);
     if (e != cudaSuccess) return e;
     g_bulk_occupancy[key] = per_sm;
@@ -704,7 +731,7 @@ cudaError_t bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
     return cudaSuccess;
 }
 
-template <bool kRotate, int kAct>
+template <bool kRotate, int kAct, int kQ>
 cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
                         unsigned *err, int num_sms, cudaStream_t stream, bool *launched) {
     *launched = false;
@@ -718,19 +745,19 @@ cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, in
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = bulk_blocks_per_sm<kRotate, kAct>(dev, threads, smem, &per_sm);
+    e = bulk_blocks_per_sm<kRotate, kAct, kQ>(dev, threads, smem, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaSuccess;
     const int64_t groups = (M + rows - 1) / rows;
     const int64_t cap = int64_t(per_sm) * num_sms;
     const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
-    quant_rows_bulk_kernel<kRotate, kAct><<<grid, threads, smem, stream>>>(
+    quant_rows_bulk_kernel<kRotate, kAct, kQ><<<grid, threads, smem, stream>>>(
         X, M, static_cast<int>(K), ldx, rows, Q, S, err, kDefaultWaitLimitNs);
     *launched = true;
     return cudaGetLastError();
 }
 
-template <bool kRotate, int kAct, typename TIn>
+template <bool kRotate, int kAct, int kQ, bool kPack4, typename TIn>
 cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
                           cudaStream_t stream) {
     const int nb = static_cast<int>(K / kBlock);
@@ -738,32 +765,55 @@ cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_
         int threads = 0;
         const int rows = pick_rows_per_cta(nb, kMaxRowsPerCta, &threads);
         const int64_t grid = (M + rows - 1) / rows;
-        quant_rows_kernel<kRotate, kAct, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
+        quant_rows_kernel<kRotate, kAct, kQ, kPack4, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
             X, M, static_cast<int>(K), ldx, rows, Q, S);
     } else {
-        quant_rows_two_pass_kernel<kRotate, kAct, TIn>
+        quant_rows_two_pass_kernel<kRotate, kAct, kQ, kPack4, TIn>
             <<<static_cast<unsigned>(M), kTwoPassQuads * 4, 0, stream>>>(
                 X, M, static_cast<int>(K), ldx, Q, S);
     }
     return cudaGetLastError();
 }
 
-template <bool kRotate, int kAct>
+template <bool kRotate, int kAct, int kQ = 127>
 cudaError_t launch_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int8_t *Q, float *S,
                         unsigned *err, int num_sms, cudaStream_t stream) {
     bool launched = false;
-    cudaError_t e = launch_bulk<kRotate, kAct>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched);
+    cudaError_t e =
+        launch_bulk<kRotate, kAct, kQ>(X, M, K, ldx, Q, S, err, num_sms, stream, &launched);
     if (e != cudaSuccess || launched) return e;
-    return launch_direct<kRotate, kAct>(X, M, K, ldx, Q, S, stream);
+    return launch_direct<kRotate, kAct, kQ, false>(X, M, K, ldx, Q, S, stream);
+}
+
+// Packed signed INT4 [rows, K/2] -> int8 codes [rows, K]: 16 bytes in, 32 out
+// per thread; nibbles sign-extended per byte ((x ^ 8) - 8, byte-wise SIMD).
+__global__ void unpack_int4_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out,
+                                   int64_t n16) {
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const uint4 v = __ldcs(in + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = __vsub4((w[j] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+            const uint32_t hi = __vsub4(((w[j] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+            o[2 * j] = __byte_perm(lo, hi, 0x5140);
+            o[2 * j + 1] = __byte_perm(lo, hi, 0x7362);
+        }
+        out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   bool rotate, int act, int8_t *Q, float *S, unsigned *err,
-                                   int num_sms, cudaStream_t stream) {
+                                   bool rotate, int act, int qmax, int8_t *Q, float *S,
+                                   unsigned *err, int num_sms, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (!rotate) return launch_bf16<false, kActNone>(X, M, K, ldx, Q, S, err, num_sms, stream);
+    if (qmax == 7) return launch_bf16<true, kActNone, 7>(X, M, K, ldx, Q, S, err, num_sms, stream);
     switch (act) {
         case kActRelu: return launch_bf16<true, kActRelu>(X, M, K, ldx, Q, S, err, num_sms, stream);
         case kActSilu: return launch_bf16<true, kActSilu>(X, M, K, ldx, Q, S, err, num_sms, stream);
@@ -773,10 +823,22 @@ cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int6
     }
 }
 
-cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, int8_t *Q, float *S,
-                                  cudaStream_t stream) {
+cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int4_packed,
+                                  int8_t *Q, float *S, cudaStream_t stream) {
     if (N <= 0) return cudaSuccess;
-    return launch_direct<true, kActNone>(W, N, K, K, Q, S, stream);
+    if (int4_packed) return launch_direct<true, kActNone, 7, true>(W, N, K, K, Q, S, stream);
+    return launch_direct<true, kActNone, 127, false>(W, N, K, K, Q, S, stream);
+}
+
+cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8,
+                               int num_sms, cudaStream_t stream) {
+    const int64_t n16 = rows * (K / 2) / 16;  // K % 256 == 0: whole 16-byte chunks
+    if (n16 <= 0) return cudaSuccess;
+    const int64_t want = (n16 + 255) / 256;
+    const int64_t cap = int64_t(num_sms) * 8;
+    unpack_int4_kernel<<<unsigned(want < cap ? want : cap), 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(Q4), reinterpret_cast<uint4 *>(Q8), n16);
+    return cudaGetLastError();
 }
 
 }  // namespace ck

@@ -326,3 +326,59 @@ def test_int8_linear_act_matches_oracle(ck, act):
     Y = ck.int8_linear(dev(X), Qw, s_w, dev(bias), input_act=act)
     Yr = oracle.int8_linear(workloads.bf16_bits(X), rqw, rsw, workloads.bf16_bits(bias), act=act)[0]
     assert_bf16_close(to_np(Y), Yr)
+
+
+# ------------------------------------------------------------------ convrot_w4a4_linear
+
+
+@pytest.mark.parametrize("M,K", [(37, 768), (130, 5376), (9, 28672), (3, 33024)])
+def test_quantize_rotate_int4_bit_exact(ck, M, K):
+    cfg = workloads.custom(M, K, 8, seed=M + 3 * K)
+    X, _, _ = workloads.make_inputs(cfg)
+    Qx, s_x = ck.quantize_rotate_rowwise_int4(dev(X))
+    rq, rs = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=True, qmax=7)
+    assert np.array_equal(to_np(s_x).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(to_np(Qx), rq)
+
+
+@pytest.mark.parametrize("N,K", [(8, 256), (264, 768), (520, 5376), (16, 33024)])
+def test_rotate_quant_weight_int4_bit_exact(ck, N, K):
+    cfg = workloads.custom(1, K, N, seed=N + 5 * K)
+    _, W, _ = workloads.make_inputs(cfg)
+    Qw4, s_w = ck.rotate_quant_weight_int4(dev(W))
+    r4, rs = oracle.rotate_quant_weight_int4(W.numpy())
+    assert np.array_equal(to_np(s_w).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(to_np(Qw4), r4)
+
+
+def test_unpack_int4_bit_exact(ck):
+    rng = np.random.default_rng(11)
+    b = rng.integers(0, 256, size=(300, 2048), dtype=np.uint8)
+    b[0, :256] = np.arange(256, dtype=np.uint8)
+    got = to_np(ck.unpack_int4(dev(torch.from_numpy(b))))
+    assert np.array_equal(got, oracle.unpack_int4(b))
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 8), (300, 1024, 264), (129, 5376, 520)])
+def test_convrot_w4a4_linear_matches_oracle(ck, M, K, N):
+    cfg = workloads.custom(M, K, N, seed=M + K + 7 * N)
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw4, s_w = ck.rotate_quant_weight_int4(dev(W))
+    r4, rs = oracle.rotate_quant_weight_int4(W.numpy())
+    Y = ck.convrot_w4a4_linear(dev(X), Qw4, s_w, dev(bias))
+    Yr = oracle.convrot_w4a4_linear(workloads.bf16_bits(X), r4, rs, workloads.bf16_bits(bias))[0]
+    assert_bf16_close(to_np(Y), Yr)
+
+
+@pytest.mark.slow
+def test_convrot_w4a4_linear_full_size_sampled_rows(ck):
+    cfg = workloads.CONFIGS[1]  # ragged M8193/K5376/N16128
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw4, s_w = ck.rotate_quant_weight_int4(dev(W))
+    r4, rs = oracle.rotate_quant_weight_int4(W.numpy())
+    assert np.array_equal(to_np(Qw4), r4)
+    Y = ck.convrot_w4a4_linear(dev(X), Qw4, s_w, dev(bias))
+    rows = _sample_rows(cfg.M)
+    Qx, s_x = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=True, qmax=7)
+    Yr = oracle.linear_rows(Qx, s_x, oracle.unpack_int4(r4), rs, workloads.bf16_bits(bias), rows)
+    assert_bf16_close(to_np(Y[torch.from_numpy(rows).cuda()]), Yr)
