@@ -144,6 +144,29 @@ ck_status ck_quantize_rotate_rowwise_act(const ck_bf16 *X, int64_t M, int64_t K,
                                          int act, int8_t *Qx, float *s_x, ck_stream_t stream);
 
 /*
+ * dequantize_int8_simple / dequantize_int8_simple_dtype (comfy-kitchen 0.2.40,
+ * "Huawei Ascend backend"): Y[m][k] = float(Q[m][k]) * s, one fp32 rounding,
+ * with s = s[0] for the whole tensor (per_row == 0) or s[m] per row
+ * (per_row != 0). out_bf16 == 0 stores fp32 Y [rows, K]; otherwise the
+ * product is rounded to bf16 (the _dtype form). Q 16-B aligned, K % 16 == 0,
+ * s 4-B aligned, Y 16-B aligned.
+ */
+ck_status ck_dequantize_int8(const int8_t *Q, const float *s, int64_t rows, int64_t K,
+                             int per_row, int out_bf16, void *Y, ck_stream_t stream);
+
+/*
+ * quantize_int8_tensorwise (same page): one scale for the whole tensor,
+ * s = absmax(X) / 127, Q = round-half-even(X / s) clamped to [-127, 127]; a
+ * zero tensor gives s = 0 and zero codes. No rotation (quantising this way
+ * before ConvRot is the ~16% error negative control of the
+ * ComfyUI-AppleSilicon-FP8 README, row 17). X [M, K] bf16 with row stride ldx
+ * (16-B aligned rows, K % 8 == 0), Q [M, K] int8, s one fp32 (its memory is
+ * also used for the absmax while the three kernels run).
+ */
+ck_status ck_quantize_int8_tensorwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                      int8_t *Q, float *s, ck_stream_t stream);
+
+/*
  * Bytes of device workspace ck_int8_linear needs for M rows of K features:
  * the INT8 codes (M*K bytes) and the row scales (4*M bytes), each part
  * rounded up to 256 bytes. Returns 0 for M <= 0 or K <= 0.

@@ -68,6 +68,8 @@ _SIGS = {
     "ck_convrot_w4a4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "ck_convrot_w4a4_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                      ctypes.c_size_t, _vp]),
+    "ck_dequantize_int8": (_st, [_vp, _vp, _i64, _i64, _st, _st, _vp, _vp]),
+    "ck_quantize_int8_tensorwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
@@ -321,6 +323,40 @@ def convrot_w4a4_linear(X: torch.Tensor, Qw4: torch.Tensor, s_w: torch.Tensor,
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "ck_convrot_w4a4_linear")
     return out
+
+
+def dequantize_int8(Q: torch.Tensor, s: torch.Tensor, per_row: bool = True,
+                    dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """dequantize_int8_simple (fp32) / _dtype (bf16): float(Q) * s."""
+    _need(Q, "Q", torch.int8, 2)
+    _rows_contiguous(Q, "Q")
+    _need(s, "s", torch.float32, 1)
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("dtype must be float32 or bfloat16")
+    rows, K = Q.shape
+    if out is None:
+        out = torch.empty((rows, K), dtype=dtype, device=Q.device)
+    _need(out, "out", dtype, 2)
+    _check(lib.ck_dequantize_int8(_ptr(Q), _ptr(s), rows, K, int(per_row),
+                                  int(dtype == torch.bfloat16), _ptr(out), _stream(stream)),
+           "ck_dequantize_int8")
+    return out
+
+
+def quantize_int8_tensorwise(X: torch.Tensor, Q: torch.Tensor | None = None,
+                             s: torch.Tensor | None = None, stream=None):
+    """quantize_int8_tensorwise: one scale for the whole bf16 tensor."""
+    _need(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    if Q is None:
+        Q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if s is None:
+        s = torch.empty((1,), dtype=torch.float32, device=X.device)
+    _check(lib.ck_quantize_int8_tensorwise(_ptr(X), M, K, ldx, _ptr(Q), _ptr(s), _stream(stream)),
+           "ck_quantize_int8_tensorwise")
+    return Q, s
 
 
 def int8_gemm_rowscale(Qx: torch.Tensor, s_x: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,

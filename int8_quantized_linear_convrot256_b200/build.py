@@ -33,8 +33,9 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
           "-ftz=false", "-prec-div=true", "-prec-sqrt=true"]
 PER_FILE = {
     "quant_rotate.cu": ["-fmad=false"],
+    "dequant.cu": ["-fmad=false"],
 }
-SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "noalloc.cu", "dequant.cu"]
 HEADERS = ["ck_device.cuh", "internal.h", "libck.map"]
 
 

@@ -237,6 +237,36 @@ ck_status ck_quantize_rotate_rowwise_int4(const ck_bf16 *X, int64_t M, int64_t K
     return quant_common(X, M, K, ldx, Qx, s_x, true, CK_ACT_NONE, stream, 7);
 }
 
+ck_status ck_dequantize_int8(const int8_t *Q, const float *s, int64_t rows, int64_t K,
+                             int per_row, int out_bf16, void *Y, ck_stream_t stream) {
+    if (rows < 0 || K <= 0) return CK_ERR_INVALID_VALUE;
+    if (rows > 0 && (!Q || !s || !Y)) return CK_ERR_INVALID_VALUE;
+    if (K % 16 != 0) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0) return CK_OK;
+    if (!aligned16(Q) || !aligned4(s) || !aligned16(Y)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    ck_status st_ = device_state(&st);
+    if (st_ != CK_OK) return st_;
+    cudaError_t e = ck::launch_dequantize_int8(Q, s, rows, K, per_row != 0, out_bf16 != 0, Y,
+                                               st->num_sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status ck_quantize_int8_tensorwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                      int8_t *Q, float *s, ck_stream_t stream) {
+    if (M < 0 || K <= 0 || ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && (!X || !Q || !s)) return CK_ERR_INVALID_VALUE;
+    if (K % 8 != 0) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return CK_OK;
+    if (!aligned16(X) || !aligned16(Q) || !aligned4(s) || ldx % 8 != 0) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    ck_status st_ = device_state(&st);
+    if (st_ != CK_OK) return st_;
+    cudaError_t e = ck::launch_quantize_int8_tensorwise(X, M, K, ldx, Q, s, st->num_sms,
+                                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
 size_t ck_convrot_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
     return round256(size_t(M) * size_t(K)) + round256(size_t(M) * 4) +

@@ -27,6 +27,16 @@ cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int
 cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8,
                                int num_sms, cudaStream_t stream);
 
+// ---- dequantize_int8_simple(_dtype), quantize_int8_tensorwise (dequant.cu)
+
+cudaError_t launch_dequantize_int8(const int8_t *Q, const float *S, int64_t rows, int64_t K,
+                                   bool per_row, bool out_bf16, void *Y, int num_sms,
+                                   cudaStream_t stream);
+
+// s receives the tensor's scale (used as scratch for the absmax first).
+cudaError_t launch_quantize_int8_tensorwise(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                            int8_t *Q, float *s, int num_sms, cudaStream_t stream);
+
 // ---- tcgen05 INT8 GEMM with fused epilogue (gemm_i8_tcgen05.cu)
 
 struct GemmParams {

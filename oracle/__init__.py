@@ -86,6 +86,10 @@ def lib():
             L.oracle_rotate_quant_weight_int4.restype = ctypes.c_int
             L.oracle_unpack_int4.argtypes = [u8p, i64, i64, i8p]
             L.oracle_unpack_int4.restype = None
+            L.oracle_dequantize_int8.argtypes = [i8p, f32p, i64, i64, ctypes.c_int, f32p, u16p]
+            L.oracle_dequantize_int8.restype = None
+            L.oracle_quantize_int8_tensorwise.argtypes = [u16p, i64, i64, i64, i8p, f32p]
+            L.oracle_quantize_int8_tensorwise.restype = None
             L.oracle_exp.argtypes = [ctypes.c_float]
             L.oracle_exp.restype = ctypes.c_float
             L.oracle_act.argtypes = [ctypes.c_int, ctypes.c_float]
@@ -243,6 +247,29 @@ def convrot_w4a4_linear(X_bits, Qw4, s_w, bias_bits=None):
     Qx, s_x = quantize_rows_bf16(X_bits, rotate=True, qmax=7.0)
     acc = gemm_i32(Qx, unpack_int4(Qw4))
     return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc
+
+
+def dequantize_int8(Q, s, per_row: bool = True):
+    """dequantize_int8_simple(_dtype): returns (fp32 [rows, K], bf16 bits [rows, K])."""
+    Q = np.ascontiguousarray(Q, dtype=np.int8)
+    s = np.ascontiguousarray(np.atleast_1d(s), dtype=np.float32)
+    rows, K = Q.shape
+    Yf = np.empty((rows, K), np.float32)
+    Yb = np.empty((rows, K), np.uint16)
+    lib().oracle_dequantize_int8(_ptr(Q, ctypes.c_int8), _ptr(s, ctypes.c_float), rows, K,
+                                 int(per_row), _ptr(Yf, ctypes.c_float), _ptr(Yb, ctypes.c_uint16))
+    return Yf, Yb
+
+
+def quantize_int8_tensorwise(X_bits):
+    """quantize_int8_tensorwise on BF16 X: returns (Q int8 [M, K], s fp32 scalar)."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    Q = np.empty((M, K), np.int8)
+    s = np.empty(1, np.float32)
+    lib().oracle_quantize_int8_tensorwise(_ptr(X_bits, ctypes.c_uint16), M, K, K,
+                                          _ptr(Q, ctypes.c_int8), _ptr(s, ctypes.c_float))
+    return Q, s[0]
 
 
 def gemm_i32(Qx: np.ndarray, Qw: np.ndarray) -> np.ndarray:

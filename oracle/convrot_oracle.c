@@ -314,6 +314,53 @@ void oracle_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8) 
     }
 }
 
+/* dequantize_int8_simple / dequantize_int8_simple_dtype (comfy-kitchen 0.2.40,
+ * "Huawei Ascend backend"): y = float(q) * s, one fp32 rounding, with s one
+ * scale for the tensor (per_row == 0: s[0]) or one per row (s[m]); the dtype
+ * form rounds y to bf16. Yf and/or Yb may be NULL. (Readings: the page lists
+ * the names only.) */
+void oracle_dequantize_int8(const int8_t *Q, const float *s, int64_t rows, int64_t K, int per_row,
+                            float *Yf, uint16_t *Yb) {
+    for (int64_t m = 0; m < rows; ++m) {
+        float sc = per_row ? s[m] : s[0];
+        for (int64_t k = 0; k < K; ++k) {
+            float y = (float)Q[m * K + k] * sc;
+            if (Yf)
+                Yf[m * K + k] = y;
+            if (Yb)
+                Yb[m * K + k] = oracle_f32_to_bf16_rne(y);
+        }
+    }
+}
+
+/* quantize_int8_tensorwise (same page): one scale s = absmax(X) / 127 for the
+ * whole tensor, q = round-half-even(x / s) clamped to [-127, 127]; a zero
+ * tensor gets s = 0 and zero codes. No rotation. */
+void oracle_quantize_int8_tensorwise(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                     int8_t *Q, float *s_out) {
+    float amax = 0.0f;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(oracle_bf16_to_f32(X[m * ldx + k]));
+            if (a > amax)
+                amax = a;
+        }
+    float s = amax / 127.0f;
+    *s_out = s;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            float r = 0.0f;
+            if (amax != 0.0f) {
+                r = nearbyintf(oracle_bf16_to_f32(X[m * ldx + k]) / s);
+                if (r > 127.0f)
+                    r = 127.0f;
+                if (r < -127.0f)
+                    r = -127.0f;
+            }
+            Q[m * K + k] = (int8_t)r;
+        }
+}
+
 /* acc[m][n] = sum_k Qx[m][k] * Qw[n][k], exact in int32 while K * 127^2 < 2^31. */
 void oracle_gemm_i32(const int8_t *Qx, const int8_t *Qw, int64_t M, int64_t N, int64_t K,
                      int32_t *acc) {

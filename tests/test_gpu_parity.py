@@ -382,3 +382,33 @@ def test_convrot_w4a4_linear_full_size_sampled_rows(ck):
     Qx, s_x = oracle.quantize_rows_bf16(workloads.bf16_bits(X), rotate=True, qmax=7)
     Yr = oracle.linear_rows(Qx, s_x, oracle.unpack_int4(r4), rs, workloads.bf16_bits(bias), rows)
     assert_bf16_close(to_np(Y[torch.from_numpy(rows).cuda()]), Yr)
+
+
+# ------------------------------------------------------------------ dequantize / tensorwise
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dequantize_int8_bit_exact(ck, per_row, dtype):
+    rng = np.random.default_rng(21)
+    Q = rng.integers(-127, 128, size=(77, 768)).astype(np.int8)
+    s = rng.uniform(1e-6, 3.0, 77).astype(np.float32)
+    Yf, Yb = oracle.dequantize_int8(Q, s if per_row else s[:1], per_row=per_row)
+    out = ck.dequantize_int8(dev(torch.from_numpy(Q)), dev(torch.from_numpy(s if per_row else s[:1])),
+                             per_row=per_row, dtype=dtype)
+    got = to_np(out)
+    if dtype == torch.float32:
+        assert np.array_equal(got.view(np.uint32), Yf.view(np.uint32))
+    else:
+        assert np.array_equal(got, Yb)
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (300, 1000), (4097, 512)])
+def test_quantize_int8_tensorwise_bit_exact(ck, M, K):
+    cfg = workloads.custom(M, 1024, 8, seed=M + K)
+    X, _, _ = workloads.make_inputs(cfg)
+    Xv = dev(X)[:, :K]  # row stride 1024 >= K
+    Q, s = ck.quantize_int8_tensorwise(Xv)
+    rQ, rs = oracle.quantize_int8_tensorwise(workloads.bf16_bits(X[:, :K].contiguous()))
+    assert to_np(s)[0].view(np.uint32) == np.float32(rs).view(np.uint32)
+    assert np.array_equal(to_np(Q), rQ)
