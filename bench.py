@@ -399,14 +399,17 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
             "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
             "dtype": "int8", "data": "synthetic", "impl": "ours",
             "config": config_dict(cfg, world, args.scaling, args.act, args.path),
-            "roofline": {"kernel": "gemm_i8_kernel (tcgen05 kind::i8 + fused epilogue)",
+            "roofline": {"kernel": ("gemm_i8_pair_kernel (2-SM tcgen05 kind::i8, fused epilogue, "
+                                    "TMA store)" if M > 128 else
+                                    "gemm_i8_kernel (tcgen05 kind::i8, fused epilogue)"),
                          "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
                          "peak_source": f"{P['source']} bf16 burst {P['bf16_tflops']} TFLOP/s x "
                                         f"nominal int8/bf16 ratio {NOMINAL_INT8_OVER_BF16}",
                          "frac_of_spec_4500": gemm_tops / 4500.0,
                          "ms_per_launch": ms_g},
-            "quantizer": {"kernel": "quant_rows_kernel (ConvRot256 + per-row INT8)",
+            "quantizer": {"kernel": ("quant_rows_bulk_kernel" if K <= 28672 else
+                                     "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)",
                           "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",
                           "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
                           "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},

@@ -15,7 +15,11 @@
 //    lane (e >> 3) & 3 of the quad; within the lane, pair j holds elements
 //    with e bit 0 = 0/1, j bit 0 = e bit 1, bit 1 = e bit 2, bits 2-4 = e
 //    bits 5-7. Lane t therefore loads 8 contiguous values at e = 8t + 32i
-//    (i = 0..7): 16-byte loads, each quad reading 64 contiguous bytes.
+//    (i = 0..7): 16-byte loads, each quad reading 64 contiguous bytes. In the
+//    staged kernel odd quads read chunk i ^ 1 into register group i (so the
+//    two quads of a quarter-warp use different shared-memory banks); the
+//    h = 32 stage, which pairs groups i and i ^ 1, and the code stores
+//    account for the swap.
 //  * Butterfly stages h = 1, 2, ..., 128 run in that order; each is one IEEE
 //    add or subtract per value (a - c as fma(c, -1, a): one rounding of the
 //    exact difference). h = 1 pairs the two halves of a float2 (scalar ops;
@@ -32,12 +36,17 @@
 //    Smaller rows follow the definition step by step (y = fl(z / 16), then the
 //    exact division).
 //  * Division: q needs round-half-even of the IEEE quotient fl(y / s). With
-//    d the divisor, r = fl(1/d) and t = fl(z * r), |t - z/d| < 2^-16 and
-//    |fl(z/d) - z/d| <= 2^-17 because |z/d| <= 127 (1 + 2^-23). So if t is
-//    farther than 2^-14 from every half-integer, rint(t) = rint(fl(z/d)).
-//    Groups of 8 values that contain a closer one (about 1 in 1000 groups)
-//    take rint(__fdiv_rn(z, d)). rint(t) itself is t + 1.5 * 2^23, whose low
-//    byte is the two's-complement code; no clamp is needed on that path.
+//    d the divisor and r = fl(1/d), the exact product z r is within
+//    127.00001 * 2^-24 < 2^-17 of z/d, and |fl(z/d) - z/d| <= 2^-18 because
+//    |z/d| < 128; so if z r is farther than 2^-17 + 2^-18 from every
+//    half-integer, rint(z r) = rint(fl(z/d)). One fma gives fl(z r + 1.5 * 2^23) =
+//    1.5 * 2^23 + rint(z r), whose low byte is the two's-complement code (no
+//    clamp is needed on that path); a second fma gives the distance of z r
+//    to that integer. Groups that hold a value within 2^-16 of a
+//    half-integer take rint(__fdiv_rn(z, d)) instead. The distance is
+//    computed as fl(rint(z r) - z r) (error <= 2^-26), so a value that is
+//    not redone lies more than 2^-16 - 2^-26 > 2^-17 + 2^-18 from every
+//    half-integer; about 1 value in 30000 is redone.
 //  * The whole row stays in registers of one CTA (rows_per_cta rows x K/256
 //    quads); the row absmax is reduced through a shared-memory atomicMax on
 //    the fp32 bit pattern, so X is read from HBM exactly once. BF16 rows are
@@ -49,6 +58,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -66,7 +76,7 @@ constexpr int kMaxThreads = 512;
 constexpr int kMaxRowsPerCta = kMaxThreads / 4;
 constexpr int kTwoPassQuads = 128;                   // quads per row in the two-pass variant
 constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
-constexpr float kNearHalf = 0.49993896484375f;       // 0.5 - 2^-14
+constexpr float kNearHalf = 0.4999847412109375f;     // 0.5 - 2^-16
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
 constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
 constexpr size_t kBulkSmemBudget = 112 * 1024;       // per-CTA staging budget (2 buffers)
@@ -270,55 +280,50 @@ __device__ __forceinline__ void act_in_smem(uint32_t saddr) {
     }
 }
 
-// Shared-memory load (input activation applied) with the h = 1 stage done.
-template <int kAct>
-__device__ __forceinline__ void load_block_smem_s1(uint32_t saddr, float2 (&P)[kPairs]) {
+// Shared-memory loads of lane t's 64 staged values (the block's bf16 at
+// saddr - 16 t; the lane's chunk i at saddr + 64 i). With sw5 = 1 the lane
+// reads chunk i ^ 1 into register group i: two neighbouring blocks then read
+// different 64-byte halves of the bank space in the same instruction, so the
+// 8 lanes of a quarter-warp hit 8 different 16-byte bank groups. Register
+// group i holds elements 8t + 32 (i ^ sw5) .. +7; the h = 32 stage and the
+// stores take the swap into account. kStage1: widening fused with h = 1.
+template <bool kStage1>
+__device__ __forceinline__ void load_block_smem(uint32_t saddr, int sw5, float2 (&P)[kPairs]) {
+    const uint32_t base[2] = {saddr + 64u * uint32_t(sw5), saddr - 64u * uint32_t(sw5)};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        uint32_t x, y, z, w;
+        uint32_t w[4];
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
-                     : "r"(saddr + 64u * i));
-        P[4 * i + 0] = widen_stage1(act_bf16x2<kAct>(x));
-        P[4 * i + 1] = widen_stage1(act_bf16x2<kAct>(y));
-        P[4 * i + 2] = widen_stage1(act_bf16x2<kAct>(z));
-        P[4 * i + 3] = widen_stage1(act_bf16x2<kAct>(w));
-    }
-}
-__device__ __forceinline__ void load_block_smem(uint32_t saddr, float2 (&P)[kPairs]) {
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(base[i & 1] + 64u * i));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t x, y, z, w;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
-                     : "r"(saddr + 64u * i));
-        P[4 * i + 0] = widen_bf16x2(x);
-        P[4 * i + 1] = widen_bf16x2(y);
-        P[4 * i + 2] = widen_bf16x2(z);
-        P[4 * i + 3] = widen_bf16x2(w);
+        for (int q = 0; q < 4; ++q) P[4 * i + q] = kStage1 ? widen_stage1(w[q]) : widen_bf16x2(w[q]);
     }
 }
 
-__device__ __forceinline__ void zero_block(float2 (&P)[kPairs]) {
+template <int NP>
+__device__ __forceinline__ void zero_block(float2 (&P)[NP]) {
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) P[j] = make_float2(0.0f, 0.0f);
+    for (int j = 0; j < NP; ++j) P[j] = make_float2(0.0f, 0.0f);
 }
 
 // h = 1: the two halves of every pair.
-__device__ __forceinline__ void stage_in_pair(float2 (&P)[kPairs]) {
+template <int NP>
+__device__ __forceinline__ void stage_in_pair(float2 (&P)[NP]) {
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
+    for (int j = 0; j < NP; ++j) {
         const float a = P[j].x;
         const float c = P[j].y;
         P[j] = make_float2(__fadd_rn(a, c), __fsub_rn(a, c));
     }
 }
 
-// Pairs j and j + J (J = 1, 2, 4, 8, 16).
-template <int J>
-__device__ __forceinline__ void stage_pairs(float2 (&P)[kPairs]) {
+// Pairs j and j + J (J a power of two): P[j] holds the element with the
+// stage's bit clear (a), P[j + J] the one with it set (c).
+template <int J, int NP>
+__device__ __forceinline__ void stage_pairs(float2 (&P)[NP]) {
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
+    for (int j = 0; j < NP; ++j) {
         if ((j & J) == 0) {
             const float2 a = P[j];
             const float2 c = P[j + J];
@@ -328,14 +333,33 @@ __device__ __forceinline__ void stage_pairs(float2 (&P)[kPairs]) {
     }
 }
 
-// Lanes t and t ^ L of the quad (L = 1, 2): the lane with the bit clear holds
-// a and computes a + c; the other holds c and computes a - c = fma(-1, c, a).
-template <int L>
-__device__ __forceinline__ void stage_lanes(float2 (&P)[kPairs], int t) {
+// As stage_pairs, for a block whose two registers of each pair may hold the
+// elements swapped (sg = -1: P[j] holds c, P[j + J] holds a). The element
+// with the bit clear must receive a + c and the other a - c:
+//   P[j]     <- fma(sg, P[j], P[j + J])   (a + c, or a - c when swapped)
+//   P[j + J] <- fma(-sg, P[j + J], P[j])  (a - c, or a + c when swapped)
+// fma(+-1, x, y) rounds the exact y +- x once, as the definition's add does.
+template <int J, int NP>
+__device__ __forceinline__ void stage_pairs_swz(float2 (&P)[NP], float2 sg, float2 nsg) {
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        if ((j & J) == 0) {
+            const float2 lo = P[j];
+            const float2 hi = P[j + J];
+            P[j] = __ffma2_rn(sg, lo, hi);
+            P[j + J] = __ffma2_rn(nsg, hi, lo);
+        }
+    }
+}
+
+// Lanes t and t ^ L (L = 1, 2): the lane with the bit clear holds a and
+// computes a + c; the other holds c and computes a - c = fma(-1, c, a).
+template <int L, int NP>
+__device__ __forceinline__ void stage_lanes(float2 (&P)[NP], int t) {
     const float s = (t & L) ? -1.0f : 1.0f;
     const float2 sg = make_float2(s, s);
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
+    for (int j = 0; j < NP; ++j) {
         const float2 p = make_float2(__shfl_xor_sync(0xFFFFFFFFu, P[j].x, L),
                                      __shfl_xor_sync(0xFFFFFFFFu, P[j].y, L));
         P[j] = __ffma2_rn(sg, P[j], p);
@@ -343,27 +367,31 @@ __device__ __forceinline__ void stage_lanes(float2 (&P)[kPairs], int t) {
 }
 
 // The 8 butterfly stages of ConvRot256, without the final * 1/16 (z = 16 y);
-// kStage1Done when h = 1 was applied while loading.
+// kStage1Done when h = 1 was applied while loading; sw5 = 1 when the
+// register groups of the h = 32 stage are swapped (staged kernel).
 template <bool kStage1Done = false>
-__device__ __forceinline__ void butterflies(float2 (&P)[kPairs], int t) {
+__device__ __forceinline__ void butterflies(float2 (&P)[kPairs], int t, int sw5 = 0) {
     if (!kStage1Done) stage_in_pair(P);    // h = 1
     stage_pairs<1>(P);   // h = 2
     stage_pairs<2>(P);   // h = 4
     stage_lanes<1>(P, t);  // h = 8
     stage_lanes<2>(P, t);  // h = 16
-    stage_pairs<4>(P);   // h = 32
+    const float s5 = sw5 ? -1.0f : 1.0f;
+    stage_pairs_swz<4>(P, make_float2(s5, s5), make_float2(-s5, -s5));  // h = 32
     stage_pairs<8>(P);   // h = 64
     stage_pairs<16>(P);  // h = 128
 }
 
-__device__ __forceinline__ float quad_absmax(const float2 (&P)[kPairs]) {
+// Largest |value| of the block, reduced over the kLanes lanes that hold it.
+template <int kLanes = 4, int NP>
+__device__ __forceinline__ float block_absmax(const float2 (&P)[NP]) {
     // four independent chains keep the reduction's dependency depth short
     float mm[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) mm[j & 3] = max3(mm[j & 3], fabsf(P[j].x), fabsf(P[j].y));
+    for (int j = 0; j < NP; ++j) mm[j & 3] = max3(mm[j & 3], fabsf(P[j].x), fabsf(P[j].y));
     float m = fmaxf(max3(mm[0], mm[1], mm[2]), mm[3]);
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+#pragma unroll
+    for (int l = 1; l < kLanes; l <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, l));
     return m;
 }
 
@@ -416,57 +444,86 @@ __device__ __forceinline__ uint32_t code_exact(float z, const RowQuant &rq) {
     return __float_as_uint(__fadd_rn(q, kMagic));
 }
 
+// Fast path for two values (z) of a row with reciprocal rc = fl(1 / d):
+// m = fl(z rc + 1.5 * 2^23) = 1.5 * 2^23 + rint(z rc), one rounding of the
+// exact product-sum (|z rc| < 128, so the sum lies in [2^23, 2^24) where the
+// spacing is 1); its low byte is the code. d = fl(rint(z rc) - z rc) is the
+// (negated) distance to that integer; dmax tracks the largest |d|.
+struct FastQuant {
+    float2 rc2, nrc2, magic2, nmagic2;
+    __device__ __forceinline__ explicit FastQuant(float rc)
+        : rc2(make_float2(rc, rc)), nrc2(make_float2(-rc, -rc)),
+          magic2(make_float2(kMagic, kMagic)), nmagic2(make_float2(-kMagic, -kMagic)) {}
+    __device__ __forceinline__ float2 code2(float2 z, float &dmax) const {
+        const float2 m = __ffma2_rn(z, rc2, magic2);
+        const float2 rt = add2(m, nmagic2);
+        const float2 d = __ffma2_rn(z, nrc2, rt);
+        dmax = max3(dmax, fabsf(d.x), fabsf(d.y));
+        return m;
+    }
+};
+
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     const uint32_t ab = __byte_perm(a, b, 0x0040);
     const uint32_t cd = __byte_perm(c, d, 0x0040);
     return __byte_perm(ab, cd, 0x5410);
 }
 
-// Stores the 8 codes of group i: 8 int8 bytes at qbase + 32 i, or (kPack4)
-// 8 signed nibbles in one 32-bit word at qbase + 16 i, element 2j in the low
-// nibble of byte j. qbase already points at this lane's first element (or
-// its packed byte).
+// Where the codes of register group i go. In the staged kernel the group
+// index is swizzled with bit 0 of the block index (sw5, see load_block_smem):
+// register group i then holds elements 8t + 32 (i ^ sw5) .. +7, whose codes
+// start at q[i & 1] + 32 i with q[0] = qbase + 32 sw5, q[1] = qbase - 32 sw5.
+// Unswizzled callers pass sw5 = 0.
+struct CodeDst {
+    int8_t *q[2];
+    __device__ __forceinline__ CodeDst(int8_t *qbase, int sw5)
+        : q{qbase + 32 * sw5, qbase - 32 * sw5} {}
+};
+
+// Stores the 8 codes of group i: 8 int8 bytes at dst.q[i & 1] + 32 i, or
+// (kPack4, unswizzled only) 8 signed nibbles in one 32-bit word at
+// q + 16 i, element 2j in the low nibble of byte j. The destination already
+// points at this lane's first element (or its packed byte).
 template <bool kPack4>
-__device__ __forceinline__ void store_group(const uint32_t (&u)[8], int i, int8_t *qbase) {
+__device__ __forceinline__ void store_group(const uint32_t (&u)[8], int i, const CodeDst &dst) {
     const uint32_t lo = pack4(u[0], u[1], u[2], u[3]);
     const uint32_t hi = pack4(u[4], u[5], u[6], u[7]);
     if (!kPack4) {
-        *reinterpret_cast<uint2 *>(qbase + 32 * i) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2 *>(dst.q[i & 1] + 32 * i) = make_uint2(lo, hi);
     } else {
         const uint32_t a = lo & 0x0F0F0F0Fu, b = hi & 0x0F0F0F0Fu;
         const uint32_t a2 = a | (a >> 4), b2 = b | (b >> 4);  // byte pairs -> one byte each
-        *reinterpret_cast<uint32_t *>(qbase + 16 * i) = __byte_perm(a2, b2, 0x6420);
+        *reinterpret_cast<uint32_t *>(dst.q[0] + 16 * i) = __byte_perm(a2, b2, 0x6420);
     }
 }
 
-// Quantise lane t's 64 values and store the codes: group i (pairs 4i..4i+3)
-// holds elements 8t + 32i .. +7, stored as 8 contiguous bytes. The fast path
-// stores every group without branching and records which groups hold a value
-// near a half-integer; those (rare) groups are then recomputed exactly and
-// stored again.
 template <bool kPack4>
 __device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int i,
-                                                  const RowQuant &rq, int8_t *qbase) {
+                                                  const RowQuant &rq, const CodeDst &dst) {
     uint32_t u[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         u[2 * k] = code_exact(P[4 * i + k].x, rq);
         u[2 * k + 1] = code_exact(P[4 * i + k].y, rq);
     }
-    store_group<kPack4>(u, i, qbase);
+    store_group<kPack4>(u, i, dst);
 }
 
+// Quantise lane t's 64 values and store the codes: group i (pairs 4i..4i+3)
+// holds 8 consecutive elements, stored as 8 contiguous bytes. The fast path
+// stores every group without branching and records which groups hold a value
+// near a half-integer; those (rare) groups are then recomputed exactly and
+// stored again.
 template <bool kPack4 = false>
 __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const RowQuant &rq,
-                                               int8_t *qbase) {
+                                               int8_t *qbase, int sw5 = 0) {
+    const CodeDst dst(qbase, sw5);
     if (!rq.fast) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) store_group_exact<kPack4>(P, i, rq, qbase);
+        for (int i = 0; i < 8; ++i) store_group_exact<kPack4>(P, i, rq, dst);
         return;
     }
-    const float2 rc2 = make_float2(rq.rc, rq.rc);
-    const float2 magic2 = make_float2(kMagic, kMagic);
-    const float2 nmagic2 = make_float2(-kMagic, -kMagic);
+    const FastQuant fq(rq.rc);
     uint32_t redo = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -474,21 +531,17 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const 
         float dmax = 0.0f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 t = __fmul2_rn(P[4 * i + k], rc2);
-            const float2 m = add2(t, magic2);
-            const float2 rt = add2(m, nmagic2);
-            const float2 d = sub2(t, rt);
-            dmax = max3(dmax, fabsf(d.x), fabsf(d.y));
+            const float2 m = fq.code2(P[4 * i + k], dmax);
             u[2 * k] = __float_as_uint(m.x);
             u[2 * k + 1] = __float_as_uint(m.y);
         }
         redo |= uint32_t(dmax >= kNearHalf) << i;
-        store_group<kPack4>(u, i, qbase);
+        store_group<kPack4>(u, i, dst);
     }
     if (redo) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            if (redo & (1u << i)) store_group_exact<kPack4>(P, i, rq, qbase);
+            if (redo & (1u << i)) store_group_exact<kPack4>(P, i, rq, dst);
     }
 }
 
@@ -517,7 +570,7 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     else
         zero_block(P);
     if (kRotate) butterflies(P, t);
-    const float m = quad_absmax(P);
+    const float m = block_absmax(P);
     __syncthreads();  // s_amax initialised
     if (active && t == 0) atomicMax(&s_amax[row_local], __float_as_uint(m));
     __syncthreads();
@@ -551,6 +604,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     const int row_local = quad / nb;
     const int blk = quad - row_local * nb;
     const int col0 = blk * kBlock + 8 * t;
+    const int sw5 = quad & 1;  // chunk swizzle of this lane (see load_block_smem)
     const int64_t ngroups = (M + R - 1) / R;
     const uint32_t row_bytes = uint32_t(K) * 2u;
     const uint32_t buf0 = smem_u32(stage_raw);
@@ -598,18 +652,14 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         float2 P[kPairs];
         const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
                             uint32_t(col0) * 2u;
-        if (kRotate) {
-            if (active) {
-                if (kAct != kActNone) act_in_smem<kAct>(sa);
-                load_block_smem_s1<kActNone>(sa, P);
-            } else {
-                zero_block(P);
-            }
-            butterflies<true>(P, t);
+        if (active) {
+            if (kAct != kActNone) act_in_smem<kAct>(sa);
+            load_block_smem<kRotate>(sa, sw5, P);
         } else {
-            if (active) load_block_smem(sa, P); else zero_block(P);
+            zero_block(P);
         }
-        const float m = quad_absmax(P);
+        if (kRotate) butterflies<true>(P, t, sw5);
+        const float m = block_absmax(P);
         if (active && t == 0) atomicMax(&s_amax[slot][row_local], __float_as_uint(m));
         if (__syncthreads_or(!ok)) {
             if (tid == 0) atomicMax(err, kDevErrTimeout);
@@ -626,7 +676,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         if (active) {
             const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[slot][row_local]));
             if (blk == 0 && t == 0) S[row] = rq.s;
-            quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0);
+            quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0, sw5);
         }
         slot = slot == 2 ? 0 : slot + 1;
     }
@@ -656,7 +706,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
         else
             zero_block(P);
         if (kRotate) butterflies(P, t);
-        m = fmaxf(m, quad_absmax(P));
+        m = fmaxf(m, block_absmax(P));
     }
     __syncthreads();
     if (t == 0) atomicMax(&s_amax, __float_as_uint(m));
@@ -681,19 +731,20 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
     }
 }
 
-// Rows per CTA: the CTA has 4 * nb * R useful threads rounded up to whole
+// Rows per CTA: the CTA has lanes * nb * R useful threads rounded up to whole
 // warps; pick the R with the fewest idle lanes, then the CTA size closest to
-// 256 threads, with at most max_rows rows.
-int pick_rows_per_cta(int nb, int max_rows, int *threads_out) {
-    int best_r = 1, best_t = ((4 * nb + 31) / 32) * 32;
+// `target` threads, with at most max_rows rows and max_threads threads.
+int pick_rows_per_cta(int nb, int lanes, int max_rows, int max_threads, int target,
+                      int *threads_out) {
+    int best_r = 1, best_t = ((lanes * nb + 31) / 32) * 32;
     double best_waste = 2.0;
     int best_dist = 1 << 30;
-    for (int r = 1; r <= max_rows && 4 * nb * r <= kMaxThreads; ++r) {
-        const int used = 4 * nb * r;
+    for (int r = 1; r <= max_rows && lanes * nb * r <= max_threads; ++r) {
+        const int used = lanes * nb * r;
         const int threads = ((used + 31) / 32) * 32;
-        if (threads > kMaxThreads) break;
+        if (threads > max_threads) break;
         const double waste = double(threads - used) / threads;
-        const int dist = threads > 256 ? threads - 256 : 256 - threads;
+        const int dist = threads > target ? threads - target : target - threads;
         if (waste < best_waste - 1e-12 || (waste < best_waste + 1e-12 && dist < best_dist)) {
             best_waste = waste;
             best_dist = dist;
@@ -736,10 +787,11 @@ cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, in
                         unsigned *err, int num_sms, cudaStream_t stream, bool *launched) {
     *launched = false;
     const int nb = static_cast<int>(K / kBlock);
-    const int max_rows = static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2));
+    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2)),
+                                  kMaxRowsPerCta);
     if (max_rows < 1 || 4 * nb > kMaxThreads) return cudaSuccess;
     int threads = 0;
-    const int rows = pick_rows_per_cta(nb, max_rows, &threads);
+    const int rows = pick_rows_per_cta(nb, 4, max_rows, kMaxThreads, 256, &threads);
     const size_t smem = 2 * size_t(rows) * size_t(K) * 2;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -763,7 +815,7 @@ cudaError_t launch_direct(const TIn *X, int64_t M, int64_t K, int64_t ldx, int8_
     const int nb = static_cast<int>(K / kBlock);
     if (4 * nb <= kMaxThreads) {
         int threads = 0;
-        const int rows = pick_rows_per_cta(nb, kMaxRowsPerCta, &threads);
+        const int rows = pick_rows_per_cta(nb, 4, kMaxRowsPerCta, kMaxThreads, 256, &threads);
         const int64_t grid = (M + rows - 1) / rows;
         quant_rows_kernel<kRotate, kAct, kQ, kPack4, TIn><<<static_cast<unsigned>(grid), threads, 0, stream>>>(
             X, M, static_cast<int>(K), ldx, rows, Q, S);
