@@ -206,6 +206,41 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
                              ck_stream_t stream);
 
 /*
+ * ck_int8_linear_act for activations and outputs in HOST memory, with the
+ * PCIe copies overlapped with the kernels. The rows are processed in chunks of
+ * chunk_rows (the last one ragged): chunk c is copied to the device while
+ * chunk c-1 is quantised and multiplied and chunk c-2 is copied back, so the
+ * call takes about as long as the larger of its two transfers. The results
+ * are those of ck_int8_linear_act row for row (rows are independent:
+ * sglang PR "Tune Kitchen INT8 row splitting for SM120", Accuracy Test).
+ *
+ *   X_host  [M, K] bf16, row stride ldx (ldx >= K) elements, host memory.
+ *           (input; page-locked memory - cudaHostAlloc, cudaHostRegister,
+ *           torch pin_memory - lets the copies run asynchronously; pageable
+ *           memory gives the same results without the overlap)
+ *   Qw, s_w, bias: device memory, as for ck_int8_linear.
+ *   Y_host  [M, N] bf16, row stride N, host memory.   (output)
+ *   chunk_rows  rows per chunk (> 0); 4096 keeps a chunk's GEMM several
+ *           waves long on a B200 for the N of the pages' workloads.
+ *   workspace   >= ck_int8_linear_host_workspace_bytes(chunk_rows, N, K)
+ *           bytes of device memory, 256-B aligned (two input and two output
+ *           chunk buffers, the chunk's codes and row scales).
+ *
+ * Ordering: the copies and kernels run on three streams the library creates
+ * once per device (together with the events that link them); they start
+ * after the work already queued on `stream`, and `stream` waits for the last
+ * copy back, so work queued on `stream` afterwards - or a synchronize of it -
+ * sees Y_host complete. Calls on one device are queued on the same internal
+ * streams in the order they are made. Nothing here blocks the host (apart
+ * from what the driver does for pageable memory).
+ */
+size_t ck_int8_linear_host_workspace_bytes(int64_t chunk_rows, int64_t N, int64_t K);
+ck_status ck_int8_linear_host(const ck_bf16 *X_host, int64_t ldx, int act, const int8_t *Qw,
+                              const float *s_w, const ck_bf16 *bias, ck_bf16 *Y_host, int64_t M,
+                              int64_t N, int64_t K, int64_t chunk_rows, void *workspace,
+                              size_t workspace_bytes, ck_stream_t stream);
+
+/*
  * convrot_w4a4_linear (comfy-kitchen 0.2.40, "Huawei Ascend backend": ConvRot
  * then signed INT4 quantisation of both operands; activation codes stay in
  * INT8 storage; packed weights are unpacked to INT8 for INT32 accumulation;

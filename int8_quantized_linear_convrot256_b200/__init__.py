@@ -71,6 +71,9 @@ _SIGS = {
     "ck_dequantize_int8": (_st, [_vp, _vp, _i64, _i64, _st, _st, _vp, _vp]),
     "ck_quantize_int8_tensorwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_int8_linear_host_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "ck_int8_linear_host": (_st, [_vp, _i64, _st, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                  _vp, ctypes.c_size_t, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
     "ck_clear_device_error": (_st, []),
@@ -225,6 +228,50 @@ def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
         _check(lib.ck_int8_linear_act(_ptr(X), ldx, ACTS[input_act], _ptr(Qw), _ptr(s_w),
                                       _ptr(bias), _ptr(out), M, N, K, _ptr(workspace), ws_bytes,
                                       _stream(stream)), "ck_int8_linear_act")
+    return out
+
+
+def host_workspace_bytes(chunk_rows: int, N: int, K: int) -> int:
+    return int(lib.ck_int8_linear_host_workspace_bytes(chunk_rows, N, K))
+
+
+def int8_linear_host(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                     bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     chunk_rows: int = 4096, workspace: torch.Tensor | None = None, stream=None,
+                     input_act: str = "none") -> torch.Tensor:
+    """int8_linear for X and Y in host memory (ck_int8_linear_host): the rows
+    go through the GPU in chunks with the copies in and out overlapped with the
+    kernels. X and ``out`` should be pinned CPU tensors for the overlap; the
+    result is ready once ``stream`` (default: the current stream of Qw's
+    device) has completed."""
+    if X.device.type != "cpu":
+        raise ValueError("X must be a CPU tensor (use int8_linear for device tensors)")
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a 2-D bf16 CPU tensor with unit column stride")
+    _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
+    _need(s_w, "s_w", torch.float32, 1)
+    M, K = X.shape
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, Qw {tuple(Qw.shape)}, s_w {tuple(s_w.shape)}")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    if (out.device.type != "cpu" or out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N)
+            or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous [M, N] bf16 CPU tensor")
+    chunk_rows = max(1, min(int(chunk_rows), max(M, 1)))
+    need = host_workspace_bytes(chunk_rows, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Qw.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    with torch.cuda.device(Qw.device):
+        _check(lib.ck_int8_linear_host(_ptr(X), ldx, ACTS[input_act], _ptr(Qw), _ptr(s_w),
+                                       _ptr(bias), _ptr(out), M, N, K, chunk_rows,
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)), "ck_int8_linear_host")
     return out
 
 

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "ck.h"
@@ -201,6 +202,40 @@ ck_status weight_common(const float *W, int64_t N, int64_t K, void *Qw, float *s
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
+// Streams and events of ck_int8_linear_host, created once per device.
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+    cudaEvent_t entry = nullptr, done = nullptr;
+    cudaEvent_t in_done[2] = {}, x_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
+    std::mutex m;
+};
+HostPipe g_pipe[kMaxDevices];
+
+ck_status host_pipe(HostPipe **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    HostPipe &hp = g_pipe[dev];
+    if (!hp.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&hp.entry, ef) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&hp.done, ef) == cudaSuccess;
+        for (int i = 0; ok && i < 2; ++i)
+            ok = cudaEventCreateWithFlags(&hp.in_done[i], ef) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&hp.x_free[i], ef) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&hp.y_ready[i], ef) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&hp.y_free[i], ef) == cudaSuccess;
+        if (!ok) return CK_ERR_CUDA;
+        hp.ready = true;
+    }
+    *out = &hp;
+    return CK_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -333,6 +368,99 @@ ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const 
                          void *workspace, size_t workspace_bytes, ck_stream_t stream) {
     return ck_int8_linear_act(X, ldx, CK_ACT_NONE, Qw, s_w, bias, Y, M, N, K, workspace,
                               workspace_bytes, stream);
+}
+
+size_t ck_int8_linear_host_workspace_bytes(int64_t chunk_rows, int64_t N, int64_t K) {
+    if (chunk_rows <= 0 || N <= 0 || K <= 0) return 0;
+    const size_t r = size_t(chunk_rows);
+    return 2 * round256(r * size_t(K) * 2) + 2 * round256(r * size_t(N) * 2) +
+           ck_int8_linear_workspace_bytes(chunk_rows, K);
+}
+
+ck_status ck_int8_linear_host(const ck_bf16 *X_host, int64_t ldx, int act, const int8_t *Qw,
+                              const float *s_w, const ck_bf16 *bias, ck_bf16 *Y_host, int64_t M,
+                              int64_t N, int64_t K, int64_t chunk_rows, void *workspace,
+                              size_t workspace_bytes, ck_stream_t stream) {
+    if (M < 0 || N < 0 || chunk_rows <= 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH)
+        return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && N > 0 && (!X_host || !Qw || !s_w || !Y_host || !workspace))
+        return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) ||
+        chunk_rows >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(Qw) || !aligned16(s_w) || (bias && !aligned16(bias)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CK_ERR_MISALIGNED;
+    if (workspace_bytes < ck_int8_linear_host_workspace_bytes(chunk_rows, N, K))
+        return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    HostPipe *hp = nullptr;
+    s = host_pipe(&hp);
+    if (s != CK_OK) return s;
+    std::lock_guard<std::mutex> lock(hp->m);
+
+    const size_t r = size_t(chunk_rows);
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    const size_t xb_bytes = round256(r * size_t(K) * 2), yb_bytes = round256(r * size_t(N) * 2);
+    ck_bf16 *xb[2] = {reinterpret_cast<ck_bf16 *>(base),
+                      reinterpret_cast<ck_bf16 *>(base + xb_bytes)};
+    ck_bf16 *yb[2] = {reinterpret_cast<ck_bf16 *>(base + 2 * xb_bytes),
+                      reinterpret_cast<ck_bf16 *>(base + 2 * xb_bytes + yb_bytes)};
+    int8_t *Qx = reinterpret_cast<int8_t *>(base + 2 * xb_bytes + 2 * yb_bytes);
+    float *s_x = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Qx) +
+                                           round256(r * size_t(K)));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+    // start after the caller's queued work and after the previous call
+    if (cudaEventRecord(hp->entry, cs) != cudaSuccess) return CK_ERR_CUDA;
+    for (cudaStream_t q : {hp->in, hp->comp, hp->out})
+        if (cudaStreamWaitEvent(q, hp->entry, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(q, hp->done, 0) != cudaSuccess)
+            return CK_ERR_CUDA;
+    const int64_t nchunks = (M + chunk_rows - 1) / chunk_rows;
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int b = int(c & 1);
+        const int64_t r0 = c * chunk_rows;
+        const int64_t rows = M - r0 < chunk_rows ? M - r0 : chunk_rows;
+        // copy in (buffer b was last read by the quantiser of chunk c - 2)
+        if (c >= 2 && cudaStreamWaitEvent(hp->in, hp->x_free[b], 0) != cudaSuccess)
+            return CK_ERR_CUDA;
+        if (cudaMemcpy2DAsync(xb[b], size_t(K) * 2, X_host + r0 * ldx, size_t(ldx) * 2,
+                              size_t(K) * 2, size_t(rows), cudaMemcpyHostToDevice,
+                              hp->in) != cudaSuccess ||
+            cudaEventRecord(hp->in_done[b], hp->in) != cudaSuccess)
+            return CK_ERR_CUDA;
+        // quantise + GEMM (output buffer b was last read by the copy out of chunk c - 2)
+        if (cudaStreamWaitEvent(hp->comp, hp->in_done[b], 0) != cudaSuccess ||
+            (c >= 2 && cudaStreamWaitEvent(hp->comp, hp->y_free[b], 0) != cudaSuccess))
+            return CK_ERR_CUDA;
+        if (ck::launch_quant_rows_bf16(xb[b], rows, K, K, true, act, 127, Qx, s_x, st->err,
+                                       st->num_sms, hp->comp) != cudaSuccess ||
+            cudaEventRecord(hp->x_free[b], hp->comp) != cudaSuccess)
+            return CK_ERR_CUDA;
+        s = run_gemm(Qx, s_x, Qw, s_w, bias, yb[b], nullptr, rows, N, K, st, hp->comp);
+        if (s != CK_OK) return s;
+        if (cudaEventRecord(hp->y_ready[b], hp->comp) != cudaSuccess) return CK_ERR_CUDA;
+        // copy out
+        if (cudaStreamWaitEvent(hp->out, hp->y_ready[b], 0) != cudaSuccess ||
+            cudaMemcpyAsync(Y_host + r0 * N, yb[b], size_t(rows) * size_t(N) * 2,
+                            cudaMemcpyDeviceToHost, hp->out) != cudaSuccess ||
+            cudaEventRecord(hp->y_free[b], hp->out) != cudaSuccess)
+            return CK_ERR_CUDA;
+    }
+    // the copy-out stream's last work follows every kernel and copy above
+    if (cudaStreamWaitEvent(hp->out, hp->x_free[(nchunks - 1) & 1], 0) != cudaSuccess ||
+        cudaEventRecord(hp->done, hp->out) != cudaSuccess ||
+        cudaStreamWaitEvent(cs, hp->done, 0) != cudaSuccess)
+        return CK_ERR_CUDA;
+    return CK_OK;
 }
 
 ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw4,

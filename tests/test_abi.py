@@ -122,3 +122,36 @@ def test_binding_rejects_cpu_tensors():
 
     with pytest.raises(ValueError, match="CUDA"):
         ck.quantize_rotate_rowwise(torch.zeros((2, 256), dtype=torch.bfloat16))
+
+
+def lin_host(X=FAKE, ldx=512, act=0, Qw=FAKE, s_w=FAKE, bias=None, Y=FAKE, M=4, N=8, K=512,
+             chunk=2, ws=FAKE, ws_bytes=1 << 30):
+    return ck.lib.ck_int8_linear_host(X, ldx, act, Qw, s_w, bias, Y, M, N, K, chunk, ws, ws_bytes,
+                                      None)
+
+
+def test_host_workspace_bytes():
+    assert ck.host_workspace_bytes(0, 8, 256) == 0
+    # two input chunks, two output chunks, the chunk's codes and row scales
+    r, N, K = 4096, 16128, 5376
+    want = 2 * r * K * 2 + 2 * r * N * 2 + r * K + 4 * r
+    assert ck.host_workspace_bytes(r, N, K) == want
+    assert ck.host_workspace_bytes(3, 8, 256) == 2 * 1536 + 2 * 256 + 768 + 256
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(X=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(Y=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(ws=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(chunk=0), ck.CK_ERR_INVALID_VALUE),
+    (dict(act=7), ck.CK_ERR_INVALID_VALUE),
+    (dict(ldx=256), ck.CK_ERR_INVALID_VALUE),
+    (dict(K=300, ldx=512), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(N=12), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(Qw=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(ws=FAKE + 16), ck.CK_ERR_MISALIGNED),
+    (dict(ws_bytes=1024), ck.CK_ERR_WORKSPACE),
+    (dict(M=0), ck.CK_OK),
+])
+def test_int8_linear_host_validation(kw, status):
+    assert lin_host(**kw) == status

@@ -412,3 +412,51 @@ def test_quantize_int8_tensorwise_bit_exact(ck, M, K):
     rQ, rs = oracle.quantize_int8_tensorwise(workloads.bf16_bits(X[:, :K].contiguous()))
     assert to_np(s)[0].view(np.uint32) == np.float32(rs).view(np.uint32)
     assert np.array_equal(to_np(Q), rQ)
+
+
+# ------------------------------------------------- host buffers, pipelined copies
+
+
+def _host_tensor(X, pinned, strided):
+    M, K = X.shape
+    buf = torch.zeros((M, K + (256 if strided else 0)), dtype=torch.bfloat16, pin_memory=pinned)
+    buf[:, :K] = X
+    return buf[:, :K]
+
+
+@pytest.mark.parametrize("M,chunk,pinned,strided", [(785, 256, True, False), (785, 256, False, True),
+                                                    (100, 4096, True, True), (1, 256, True, False),
+                                                    (512, 256, True, False)])
+def test_int8_linear_host_matches_oracle(ck, M, chunk, pinned, strided):
+    K, N = 768, 264
+    cfg = workloads.custom(M, K, N, seed=M + chunk)
+    X, W, bias = workloads.make_inputs(cfg)
+    Yr, _, _ = _oracle_linear(X, W, bias)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    Xh = _host_tensor(X, pinned, strided)
+    out = torch.full((M, N), 7.0, dtype=torch.bfloat16, pin_memory=pinned)
+    Y = ck.int8_linear_host(Xh, Qw, s_w, dev(bias), out=out, chunk_rows=chunk)
+    torch.cuda.current_stream().synchronize()
+    assert Y.data_ptr() == out.data_ptr()
+    assert_bf16_close(workloads.bf16_bits(Y), Yr)
+
+
+def test_int8_linear_host_equals_device_call_with_act_and_reused_workspace(ck):
+    """Two calls back to back on one workspace (different inputs, silu) give
+    exactly the device-side int8_linear results, at a size that spans several
+    GEMM tiles per chunk and a ragged last chunk."""
+    K, N = 5376, 520
+    Qw = None
+    ws = None
+    for seed, M in ((1, 1300), (2, 777)):
+        cfg = workloads.custom(M, K, N, seed=seed)
+        X, W, bias = workloads.make_inputs(cfg)
+        if Qw is None:
+            Qw, s_w = ck.rotate_quant_weight(dev(W))
+            ws = torch.empty(ck.host_workspace_bytes(512, N, K), dtype=torch.uint8, device="cuda")
+        ref = to_np(ck.int8_linear(dev(X), Qw, s_w, dev(bias), input_act="silu"))
+        Xh = _host_tensor(X, True, False)
+        Y = ck.int8_linear_host(Xh, Qw, s_w, dev(bias), chunk_rows=512, workspace=ws,
+                                input_act="silu")
+        torch.cuda.current_stream().synchronize()
+        assert np.array_equal(workloads.bf16_bits(Y), ref)
