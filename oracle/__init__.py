@@ -20,6 +20,12 @@ What each function follows (page title, section):
   - ``gemm_i32`` / ``epilogue`` / ``int8_linear``: ComfyUI-AppleSilicon-FP8
     README row 17 (INT8 x INT8 -> INT32, per-row rescale + bias in the store
     epilogue) and comfy-kitchen "int8_linear".
+  - ``e2m1_*``, ``e4m3_*``, ``nvfp4_*``: ComfyUI-HSWQ-Loader-and-Tools, "NVFP4
+    torch.compile Fix", section 5-1 (nvfp4_gemm.py): the E2M1 value table,
+    16-value blocks, the blocked scale layout that from_blocked undoes, a
+    per-tensor scale, dequantisation and a_dq @ w_dq.T + bias; the quantiser
+    (two-level scales: s_t = amax / 2688, E4M3 block scales) is this build's
+    reading, stated in convrot_oracle.c.
 """
 from __future__ import annotations
 
@@ -103,6 +109,30 @@ def lib():
             L.oracle_linear_rows.argtypes = [i8p, f32p, i8p, f32p, u16p, i64, i64,
                                              _P(ctypes.c_int64), i64, u16p]
             L.oracle_linear_rows.restype = None
+            L.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+            L.oracle_e2m1_to_f32.restype = ctypes.c_float
+            L.oracle_f32_to_e2m1_rne.argtypes = [ctypes.c_float]
+            L.oracle_f32_to_e2m1_rne.restype = ctypes.c_uint8
+            L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+            L.oracle_e4m3_to_f32.restype = ctypes.c_float
+            L.oracle_f32_to_e4m3_rne.argtypes = [ctypes.c_float]
+            L.oracle_f32_to_e4m3_rne.restype = ctypes.c_uint8
+            L.oracle_nvfp4_sf_offset.argtypes = [i64, i64, i64]
+            L.oracle_nvfp4_sf_offset.restype = i64
+            L.oracle_nvfp4_sf_bytes.argtypes = [i64, i64]
+            L.oracle_nvfp4_sf_bytes.restype = i64
+            L.oracle_quantize_rotate_nvfp4_bf16.argtypes = [u16p, i64, i64, i64, u8p, u8p, f32p]
+            L.oracle_quantize_rotate_nvfp4_bf16.restype = ctypes.c_int
+            L.oracle_rotate_quant_weight_nvfp4.argtypes = [f32p, i64, i64, u8p, u8p, f32p]
+            L.oracle_rotate_quant_weight_nvfp4.restype = ctypes.c_int
+            L.oracle_dequantize_nvfp4.argtypes = [u8p, u8p, ctypes.c_float, i64, i64, ctypes.c_int,
+                                                  f32p]
+            L.oracle_dequantize_nvfp4.restype = None
+            L.oracle_nvfp4_linear_rows.argtypes = [u8p, u8p, ctypes.c_float, i64, u8p, u8p,
+                                                   ctypes.c_float, i64, u16p, i64,
+                                                   _P(ctypes.c_int64), i64, u16p,
+                                                   _P(ctypes.c_double)]
+            L.oracle_nvfp4_linear_rows.restype = None
             L.oracle_num_threads.argtypes = []
             L.oracle_num_threads.restype = ctypes.c_int
             _lib = L
@@ -324,3 +354,96 @@ def int8_linear(X_bits, Qw, s_w, bias_bits=None, act: str = "none"):
     Qx, s_x = quantize_rows_bf16(X_bits, rotate=True, act=act)
     acc = gemm_i32(Qx, Qw)
     return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc
+
+
+# ----------------------------------------------------------------- NVFP4
+
+
+def e2m1_to_f32(codes) -> np.ndarray:
+    L = lib()
+    c = np.asarray(codes, dtype=np.uint8).ravel()
+    return np.array([L.oracle_e2m1_to_f32(int(x)) for x in c], dtype=np.float32)
+
+
+def f32_to_e2m1(v) -> np.ndarray:
+    L = lib()
+    x = np.asarray(v, dtype=np.float32).ravel()
+    return np.array([L.oracle_f32_to_e2m1_rne(float(t)) for t in x], dtype=np.uint8)
+
+
+def e4m3_to_f32(codes) -> np.ndarray:
+    L = lib()
+    c = np.asarray(codes, dtype=np.uint8).ravel()
+    return np.array([L.oracle_e4m3_to_f32(int(x)) for x in c], dtype=np.float32)
+
+
+def f32_to_e4m3(v) -> np.ndarray:
+    L = lib()
+    x = np.asarray(v, dtype=np.float32).ravel()
+    return np.array([L.oracle_f32_to_e4m3_rne(float(t)) for t in x], dtype=np.uint8)
+
+
+def nvfp4_sf_offset(r: int, c: int, C: int) -> int:
+    return int(lib().oracle_nvfp4_sf_offset(r, c, C))
+
+
+def nvfp4_sf_bytes(R: int, K: int) -> int:
+    return int(lib().oracle_nvfp4_sf_bytes(R, K))
+
+
+def _nvfp4_out(R, K):
+    return (np.zeros((R, K // 2), dtype=np.uint8), np.zeros(nvfp4_sf_bytes(R, K), dtype=np.uint8),
+            np.zeros(1, dtype=np.float32))
+
+
+def quantize_rotate_nvfp4(X_bits: np.ndarray):
+    """ConvRot NVFP4 of bf16 rows: (codes [M, K/2], blocked scales, s_t)."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    Q, S, st = _nvfp4_out(M, K)
+    rc = lib().oracle_quantize_rotate_nvfp4_bf16(_ptr(X_bits, ctypes.c_uint16), M, K, K,
+                                                  _ptr(Q, ctypes.c_uint8), _ptr(S, ctypes.c_uint8),
+                                                  _ptr(st, ctypes.c_float))
+    assert rc == 0, rc
+    return Q, S, float(st[0])
+
+
+def rotate_quant_weight_nvfp4(W):
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Q, S, st = _nvfp4_out(N, K)
+    rc = lib().oracle_rotate_quant_weight_nvfp4(_ptr(W, ctypes.c_float), N, K,
+                                                _ptr(Q, ctypes.c_uint8), _ptr(S, ctypes.c_uint8),
+                                                _ptr(st, ctypes.c_float))
+    assert rc == 0, rc
+    return Q, S, float(st[0])
+
+
+def dequantize_nvfp4(Q, S, s_t: float, hi_first: bool = False) -> np.ndarray:
+    Q = np.ascontiguousarray(Q, dtype=np.uint8)
+    S = np.ascontiguousarray(S, dtype=np.uint8)
+    R, K2 = Q.shape
+    out = np.zeros((R, 2 * K2), dtype=np.float32)
+    lib().oracle_dequantize_nvfp4(_ptr(Q, ctypes.c_uint8), _ptr(S, ctypes.c_uint8), float(s_t),
+                                  R, 2 * K2, int(bool(hi_first)), _ptr(out, ctypes.c_float))
+    return out
+
+
+def nvfp4_linear_rows(Qa, Sa, s_ta, Qw, Sw, s_tw, bias_bits=None, rows=None):
+    """Rows of Y = bf16(float(sum) * s_ta * s_tw + bias); also sum |term| * alpha."""
+    Qa = np.ascontiguousarray(Qa, dtype=np.uint8)
+    Qw = np.ascontiguousarray(Qw, dtype=np.uint8)
+    Sa = np.ascontiguousarray(Sa, dtype=np.uint8)
+    Sw = np.ascontiguousarray(Sw, dtype=np.uint8)
+    M, K2 = Qa.shape
+    N = Qw.shape[0]
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    Y = np.zeros((len(rows), N), dtype=np.uint16)
+    mag = np.zeros((len(rows), N), dtype=np.float64)
+    bb = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    lib().oracle_nvfp4_linear_rows(_ptr(Qa, ctypes.c_uint8), _ptr(Sa, ctypes.c_uint8), float(s_ta), M,
+                                   _ptr(Qw, ctypes.c_uint8), _ptr(Sw, ctypes.c_uint8), float(s_tw), N,
+                                   None if bb is None else _ptr(bb, ctypes.c_uint16), 2 * K2,
+                                   _ptr(rows, ctypes.c_int64), len(rows),
+                                   _ptr(Y, ctypes.c_uint16), _ptr(mag, ctypes.c_double))
+    return Y, mag

@@ -30,6 +30,9 @@
  * [-127, 127]; an all-zero row gets s = 0 and all-zero codes. Epilogue:
  * y = bf16_rne(((float(acc) * s_x) * s_w) + float(bias)), each step rounded
  * to fp32; a missing bias adds +0.0f.
+ *
+ * The last section holds ConvRot NVFP4 (FP4 E2M1 codes with E4M3 block
+ * scales), with its own sources and readings stated there.
  */
 #include <math.h>
 #include <stdint.h>
@@ -422,4 +425,247 @@ int oracle_num_threads(void) {
 #else
     return 1;
 #endif
+}
+
+/* ===================================================================== NVFP4
+ * ConvRot NVFP4 (ComfyUI-HSWQ-Loader-and-Tools, "NVFP4 torch.compile Fix",
+ * section 5-1, nvfp4_gemm.py): FP4 E2M1 codes with one scale per 16 values
+ * along K, the block scales kept in the cuBLAS 128 x 4 blocked layout that
+ * from_blocked undoes, and a per-tensor scale; dequantisation is the code's
+ * value times (per-tensor scale x block scale), and the linear is
+ * a_dq @ w_dq.T (+ bias). The pages print no quantiser; the reading here is
+ * the usual two-level NVFP4 one, on the ConvRot256-rotated rows:
+ *   s_t = amax(tensor) / 2688            (6 = largest E2M1, 448 = largest E4M3)
+ *   b   = E4M3_rne_sat((amax(block) / 6) / s_t)       (0 when s_t == 0)
+ *   d   = float(b) * s_t
+ *   q   = E2M1_rne_sat(y / d)            (+0 when d == 0)
+ * Two codes per byte, element 2j in the low nibble (the tensor cores' order;
+ * the page's decoder also reads the high nibble first, hi_first). */
+
+/* E2M1: sign bit 3, exponent bits 2-1 (bias 1), mantissa bit 0; exponent 0
+ * holds 0 and 0.5. Values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives. */
+float oracle_e2m1_to_f32(uint8_t c) {
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    float mag = (e == 0) ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Nearest E2M1 value, ties to the even mantissa, magnitudes above 6 saturate
+ * to 6; the sign is kept (a negative value that rounds to zero gives -0).
+ * The distances to the two nearest candidates are exact (Sterbenz), so ties
+ * are seen exactly. */
+uint8_t oracle_f32_to_e2m1_rne(float v) {
+    uint8_t sign = signbit(v) ? 8u : 0u;
+    float a = fabsf(v);
+    if (a >= 6.0f)
+        return (uint8_t)(sign | 7u);
+    uint8_t best = 0;
+    float bestd = a;
+    for (uint8_t c = 1; c < 8; ++c) {
+        float d = fabsf(a - oracle_e2m1_to_f32(c));
+        if (d < bestd || (d == bestd && (c & 1u) == 0)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* E4M3 (the finite-only variant): sign bit 7, exponent bits 6-3 (bias 7),
+ * mantissa bits 2-0; exponent 0 is subnormal (m * 2^-9); largest 448. */
+float oracle_e4m3_to_f32(uint8_t b) {
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    float mag = (e == 0) ? ldexpf((float)m, -9) : ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Non-negative v to the nearest E4M3 value, ties to the even mantissa,
+ * saturating at 448: with 2^E the leading power of two of v (E >= -6, the
+ * subnormals sharing the spacing of the first binade), the spacing is
+ * u = 2^(E-3), v / u is exact and rounding it to the nearest even integer k
+ * gives the value k * u. */
+uint8_t oracle_f32_to_e4m3_rne(float v) {
+    if (!(v > 0.0f))
+        return 0;
+    if (v >= 448.0f)
+        return 0x7E;
+    int e;
+    frexpf(v, &e);
+    int E = e - 1;
+    if (E < -6)
+        E = -6;
+    float u = ldexpf(1.0f, E - 3);
+    float k = nearbyintf(v / u);
+    float r = k * u;
+    if (r == 0.0f)
+        return 0;
+    frexpf(r, &e);
+    E = e - 1;
+    if (E < -6)
+        return (uint8_t)(r / ldexpf(1.0f, -9)); /* subnormal: m * 2^-9 */
+    int m = (int)(r / ldexpf(1.0f, E - 3)) - 8;
+    return (uint8_t)(((E + 7) << 3) | m);
+}
+
+/* Byte offset of the scale of row r, scale column c (= k / 16) among C
+ * columns, in the blocked layout: 512-byte tiles of 128 rows x 4 columns,
+ * tiles in row-block-major order with the column blocks fastest; inside a
+ * tile, rows r, r + 32, r + 64, r + 96 share the 16-byte line r % 32. */
+int64_t oracle_nvfp4_sf_offset(int64_t r, int64_t c, int64_t C) {
+    int64_t tiles_c = (C + 3) / 4;
+    int64_t tile = (r / 128) * tiles_c + c / 4;
+    return tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4;
+}
+
+/* Bytes of the blocked scales of a [R, K] tensor (rows padded to 128, scale
+ * columns to 4; padding bytes are zero). */
+int64_t oracle_nvfp4_sf_bytes(int64_t R, int64_t K) {
+    return ((R + 127) / 128) * 128 * (((K / 16) + 3) / 4) * 4;
+}
+
+static void nvfp4_load_rotated(const void *X, int bf16, int64_t ldx, int64_t r, int64_t K,
+                               float *buf) {
+    for (int64_t k = 0; k < K; ++k)
+        buf[k] = bf16 ? oracle_bf16_to_f32(((const uint16_t *)X)[r * ldx + k])
+                      : ((const float *)X)[r * ldx + k];
+    for (int64_t b = 0; b < K; b += ROT_N)
+        oracle_rot256(buf + b);
+}
+
+/* ConvRot NVFP4 quantisation of R rows (bf16 when bf16 != 0, else fp32) with
+ * row stride ldx: Q [R, K/2] packed codes, S the blocked block scales
+ * (oracle_nvfp4_sf_bytes(R, K) bytes), *s_t the per-tensor scale. Two passes
+ * over the rows: the tensor's absmax first, then the codes. */
+static int nvfp4_rows(const void *X, int bf16, int64_t R, int64_t K, int64_t ldx, uint8_t *Q,
+                      uint8_t *S, float *s_t_out) {
+    if (K % ROT_N != 0 || ldx < K)
+        return 1;
+    float amax = 0.0f;
+    int err = 0;
+#pragma omp parallel reduction(max : amax)
+    {
+        float *buf = (float *)malloc((size_t)K * sizeof(float));
+        if (!buf) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t r = 0; r < R; ++r) {
+                nvfp4_load_rotated(X, bf16, ldx, r, K, buf);
+                for (int64_t k = 0; k < K; ++k)
+                    if (fabsf(buf[k]) > amax)
+                        amax = fabsf(buf[k]);
+            }
+            free(buf);
+        }
+    }
+    if (err)
+        return err;
+    const float s_t = amax / 2688.0f;
+    *s_t_out = s_t;
+    const int64_t C = K / 16;
+    memset(S, 0, (size_t)oracle_nvfp4_sf_bytes(R, K));
+#pragma omp parallel
+    {
+        float *buf = (float *)malloc((size_t)K * sizeof(float));
+        if (!buf) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t r = 0; r < R; ++r) {
+                nvfp4_load_rotated(X, bf16, ldx, r, K, buf);
+                uint8_t *q = Q + r * (K / 2);
+                memset(q, 0, (size_t)(K / 2));
+                for (int64_t c = 0; c < C; ++c) {
+                    const float *y = buf + 16 * c;
+                    float ab = 0.0f;
+                    for (int i = 0; i < 16; ++i)
+                        if (fabsf(y[i]) > ab)
+                            ab = fabsf(y[i]);
+                    uint8_t b = 0;
+                    if (s_t > 0.0f) {
+                        float t = ab / 6.0f;
+                        t = t / s_t;
+                        b = oracle_f32_to_e4m3_rne(t);
+                    }
+                    S[oracle_nvfp4_sf_offset(r, c, C)] = b;
+                    const float d = oracle_e4m3_to_f32(b) * s_t;
+                    for (int i = 0; i < 16; ++i) {
+                        uint8_t code = 0;
+                        if (d != 0.0f)
+                            code = oracle_f32_to_e2m1_rne(y[i] / d);
+                        int64_t k = 16 * c + i;
+                        q[k / 2] = (uint8_t)(q[k / 2] | (code << (4 * (k & 1))));
+                    }
+                }
+            }
+            free(buf);
+        }
+    }
+    return err;
+}
+
+int oracle_quantize_rotate_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                      uint8_t *Q, uint8_t *S, float *s_t) {
+    return nvfp4_rows(X, 1, M, K, ldx, Q, S, s_t);
+}
+
+int oracle_rotate_quant_weight_nvfp4(const float *W, int64_t N, int64_t K, uint8_t *Q,
+                                     uint8_t *S, float *s_t) {
+    return nvfp4_rows(W, 0, N, K, K, Q, S, s_t);
+}
+
+/* Dequantisation as the page's decoder does it, in fp32: value =
+ * e2m1(code) * (s_t * e4m3(block scale)); hi_first reads the high nibble of
+ * each byte as the first of its two elements. */
+void oracle_dequantize_nvfp4(const uint8_t *Q, const uint8_t *S, float s_t, int64_t R, int64_t K,
+                             int hi_first, float *out) {
+    const int64_t C = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = Q[r * (K / 2) + k / 2];
+            int first = (k & 1) == 0;
+            uint8_t code = (first == hi_first) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
+            float scale = s_t * oracle_e4m3_to_f32(S[oracle_nvfp4_sf_offset(r, k / 16, C)]);
+            out[r * K + k] = oracle_e2m1_to_f32(code) * scale;
+        }
+}
+
+/* Rows of the NVFP4 linear: for each listed row m of A and every n,
+ * acc = sum_k (e2m1(qa) e4m3(ba)) (e2m1(qw) e4m3(bw)) summed in double (each
+ * term is exact), Y = bf16_rne(fl(fl(float(acc) * alpha) + bias)) with
+ * alpha = fl(s_ta * s_tw); mag = sum_k |term| * alpha (for error bounds of a
+ * float accumulation). */
+void oracle_nvfp4_linear_rows(const uint8_t *Qa, const uint8_t *Sa, float s_ta, int64_t M,
+                              const uint8_t *Qw, const uint8_t *Sw, float s_tw, int64_t N,
+                              const uint16_t *bias, int64_t K, const int64_t *rows, int64_t nrows,
+                              uint16_t *Y, double *mag) {
+    const int64_t C = K / 16;
+    const float alpha = s_ta * s_tw;
+    (void)M;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t m = rows[i];
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, am = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                uint8_t ca = (uint8_t)((Qa[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 15u);
+                uint8_t cw = (uint8_t)((Qw[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 15u);
+                double a = (double)oracle_e2m1_to_f32(ca) *
+                           (double)oracle_e4m3_to_f32(Sa[oracle_nvfp4_sf_offset(m, k / 16, C)]);
+                double w = (double)oracle_e2m1_to_f32(cw) *
+                           (double)oracle_e4m3_to_f32(Sw[oracle_nvfp4_sf_offset(n, k / 16, C)]);
+                acc += a * w;
+                am += fabs(a * w);
+            }
+            float f = (float)acc;
+            f = f * alpha;
+            f = f + (bias ? oracle_bf16_to_f32(bias[n]) : 0.0f);
+            Y[i * N + n] = oracle_f32_to_bf16_rne(f);
+            if (mag)
+                mag[i * N + n] = am * (double)alpha;
+        }
+    }
 }

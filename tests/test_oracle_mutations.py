@@ -37,6 +37,15 @@ MUTATIONS = {
     "int4_nibbles_swapped": ("(uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));",
                              "(uint8_t)(((uint8_t)q[2 * j + 1] & 0xFu) | (((uint8_t)q[2 * j] & 0xFu) << 4));"),
     "int4_unpack_no_sign": ("Q8[2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);", "Q8[2 * i] = (int8_t)lo;"),
+    "e2m1_ties_away_from_zero": ("if (d < bestd || (d == bestd && (c & 1u) == 0)) {", "if (d <= bestd) {"),
+    "e4m3_truncates": ("float k = nearbyintf(v / u);", "float k = floorf(v / u);"),
+    "nvfp4_scale_tile_lines_swapped": ("return tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4;",
+                                       "return tile * 512 + ((r % 128) / 32) * 16 + (r % 32) * 4 + c % 4;"),
+    "nvfp4_nibble_order_swapped": ("q[k / 2] = (uint8_t)(q[k / 2] | (code << (4 * (k & 1))));",
+                                   "q[k / 2] = (uint8_t)(q[k / 2] | (code << (4 * ((k + 1) & 1))));"),
+    "nvfp4_tensor_scale_constant": ("const float s_t = amax / 2688.0f;", "const float s_t = amax / 2682.0f;"),
+    "nvfp4_block_amax_signed": ("                        if (fabsf(y[i]) > ab)\n                            ab = fabsf(y[i]);",
+                                "                        if (y[i] > ab)\n                            ab = y[i];"),
     "act_not_rounded_to_bf16": ("v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));",
                                 "v = oracle_act(act, v);"),
 }
@@ -56,6 +65,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                         os.path.join(ROOT, "tests", "test_oracle_act_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_w4a4_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_w4a4_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_nvfp4_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
