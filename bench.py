@@ -45,6 +45,7 @@ UNIT = "TOPS"
 PAGE_MS = {"qkv_m32700_k5376_n16128": 10.5752, "ragged_m8193_k5376_n16128": 2.7743}
 L2_FLUSH_BYTES = 256 << 20
 NOMINAL_INT8_OVER_BF16 = 2.0  # dense tensor peaks: 4.5 POPS int8 / 2.25 PFLOP/s bf16
+NOMINAL_FP4_OVER_BF16 = 4.0  # 9 PFLOP/s dense fp4 / 2.25 PFLOP/s bf16
 
 
 def peaks():
@@ -251,12 +252,18 @@ def run_ours(args, cfg, rank, world, local_rank):
     if args.path == "w4a4":
         Qw4, s_w = ck.rotate_quant_weight_int4(W.to(dev))
         Qw = torch.empty((cfg.N, cfg.K), dtype=torch.int8, device=dev)
+    elif args.path == "nvfp4":
+        Qw, Sw, s_w = ck.rotate_quant_weight_nvfp4(W.to(dev))
     else:
         Qw, s_w = ck.rotate_quant_weight(W.to(dev))
     Wcpu = W
     M, N, K = X.shape[0], cfg.N, cfg.K
     Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
     s_x = torch.empty((M,), dtype=torch.float32, device=dev)
+    if args.path == "nvfp4":
+        Qx = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        Sx = torch.empty((ck.nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+        s_x = torch.empty((1,), dtype=torch.float32, device=dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
@@ -268,14 +275,22 @@ def run_ours(args, cfg, rank, world, local_rank):
         if args.path == "w4a4":
             ck.quantize_rotate_rowwise_int4(Xd, Qx, s_x)
             ck.unpack_int4(Qw4, out=Qw)
+        elif args.path == "nvfp4":
+            ck.quantize_rotate_nvfp4(Xd, Qx, Sx, s_x)
         elif args.act == "none":
             ck.quantize_rotate_rowwise(Xd, Qx, s_x)
         else:
             ck.quantize_rotate_rowwise_act(Xd, args.act, Qx, s_x)
 
+    def gemm():
+        if args.path == "nvfp4":
+            ck.nvfp4_gemm(Qx, Sx, s_x, Qw, Sw, s_w, bd, out=Y)
+        else:
+            ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+
     def step():
         quantize()
-        ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+        gemm()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -295,7 +310,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         ev[i][0].record(stream)
         quantize()
         ev[i][1].record(stream)
-        ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+        gemm()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -315,7 +330,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     ms_step, ms_q, ms_g = max_over_ranks([ms_step, ms_q, ms_g], dev)
 
     # ---- end to end through the public composite call, host buffers
-    if args.no_e2e or args.path == "w4a4":
+    if args.no_e2e or args.path in ("w4a4", "nvfp4"):
         ms_e2e = float("nan")
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
@@ -370,9 +385,15 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
     value = job_ops / (ms_step / 1e3) / 1e12
     e2e_value = job_ops / (ms_e2e / 1e3) / 1e12
     gemm_tops = ops / (ms_g / 1e3) / 1e12
-    q_bytes = 3.0 * M * K + 4.0 * M
+    if args.path == "nvfp4":
+        # bf16 X read once (the second, absmax pass is not algorithmic), packed
+        # FP4 codes and one E4M3 scale per 16 values written
+        q_bytes = 2.0 * M * K + 0.5 * M * K + M * K / 16.0 + 4.0
+        int8_peak = P["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    else:
+        q_bytes = 3.0 * M * K + 4.0 * M
+        int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     q_gbs = q_bytes / (ms_q / 1e3) / 1e9
-    int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     traffic = None
     prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(prof):
@@ -403,28 +424,36 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": args.scaling,
             "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
-            "dtype": "int8", "data": "synthetic", "impl": "ours",
+            "dtype": "fp4-e2m1" if args.path == "nvfp4" else "int8", "data": "synthetic",
+            "impl": "ours",
             "config": config_dict(cfg, world, args.scaling, args.act, args.path),
-            "roofline": {"kernel": ("gemm_i8_pair_kernel (2-SM tcgen05 kind::i8, fused epilogue, "
+            "roofline": {"kernel": ("gemm_nvfp4_kernel (tcgen05 kind::mxf4nvf4, E4M3 block "
+                                    "scales, fused epilogue)" if args.path == "nvfp4" else
+                                    "gemm_i8_pair_kernel (2-SM tcgen05 kind::i8, fused epilogue, "
                                     "TMA store)" if M > 128 else
                                     "gemm_i8_kernel (tcgen05 kind::i8, fused epilogue)"),
                          "bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tops / int8_peak, "traffic": traffic,
                          "peak_source": f"{P['source']} bf16 burst {P['bf16_tflops']} TFLOP/s x "
-                                        f"nominal int8/bf16 ratio {NOMINAL_INT8_OVER_BF16}",
-                         "frac_of_spec_4500": gemm_tops / 4500.0,
+                                        + (f"nominal fp4/bf16 ratio {NOMINAL_FP4_OVER_BF16}"
+                                           if args.path == "nvfp4" else
+                                           f"nominal int8/bf16 ratio {NOMINAL_INT8_OVER_BF16}"),
+                         ("frac_of_spec_9000" if args.path == "nvfp4" else "frac_of_spec_4500"):
+                             gemm_tops / (9000.0 if args.path == "nvfp4" else 4500.0),
                          "ms_per_launch": ms_g},
-            "quantizer": {"kernel": ("quant_rows_bulk_kernel" if K <= 28672 else
-                                     "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)",
+            "quantizer": {"kernel": ("nvfp4_amax_kernel + nvfp4_quant_kernel (ConvRot256 + "
+                                     "NVFP4, two passes over X)" if args.path == "nvfp4" else
+                                     ("quant_rows_bulk_kernel" if K <= 28672 else
+                                      "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)"),
                           "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",
                           "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
                           "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},
             "cpu_baseline": cpu,
-            "e2e": None if (args.no_e2e or args.path == "w4a4") else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
+            "e2e": None if (args.no_e2e or args.path in ("w4a4", "nvfp4")) else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
                     "call": f"ck_int8_linear_host: X from and Y to pinned host memory, chunks of "
                             f"{min(E2E_CHUNK_ROWS, M)} rows with copies overlapped with the kernels"},
-            "gpu_launches": (3 if args.path == "w4a4" else 2) * args.steps,
+            "gpu_launches": {"w4a4": 3, "nvfp4": 4}.get(args.path, 2) * args.steps,
             "clocks": clocks.summary(t_wall0, t_wall1),
         }
     return line
@@ -440,9 +469,10 @@ def main(argv=None):
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: every rank runs the whole batch (replicas); strong: the "
                          "batch's rows are split over the ranks")
-    ap.add_argument("--path", default="int8", choices=["int8", "w4a4"],
+    ap.add_argument("--path", default="int8", choices=["int8", "w4a4", "nvfp4"],
                     help="int8: int8_linear; w4a4: convrot_w4a4_linear (INT4 codes, packed "
-                         "INT4 weights unpacked per step)")
+                         "INT4 weights unpacked per step); nvfp4: ConvRot NVFP4 (two-pass "
+                         "FP4 quantiser + block-scaled FP4 GEMM)")
     ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

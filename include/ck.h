@@ -286,6 +286,61 @@ ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t
                                 const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
                                 int64_t N, int64_t K, ck_stream_t stream);
 
+/*
+ * ConvRot NVFP4 (ComfyUI-HSWQ-Loader-and-Tools, "NVFP4 torch.compile Fix",
+ * section 5-1, nvfp4_gemm.py: FP4 E2M1 codes, one scale per 16 values along
+ * K in the cuBLAS 128 x 4 blocked layout, a per-tensor scale, dequantisation
+ * as value x (per-tensor scale x block scale), a_dq @ w_dq.T + bias).
+ * Readings (the pages print no quantiser), on ConvRot256-rotated rows y:
+ *   s_t = amax(tensor) / 2688                       (fp32 division; 6 x 448)
+ *   b   = E4M3 of (amax(block of 16) / 6) / s_t, round to nearest even,
+ *         saturating at 448 (0 when s_t == 0)
+ *   q   = E2M1 of y / (float(b) * s_t), round to nearest even, saturating at
+ *         6, sign kept (+0 when the divisor is 0)
+ * Codes: [rows, K/2] bytes, element 2j in the low nibble of byte j (the
+ * tensor cores' order). Scales: ck_nvfp4_scale_bytes(rows, K) bytes, E4M3,
+ * blocked: the scale of row r, column c = k/16 sits at
+ *   ((r/128) * (K/64) + c/4) * 512 + (r%32) * 16 + ((r%128)/32) * 4 + c%4,
+ * rows padded to a multiple of 128 with zero bytes. s_t: one fp32 in device
+ * memory. Requires K % 256 == 0 and K <= 32768; pointers 16-B aligned (s_t
+ * 4-B). Codes and scales are bit-exact against the CPU oracle.
+ */
+size_t ck_nvfp4_scale_bytes(int64_t rows, int64_t K);
+
+/* bf16 X [M, K] (row stride ldx) -> Q [M, K/2], S, *s_t (all device). Two
+ * passes over X: the rotated tensor's absmax, then the codes. */
+ck_status ck_quantize_rotate_nvfp4(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                   uint8_t *Q, uint8_t *S, float *s_t, ck_stream_t stream);
+
+/* Offline: fp32 W [N, K] (row stride K) -> Qw [N, K/2], Sw, *s_tw. */
+ck_status ck_rotate_quant_weight_nvfp4(const float *W, int64_t N, int64_t K, uint8_t *Qw,
+                                       uint8_t *Sw, float *s_tw, ck_stream_t stream);
+
+/* Decoding as the page's dequantiser, in fp32: out[r][k] =
+ * e2m1(code) * (s_t * e4m3(scale)); hi_first != 0 reads the high nibble of
+ * each byte as the first of its two elements (the page's default order). */
+ck_status ck_dequantize_nvfp4(const uint8_t *Q, const uint8_t *S, const float *s_t, int64_t rows,
+                              int64_t K, int hi_first, float *out, ck_stream_t stream);
+
+/* Block-scaled FP4 GEMM (tcgen05 kind::mxf4nvf4) with the epilogue
+ * Y = bf16_rne(fl(acc * fl(s_ta * s_tw)) + float(bias)); acc is the tensor
+ * cores' fp32 sum of the exact products (summation order theirs), so Y
+ * matches the oracle within the float accumulation bound, not bit for bit.
+ * Requires N % 8 == 0 (plus the constraints above). */
+ck_status ck_nvfp4_gemm(const uint8_t *Qa, const uint8_t *Sa, const float *s_ta,
+                        const uint8_t *Qw, const uint8_t *Sw, const float *s_tw,
+                        const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                        ck_stream_t stream);
+
+/* ConvRot NVFP4 linear: quantise X (ck_quantize_rotate_nvfp4) into the
+ * workspace, then ck_nvfp4_gemm. Workspace: codes, scales and s_t of X, each
+ * part rounded up to 256 bytes, 256-B aligned. */
+size_t ck_convrot_nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
+ck_status ck_convrot_nvfp4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw,
+                                  const uint8_t *Sw, const float *s_tw, const ck_bf16 *bias,
+                                  ck_bf16 *Y, int64_t M, int64_t N, int64_t K, void *workspace,
+                                  size_t workspace_bytes, ck_stream_t stream);
+
 /* Size of the device array that ck_int8_linear_noalloc uses as its
  * workspace: 32 MiB, enough for ck_int8_linear_workspace_bytes(M, K) of e.g.
  * M = 4096, K = 8000 or M = 1024, K = 32512. */

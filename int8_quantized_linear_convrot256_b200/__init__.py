@@ -72,6 +72,14 @@ _SIGS = {
     "ck_quantize_int8_tensorwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_int8_linear_host_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "ck_nvfp4_scale_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "ck_quantize_rotate_nvfp4": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "ck_rotate_quant_weight_nvfp4": (_st, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "ck_dequantize_nvfp4": (_st, [_vp, _vp, _vp, _i64, _i64, _st, _vp, _vp]),
+    "ck_nvfp4_gemm": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "ck_convrot_nvfp4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "ck_convrot_nvfp4_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                      ctypes.c_size_t, _vp]),
     "ck_int8_linear_host": (_st, [_vp, _i64, _st, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                   _vp, ctypes.c_size_t, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
@@ -459,3 +467,90 @@ def clear_device_error() -> None:
 
 def inject_producer_stall(mode: int = 1, wait_limit_ns: int = 0) -> None:
     _check(lib.ck_test_inject_producer_stall(mode, wait_limit_ns), "ck_test_inject_producer_stall")
+
+
+# ----------------------------------------------------------------- ConvRot NVFP4
+
+
+def nvfp4_scale_bytes(rows: int, K: int) -> int:
+    return int(lib.ck_nvfp4_scale_bytes(rows, K))
+
+
+def _nvfp4_out(rows, K, device):
+    Q = torch.empty((rows, K // 2), dtype=torch.uint8, device=device)
+    S = torch.empty((max(nvfp4_scale_bytes(rows, K), 1),), dtype=torch.uint8, device=device)
+    s_t = torch.empty((1,), dtype=torch.float32, device=device)
+    return Q, S, s_t
+
+
+def quantize_rotate_nvfp4(X: torch.Tensor, Q=None, S=None, s_t=None, stream=None):
+    """ConvRot NVFP4 of bf16 X [M, K]: (codes [M, K/2] uint8, blocked E4M3
+    scales (uint8), per-tensor scale [1] fp32), all on X's device; Q, S and
+    s_t may be given (sizes as returned)."""
+    _need(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if Q is None or S is None or s_t is None:
+        Q, S, s_t = _nvfp4_out(M, K, X.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_quantize_rotate_nvfp4(_ptr(X), M, K, ldx, _ptr(Q), _ptr(S), _ptr(s_t),
+                                        _stream(stream)), "ck_quantize_rotate_nvfp4")
+    return Q, S, s_t
+
+
+def rotate_quant_weight_nvfp4(W: torch.Tensor, stream=None):
+    _need(W, "W", torch.float32, 2)
+    _rows_contiguous(W, "W")
+    N, K = W.shape
+    Q, S, s_t = _nvfp4_out(N, K, W.device)
+    _check(lib.ck_rotate_quant_weight_nvfp4(_ptr(W), N, K, _ptr(Q), _ptr(S), _ptr(s_t),
+                                            _stream(stream)), "ck_rotate_quant_weight_nvfp4")
+    return Q, S, s_t
+
+
+def dequantize_nvfp4(Q: torch.Tensor, S: torch.Tensor, s_t: torch.Tensor, hi_first: bool = False,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(Q, "Q", torch.uint8, 2)
+    rows, K2 = Q.shape
+    if out is None:
+        out = torch.empty((rows, 2 * K2), dtype=torch.float32, device=Q.device)
+    _check(lib.ck_dequantize_nvfp4(_ptr(Q), _ptr(S), _ptr(s_t), rows, 2 * K2, int(bool(hi_first)),
+                                   _ptr(out), _stream(stream)), "ck_dequantize_nvfp4")
+    return out
+
+
+def nvfp4_gemm(Qa, Sa, s_ta, Qw, Sw, s_tw, bias: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(Qa, "Qa", torch.uint8, 2)
+    _need(Qw, "Qw", torch.uint8, 2)
+    M, K2 = Qa.shape
+    N = Qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Qa.device)
+    _check(lib.ck_nvfp4_gemm(_ptr(Qa), _ptr(Sa), _ptr(s_ta), _ptr(Qw), _ptr(Sw), _ptr(s_tw),
+                             _ptr(bias), _ptr(out), M, N, 2 * K2, _stream(stream)), "ck_nvfp4_gemm")
+    return out
+
+
+def nvfp4_workspace_bytes(M: int, K: int) -> int:
+    return int(lib.ck_convrot_nvfp4_linear_workspace_bytes(M, K))
+
+
+def convrot_nvfp4_linear(X: torch.Tensor, Qw, Sw, s_tw, bias: torch.Tensor | None = None,
+                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """ConvRot NVFP4 linear: rotate + NVFP4-quantise X, block-scaled FP4 GEMM,
+    Y = bf16(acc * s_ta * s_tw + bias)."""
+    _need(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    N = Qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = nvfp4_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_convrot_nvfp4_linear(_ptr(X), ldx, _ptr(Qw), _ptr(Sw), _ptr(s_tw), _ptr(bias),
+                                       _ptr(out), M, N, K, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)), "ck_convrot_nvfp4_linear")
+    return out

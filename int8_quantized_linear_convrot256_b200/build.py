@@ -35,7 +35,8 @@ PER_FILE = {
     "quant_rotate.cu": ["-fmad=false"],
     "dequant.cu": ["-fmad=false"],
 }
-SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "noalloc.cu", "dequant.cu"]
+SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "gemm_nvfp4_tcgen05.cu", "noalloc.cu",
+           "dequant.cu"]
 HEADERS = ["ck_device.cuh", "internal.h", "libck.map"]
 
 

@@ -463,6 +463,170 @@ ck_status ck_int8_linear_host(const ck_bf16 *X_host, int64_t ldx, int act, const
     return CK_OK;
 }
 
+// ---------------------------------------------------------------- NVFP4
+
+size_t ck_nvfp4_scale_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return size_t((rows + 127) / 128) * 128 * size_t(K / 16);
+}
+
+namespace {
+constexpr int64_t kNvfp4MaxK = 32768;
+
+ck_status nvfp4_check_k(int64_t K) {
+    if (K <= 0) return CK_ERR_INVALID_VALUE;
+    if (K % kBlock != 0 || K > kNvfp4MaxK) return CK_ERR_UNSUPPORTED_SHAPE;
+    return CK_OK;
+}
+}  // namespace
+
+ck_status ck_quantize_rotate_nvfp4(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
+                                   uint8_t *Q, uint8_t *S, float *s_t, ck_stream_t stream) {
+    if (M < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = nvfp4_check_k(K);
+    if (s == CK_ERR_INVALID_VALUE || ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && (!X || !Q || !S || !s_t)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (M >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return CK_OK;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Q) || !aligned16(S) || !aligned4(s_t))
+        return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return ck::launch_quant_nvfp4_bf16(X, M, K, ldx, Q, S, ck_nvfp4_scale_bytes(M, K), s_t,
+                                       reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CK_OK
+               : CK_ERR_CUDA;
+}
+
+ck_status ck_rotate_quant_weight_nvfp4(const float *W, int64_t N, int64_t K, uint8_t *Qw,
+                                       uint8_t *Sw, float *s_tw, ck_stream_t stream) {
+    if (N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = nvfp4_check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (N > 0 && (!W || !Qw || !Sw || !s_tw)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return CK_OK;
+    if (!aligned16(W) || !aligned16(Qw) || !aligned16(Sw) || !aligned4(s_tw))
+        return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return ck::launch_quant_nvfp4_f32(W, N, K, Qw, Sw, ck_nvfp4_scale_bytes(N, K), s_tw,
+                                      reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CK_OK
+               : CK_ERR_CUDA;
+}
+
+ck_status ck_dequantize_nvfp4(const uint8_t *Q, const uint8_t *S, const float *s_t, int64_t rows,
+                              int64_t K, int hi_first, float *out, ck_stream_t stream) {
+    if (rows < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = nvfp4_check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (rows > 0 && (!Q || !S || !s_t || !out)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (rows == 0) return CK_OK;
+    if (!aligned16(Q) || !aligned16(out) || !aligned4(s_t)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return ck::launch_dequant_nvfp4(Q, S, s_t, rows, K, hi_first != 0, out, st->num_sms,
+                                    reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CK_OK
+               : CK_ERR_CUDA;
+}
+
+namespace {
+ck_status nvfp4_gemm_checked(const uint8_t *Qa, const uint8_t *Sa, const float *s_ta,
+                             const uint8_t *Qw, const uint8_t *Sw, const float *s_tw,
+                             const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                             DeviceState *st, cudaStream_t stream) {
+    CUtensorMap tmA, tmB;
+    std::memset(&tmA, 0, sizeof tmA);
+    std::memset(&tmB, 0, sizeof tmB);
+    ck_status s = make_tmap_i8(&tmA, Qa, M, K / 2, ck::kNvfp4BM);
+    if (s != CK_OK) return s;
+    s = make_tmap_i8(&tmB, Qw, N, K / 2, ck::kNvfp4BN);
+    if (s != CK_OK) return s;
+    ck::Nvfp4GemmParams p{};
+    p.sfa = Sa;
+    p.sfb = Sw;
+    p.s_ta = s_ta;
+    p.s_tb = s_tw;
+    p.bias = bias;
+    p.Y = Y;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.err = st->err;
+    p.wait_limit_ns = ck::kDefaultWaitLimitNs;
+    return ck::launch_gemm_nvfp4(tmA, tmB, p, st->num_sms, stream) == cudaSuccess ? CK_OK
+                                                                                  : CK_ERR_CUDA;
+}
+}  // namespace
+
+ck_status ck_nvfp4_gemm(const uint8_t *Qa, const uint8_t *Sa, const float *s_ta,
+                        const uint8_t *Qw, const uint8_t *Sw, const float *s_tw,
+                        const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                        ck_stream_t stream) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = nvfp4_check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (M > 0 && N > 0 && (!Qa || !Sa || !s_ta || !Qw || !Sw || !s_tw || !Y))
+        return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(Qa) || !aligned16(Sa) || !aligned16(Qw) || !aligned16(Sw) || !aligned4(s_ta) ||
+        !aligned4(s_tw) || !aligned16(Y) || (bias && !aligned16(bias)))
+        return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    return nvfp4_gemm_checked(Qa, Sa, s_ta, Qw, Sw, s_tw, bias, Y, M, N, K, st,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ck_convrot_nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return round256(size_t(M) * size_t(K / 2)) + round256(ck_nvfp4_scale_bytes(M, K)) + 256;
+}
+
+ck_status ck_convrot_nvfp4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw,
+                                  const uint8_t *Sw, const float *s_tw, const ck_bf16 *bias,
+                                  ck_bf16 *Y, int64_t M, int64_t N, int64_t K, void *workspace,
+                                  size_t workspace_bytes, ck_stream_t stream) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = nvfp4_check_k(K);
+    if (s == CK_ERR_INVALID_VALUE || ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && N > 0 && (!X || !Qw || !Sw || !s_tw || !Y || !workspace))
+        return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Qw) || !aligned16(Sw) || !aligned4(s_tw) ||
+        !aligned16(Y) || (bias && !aligned16(bias)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CK_ERR_MISALIGNED;
+    if (workspace_bytes < ck_convrot_nvfp4_linear_workspace_bytes(M, K)) return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    uint8_t *Qa = base;
+    uint8_t *Sa = base + round256(size_t(M) * size_t(K / 2));
+    float *s_ta = reinterpret_cast<float *>(Sa + round256(ck_nvfp4_scale_bytes(M, K)));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (ck::launch_quant_nvfp4_bf16(X, M, K, ldx, Qa, Sa, ck_nvfp4_scale_bytes(M, K), s_ta, cs) !=
+        cudaSuccess)
+        return CK_ERR_CUDA;
+    return nvfp4_gemm_checked(Qa, Sa, s_ta, Qw, Sw, s_tw, bias, Y, M, N, K, st, cs);
+}
+
 ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Qw4,
                                  const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
                                  int64_t N, int64_t K, void *workspace, size_t workspace_bytes,

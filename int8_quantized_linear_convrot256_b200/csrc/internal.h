@@ -23,6 +23,16 @@ cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int6
 cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int4_packed,
                                   int8_t *Q, float *S, cudaStream_t stream);
 
+// ConvRot NVFP4 quantisation (codes [rows, K/2], blocked scales of s_bytes
+// bytes, per-tensor scale in *s_t) and decoding to fp32.
+cudaError_t launch_quant_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                    uint8_t *Q, uint8_t *S, size_t s_bytes, float *s_t,
+                                    cudaStream_t stream);
+cudaError_t launch_quant_nvfp4_f32(const float *W, int64_t N, int64_t K, uint8_t *Q, uint8_t *S,
+                                   size_t s_bytes, float *s_t, cudaStream_t stream);
+cudaError_t launch_dequant_nvfp4(const uint8_t *Q, const uint8_t *S, const float *s_t,
+                                 int64_t rows, int64_t K, bool hi_first, float *out, int num_sms,
+                                 cudaStream_t stream);
 // Packed signed INT4 [rows, K/2] -> int8 [rows, K].
 cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8,
                                int num_sms, cudaStream_t stream);
@@ -76,5 +86,26 @@ constexpr int kGemmYBoxRows = 32;
 cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmY,
                            const GemmParams &p, bool raw_i32, const GemmPlan &plan,
                            cudaStream_t stream);
+
+// ---- block-scaled NVFP4 GEMM with fused epilogue (gemm_nvfp4_tcgen05.cu)
+
+struct Nvfp4GemmParams {
+    const uint8_t *sfa;     // blocked E4M3 scales of A (rows padded to 128)
+    const uint8_t *sfb;     // blocked E4M3 scales of B
+    const float *s_ta;      // per-tensor scales (device scalars)
+    const float *s_tb;
+    const uint16_t *bias;   // [N] bf16 bits or nullptr
+    uint16_t *Y;            // [M, N] bf16 bits
+    int M, N, K;
+    unsigned *err;
+    uint64_t wait_limit_ns;
+};
+
+constexpr int kNvfp4BM = 128;      // rows of A per tile (TMA box rows)
+constexpr int kNvfp4BN = 128;      // rows of B per tile
+constexpr int kNvfp4BKBytes = 128; // packed bytes of K per stage (256 values)
+
+cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                              const Nvfp4GemmParams &p, int num_sms, cudaStream_t stream);
 
 }  // namespace ck

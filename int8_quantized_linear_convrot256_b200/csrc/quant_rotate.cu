@@ -56,6 +56,7 @@
 //    (rows re-read from L2); fp32 weights (offline) take direct loads.
 //  * No FMA contraction: every operation is an explicit _rn intrinsic.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -858,6 +859,164 @@ __global__ void unpack_int4_kernel(const uint4 *__restrict__ in, uint4 *__restri
     }
 }
 
+// ------------------------------------------------------------------ NVFP4
+// ConvRot NVFP4 (ComfyUI-HSWQ-Loader-and-Tools, "NVFP4 torch.compile Fix",
+// section 5-1: FP4 E2M1 codes, one E4M3 scale per 16 values, the 128 x 4
+// blocked scale layout, a per-tensor scale). On the ConvRot256-rotated rows:
+//   s_t = amax(tensor) / 2688, b = E4M3_rne_sat((amax(block) / 6) / s_t),
+//   d = float(b) * s_t, q = E2M1_rne_sat(y / d) (+0 when d == 0),
+// two codes per byte with the lower element in the low nibble. The
+// conversions use the hardware's round-to-nearest-even, saturating cvt; each
+// cvt gets the same value twice, so the result does not depend on which half
+// of the packed pair an operand lands in.
+
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(v));
+    return uint32_t(r) & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const uint16_t pair = uint16_t(b | (b << 8));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    return __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ uint32_t e2m1_rne_sat(float v) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u16.u8 %0, t;\n\t}"
+        : "=h"(r) : "f"(v));
+    return uint32_t(r) & 0xFu;
+}
+
+// Offset of the scale of row r, scale column c (of C) in the blocked layout:
+// 512-byte tiles of 128 rows x 4 columns, column tiles fastest; rows r, r + 32,
+// r + 64, r + 96 of a tile share the 16-byte line r % 32.
+__device__ __forceinline__ int64_t nvfp4_sf_offset(int64_t r, int c, int C) {
+    const int64_t tile = (r >> 7) * int64_t((C + 3) >> 2) + (c >> 2);
+    return tile * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
+}
+
+// Pass 1: absmax of the rotated tensor (of z = 16 y), as the bits of a
+// non-negative float, atomicMax'ed into *amax_bits (zeroed before).
+template <typename TIn>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+nvfp4_amax_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
+                  unsigned *amax_bits) {
+    __shared__ unsigned s_max;
+    const int tid = threadIdx.x;
+    const int t = tid & 3;
+    const int quad = tid >> 2;
+    const int nb = K >> 8;
+    const int row_local = quad / nb;
+    const int blk = quad - row_local * nb;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + row_local;
+    const bool active = row_local < rows_per_cta && row < M;
+    if (tid == 0) s_max = 0u;
+    float2 P[kPairs];
+    if (active)
+        load_block<kActNone>(X + row * ldx + blk * kBlock + 8 * t, P);
+    else
+        zero_block(P);
+    butterflies(P, t);
+    const float m = block_absmax(P);
+    __syncthreads();
+    if (active && t == 0) atomicMax(&s_max, __float_as_uint(m));
+    __syncthreads();
+    if (tid == 0 && s_max != 0u) atomicMax(amax_bits, s_max);
+}
+
+// Pass 2: block scales and codes. Lane t of a quad holds elements
+// 8t + 32i .. +7 of its 256-block (chunk i); a 16-value scale block is chunk
+// i of lanes t and t ^ 1.
+template <typename TIn>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
+                   const unsigned *__restrict__ amax_bits, uint8_t *__restrict__ Q,
+                   uint8_t *__restrict__ S) {
+    const int tid = threadIdx.x;
+    const int t = tid & 3;
+    const int quad = tid >> 2;
+    const int nb = K >> 8;
+    const int row_local = quad / nb;
+    const int blk = quad - row_local * nb;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + row_local;
+    const bool active = row_local < rows_per_cta && row < M;
+    const int col0 = blk * kBlock + 8 * t;
+    float2 P[kPairs];
+    if (active)
+        load_block<kActNone>(X + row * ldx + col0, P);
+    else
+        zero_block(P);
+    butterflies(P, t);
+    const float amax = __fmul_rn(__uint_as_float(*amax_bits), 0.0625f);
+    const float s_t = __fdiv_rn(amax, 2688.0f);
+    const int C = K >> 4;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float y[8];
+        float m8 = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 z = P[4 * i + k];
+            y[2 * k] = __fmul_rn(z.x, 0.0625f);
+            y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
+            m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
+        }
+        const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
+        uint32_t b = 0;
+        if (s_t > 0.0f) b = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
+        const float d = __fmul_rn(e4m3_to_f32(b), s_t);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float v = d != 0.0f ? __fdiv_rn(y[j], d) : 0.0f;
+            packed |= e2m1_rne_sat(v) << (4 * j);
+        }
+        if (active) {
+            const int e0 = col0 + 32 * i;
+            *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
+            if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(b);
+        }
+    }
+}
+
+// Turns the absmax bits of z into the per-tensor scale, in place.
+__global__ void nvfp4_scale_kernel(float *s_t) {
+    const float amax = __fmul_rn(__uint_as_float(*reinterpret_cast<unsigned *>(s_t)), 0.0625f);
+    *s_t = __fdiv_rn(amax, 2688.0f);
+}
+
+// Decoding: value = e2m1(code) * (s_t * e4m3(scale)); 8 values per thread.
+__global__ void nvfp4_dequant_kernel(const uint8_t *__restrict__ Q, const uint8_t *__restrict__ S,
+                                     const float *__restrict__ s_t, int64_t rows, int K,
+                                     int hi_first, float *__restrict__ out) {
+    const int C = K >> 4;
+    const int64_t groups = rows * int64_t(K / 8);
+    const float st = *s_t;
+    for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+         g += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = g / (K / 8);
+        const int k0 = int(g - r * (K / 8)) * 8;
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(Q + r * int64_t(K / 2) + k0 / 2);
+        const float scale = __fmul_rn(st, e4m3_to_f32(S[nvfp4_sf_offset(r, k0 >> 4, C)]));
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t byte = (w >> (8 * (j >> 1))) & 0xFFu;
+            const bool high = ((j & 1) == 0) == (hi_first != 0);
+            const uint32_t c = high ? (byte >> 4) : (byte & 15u);
+            const uint32_t e = (c >> 1) & 3u, mbit = c & 1u;
+            float mag = e == 0 ? 0.5f * float(mbit) : __uint_as_float((e + 126u) << 23) * (1.0f + 0.5f * float(mbit));
+            v[j] = __fmul_rn((c & 8u) ? -mag : mag, scale);
+        }
+        float4 *o = reinterpret_cast<float4 *>(out + r * int64_t(K) + k0);
+        o[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
@@ -890,6 +1049,49 @@ cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_
     const int64_t cap = int64_t(num_sms) * 8;
     unpack_int4_kernel<<<unsigned(want < cap ? want : cap), 256, 0, stream>>>(
         reinterpret_cast<const uint4 *>(Q4), reinterpret_cast<uint4 *>(Q8), n16);
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_nvfp4_impl(const TIn *X, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
+                              uint8_t *S, size_t s_bytes, float *s_t, cudaStream_t stream) {
+    if (M <= 0) return cudaSuccess;
+    const int nb = static_cast<int>(K / kBlock);
+    if (4 * nb > kMaxThreads) return cudaErrorInvalidValue;
+    int threads = 0;
+    const int rows = pick_rows_per_cta(nb, 4, kMaxRowsPerCta, kMaxThreads, 256, &threads);
+    const unsigned grid = static_cast<unsigned>((M + rows - 1) / rows);
+    cudaError_t e = cudaMemsetAsync(s_t, 0, sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(S, 0, s_bytes, stream);
+    if (e != cudaSuccess) return e;
+    nvfp4_amax_kernel<TIn><<<grid, threads, 0, stream>>>(X, M, static_cast<int>(K), ldx, rows,
+                                                       reinterpret_cast<unsigned *>(s_t));
+    nvfp4_quant_kernel<TIn><<<grid, threads, 0, stream>>>(
+        X, M, static_cast<int>(K), ldx, rows, reinterpret_cast<const unsigned *>(s_t), Q, S);
+    nvfp4_scale_kernel<<<1, 1, 0, stream>>>(s_t);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                    uint8_t *Q, uint8_t *S, size_t s_bytes, float *s_t,
+                                    cudaStream_t stream) {
+    return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
+}
+
+cudaError_t launch_quant_nvfp4_f32(const float *W, int64_t N, int64_t K, uint8_t *Q, uint8_t *S,
+                                   size_t s_bytes, float *s_t, cudaStream_t stream) {
+    return launch_nvfp4_impl(W, N, K, K, Q, S, s_bytes, s_t, stream);
+}
+
+cudaError_t launch_dequant_nvfp4(const uint8_t *Q, const uint8_t *S, const float *s_t,
+                                 int64_t rows, int64_t K, bool hi_first, float *out, int num_sms,
+                                 cudaStream_t stream) {
+    const int64_t groups = rows * (K / 8);
+    if (groups <= 0) return cudaSuccess;
+    const int64_t want = (groups + 255) / 256;
+    const int64_t cap = int64_t(num_sms) * 8;
+    nvfp4_dequant_kernel<<<unsigned(want < cap ? want : cap), 256, 0, stream>>>(
+        Q, S, s_t, rows, static_cast<int>(K), hi_first ? 1 : 0, out);
     return cudaGetLastError();
 }
 

@@ -155,3 +155,40 @@ def test_host_workspace_bytes():
 ])
 def test_int8_linear_host_validation(kw, status):
     assert lin_host(**kw) == status
+
+
+def test_nvfp4_scale_bytes():
+    assert ck.nvfp4_scale_bytes(0, 256) == 0
+    assert ck.nvfp4_scale_bytes(1, 256) == 128 * 16
+    assert ck.nvfp4_scale_bytes(129, 5376) == 256 * 336
+    assert ck.nvfp4_workspace_bytes(3, 256) == 512 + 2048 + 256
+
+
+@pytest.mark.parametrize("call,status", [
+    (lambda: ck.lib.ck_quantize_rotate_nvfp4(FAKE, 4, 512, 512, FAKE, FAKE, FAKE, None), None),
+    (lambda: ck.lib.ck_quantize_rotate_nvfp4(FAKE, 4, 33024, 33024, FAKE, FAKE, FAKE, None),
+     ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (lambda: ck.lib.ck_quantize_rotate_nvfp4(FAKE, 4, 300, 512, FAKE, FAKE, FAKE, None),
+     ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (lambda: ck.lib.ck_quantize_rotate_nvfp4(None, 4, 512, 512, FAKE, FAKE, FAKE, None),
+     ck.CK_ERR_INVALID_VALUE),
+    (lambda: ck.lib.ck_quantize_rotate_nvfp4(FAKE, 4, 512, 512, MIS, FAKE, FAKE, None),
+     ck.CK_ERR_MISALIGNED),
+    (lambda: ck.lib.ck_rotate_quant_weight_nvfp4(FAKE, 4, 512, FAKE, MIS, FAKE, None),
+     ck.CK_ERR_MISALIGNED),
+    (lambda: ck.lib.ck_nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 12, 512, None),
+     ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (lambda: ck.lib.ck_nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 4, 8, 512, None),
+     ck.CK_ERR_INVALID_VALUE),
+    (lambda: ck.lib.ck_nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 0, 8, 512, None),
+     ck.CK_OK),
+    (lambda: ck.lib.ck_convrot_nvfp4_linear(FAKE, 512, FAKE, FAKE, FAKE, None, FAKE, 4, 8, 512, FAKE,
+                                            16, None), ck.CK_ERR_WORKSPACE),
+    (lambda: ck.lib.ck_dequantize_nvfp4(FAKE, FAKE, FAKE, 4, 512, 0, MIS, None), ck.CK_ERR_MISALIGNED),
+])
+def test_nvfp4_validation(call, status):
+    got = call()
+    if status is None:  # a valid call: without a GPU it can only fail in the CUDA runtime
+        assert got in (ck.CK_ERR_CUDA, ck.CK_ERR_ARCH)
+    else:
+        assert got == status

@@ -1,0 +1,116 @@
+"""ConvRot NVFP4 on the GPU against the CPU oracle (through the C ABI).
+
+Codes, block scales, the per-tensor scale and decoded values are compared bit
+for bit. The block-scaled GEMM accumulates the exact products in the tensor
+cores' fp32 (their summation order), so its outputs are compared with the
+oracle's (double-precision sum, then the same fp32 epilogue) within one bf16
+ulp plus the float accumulation bound K * 2^-24 * sum|products| * alpha.
+Source: ComfyUI-HSWQ-Loader-and-Tools, "NVFP4 torch.compile Fix", section 5-1.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ck():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import int8_quantized_linear_convrot256_b200 as m
+
+    m.clear_device_error()
+    yield m
+    assert m.device_error() == m.CK_OK
+
+
+def _np(t):
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (37, 768), (130, 5376), (5, 28672), (300, 512)])
+def test_quantize_rotate_nvfp4_bit_exact(ck, M, K):
+    cfg = workloads.custom(M, K, 8, seed=M * 7 + K)
+    X, _, _ = workloads.make_inputs(cfg)
+    Qr, Sr, sr = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X))
+    Q, S, s_t = ck.quantize_rotate_nvfp4(X.cuda())
+    assert np.float32(_np(s_t)[0]) == np.float32(sr)
+    assert np.array_equal(_np(S)[: Sr.size], Sr)
+    assert np.array_equal(_np(Q), Qr)
+
+
+@pytest.mark.parametrize("N,K", [(264, 768), (520, 5376), (8, 256)])
+def test_rotate_quant_weight_nvfp4_bit_exact(ck, N, K):
+    cfg = workloads.custom(4, K, N, seed=N + K)
+    _, W, _ = workloads.make_inputs(cfg)
+    Qr, Sr, sr = oracle.rotate_quant_weight_nvfp4(W.numpy())
+    Q, S, s_t = ck.rotate_quant_weight_nvfp4(W.cuda())
+    assert np.float32(_np(s_t)[0]) == np.float32(sr)
+    assert np.array_equal(_np(S)[: Sr.size], Sr)
+    assert np.array_equal(_np(Q), Qr)
+
+
+def test_quantize_nvfp4_zero_and_scaled_tensors(ck):
+    Z = torch.zeros((3, 512), dtype=torch.bfloat16, device="cuda")
+    Q, S, s_t = ck.quantize_rotate_nvfp4(Z)
+    assert float(s_t[0]) == 0.0 and not Q.any() and not S.any()
+    cfg = workloads.custom(6, 512, 8, seed=3)
+    X, _, _ = workloads.make_inputs(cfg)
+    a = ck.quantize_rotate_nvfp4(X.cuda())
+    b = ck.quantize_rotate_nvfp4((X * 4).cuda())
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and float(b[2][0]) == 4 * float(a[2][0])
+
+
+@pytest.mark.parametrize("hi_first", [False, True])
+def test_dequantize_nvfp4_bit_exact(ck, hi_first):
+    cfg = workloads.custom(33, 768, 8, seed=21)
+    X, _, _ = workloads.make_inputs(cfg)
+    Q, S, s_t = ck.quantize_rotate_nvfp4(X.cuda())
+    got = _np(ck.dequantize_nvfp4(Q, S, s_t, hi_first=hi_first))
+    want = oracle.dequantize_nvfp4(_np(Q), _np(S), float(_np(s_t)[0]), hi_first=hi_first)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def _bf16_val(bits):
+    return workloads.from_bf16_bits(bits).double().numpy()
+
+
+def _assert_gemm_close(Y_bits, Yr_bits, mag, K):
+    y, r = _bf16_val(Y_bits), _bf16_val(Yr_bits)
+    ulp = np.maximum(np.abs(r), np.abs(y)) * 2.0 ** -7  # one bf16 ulp, generously
+    tol = ulp + K * 2.0 ** -24 * mag + 1e-30
+    bad = np.abs(y - r) > tol
+    assert not bad.any(), f"{bad.sum()} outputs off, first at {np.argwhere(bad)[0]}: {y[bad][0]} vs {r[bad][0]}"
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 256, 128), (1, 256, 8), (129, 768, 264), (300, 5376, 520),
+                                   (257, 1024, 136)])
+def test_nvfp4_gemm_matches_oracle(ck, M, K, N):
+    cfg = workloads.custom(M, K, N, seed=M + 3 * N + K)
+    X, W, bias = workloads.make_inputs(cfg)
+    Qa, Sa, sa = ck.quantize_rotate_nvfp4(X.cuda())
+    Qw, Sw, sw = ck.rotate_quant_weight_nvfp4(W.cuda())
+    Y = ck.nvfp4_gemm(Qa, Sa, sa, Qw, Sw, sw, bias.cuda())
+    Yr, mag = oracle.nvfp4_linear_rows(_np(Qa), _np(Sa), float(_np(sa)[0]), _np(Qw), _np(Sw),
+                                       float(_np(sw)[0]), workloads.bf16_bits(bias))
+    _assert_gemm_close(workloads.bf16_bits(Y.cpu()), Yr, mag, K)
+
+
+def test_convrot_nvfp4_linear_matches_oracle_and_fp64(ck):
+    M, K, N = 200, 1024, 264
+    cfg = workloads.custom(M, K, N, seed=31)
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw, Sw, sw = ck.rotate_quant_weight_nvfp4(W.cuda())
+    Y = ck.convrot_nvfp4_linear(X.cuda(), Qw, Sw, sw, bias.cuda())
+    Qa, Sa, sa = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X))
+    Yr, mag = oracle.nvfp4_linear_rows(Qa, Sa, sa, _np(Qw), _np(Sw), float(_np(sw)[0]),
+                                       workloads.bf16_bits(bias))
+    _assert_gemm_close(workloads.bf16_bits(Y.cpu()), Yr, mag, K)
+    # and the quantised linear is close to the unquantised one (FP4: a few per cent)
+    ref = X.double().numpy() @ W.double().numpy().T + _bf16_val(workloads.bf16_bits(bias))[None, :]
+    rel = np.linalg.norm(_bf16_val(workloads.bf16_bits(Y.cpu())) - ref) / np.linalg.norm(ref)
+    assert rel < 0.2, rel
