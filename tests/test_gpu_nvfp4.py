@@ -114,3 +114,27 @@ def test_convrot_nvfp4_linear_matches_oracle_and_fp64(ck):
     ref = X.double().numpy() @ W.double().numpy().T + _bf16_val(workloads.bf16_bits(bias))[None, :]
     rel = np.linalg.norm(_bf16_val(workloads.bf16_bits(Y.cpu())) - ref) / np.linalg.norm(ref)
     assert rel < 0.2, rel
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["ragged_m8193_k5376_n16128", "qkv_m32700_k5376_n16128"])
+def test_full_size_nvfp4_codes_and_sampled_rows(ck, name):
+    """The benchmark's shapes: every code and scale bit-exact, and sampled
+    output rows (first, last, tile edges, random) within the GEMM bound."""
+    cfg = workloads.BY_NAME[name]
+    X, W, bias = workloads.make_inputs(cfg)
+    Qr, Sr, sr = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X))
+    Xd = X.cuda()
+    Qw, Sw, sw = ck.rotate_quant_weight_nvfp4(W.cuda())
+    Qa, Sa, sa = ck.quantize_rotate_nvfp4(Xd)
+    assert np.float32(_np(sa)[0]) == np.float32(sr)
+    assert np.array_equal(_np(Sa)[: Sr.size], Sr)
+    assert np.array_equal(_np(Qa), Qr)
+    Y = ck.convrot_nvfp4_linear(Xd, Qw, Sw, sw, bias.cuda())
+    M = cfg.M
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 127, 128, M // 2, M - 1], rng.integers(0, M, 8)]))
+    Yr, mag = oracle.nvfp4_linear_rows(Qr, Sr, sr, _np(Qw), _np(Sw), float(_np(sw)[0]),
+                                       workloads.bf16_bits(bias), rows=rows)
+    got = workloads.bf16_bits(Y[torch.from_numpy(rows).cuda()].cpu())
+    _assert_gemm_close(got, Yr, mag, cfg.K)
