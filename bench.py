@@ -427,7 +427,8 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
             "dtype": "fp4-e2m1" if args.path == "nvfp4" else "int8", "data": "synthetic",
             "impl": "ours",
             "config": config_dict(cfg, world, args.scaling, args.act, args.path),
-            "roofline": {"kernel": ("gemm_nvfp4_kernel (tcgen05 kind::mxf4nvf4, E4M3 block "
+            "roofline": {"kernel": (("gemm_nvfp4_pair_kernel (2-SM " if M > 128 else
+                                     "gemm_nvfp4_kernel (") + "tcgen05 kind::mxf4nvf4, E4M3 block "
                                     "scales, fused epilogue)" if args.path == "nvfp4" else
                                     "gemm_i8_pair_kernel (2-SM tcgen05 kind::i8, fused epilogue, "
                                     "TMA store)" if M > 128 else

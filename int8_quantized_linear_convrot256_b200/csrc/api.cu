@@ -110,6 +110,20 @@ ck_status make_tmap_y(CUtensorMap *tm, const void *base, int64_t M, int64_t N) {
     return r == CUDA_SUCCESS ? CK_OK : CK_ERR_CUDA;
 }
 
+// Blocked NVFP4 scales viewed as rows of 256 bytes; box = 8 rows (2 KB, four
+// 512-byte scale tiles), no swizzle.
+ck_status make_tmap_sf(CUtensorMap *tm, const void *base, size_t bytes) {
+    cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, 8};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CK_OK : CK_ERR_CUDA;
+}
+
 ck_status run_gemm(const int8_t *Qx, const float *s_x, const int8_t *Qw, const float *s_w,
                    const ck_bf16 *bias, ck_bf16 *Y, int32_t *acc, int64_t M, int64_t N, int64_t K,
                    DeviceState *st, cudaStream_t stream) {
@@ -543,12 +557,18 @@ ck_status nvfp4_gemm_checked(const uint8_t *Qa, const uint8_t *Sa, const float *
                              const uint8_t *Qw, const uint8_t *Sw, const float *s_tw,
                              const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
                              DeviceState *st, cudaStream_t stream) {
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB;
     std::memset(&tmA, 0, sizeof tmA);
     std::memset(&tmB, 0, sizeof tmB);
+    std::memset(&tmSFA, 0, sizeof tmSFA);
+    std::memset(&tmSFB, 0, sizeof tmSFB);
     ck_status s = make_tmap_i8(&tmA, Qa, M, K / 2, ck::kNvfp4BM);
     if (s != CK_OK) return s;
     s = make_tmap_i8(&tmB, Qw, N, K / 2, ck::kNvfp4BN);
+    if (s != CK_OK) return s;
+    s = make_tmap_sf(&tmSFA, Sa, ck_nvfp4_scale_bytes(M, K));
+    if (s != CK_OK) return s;
+    s = make_tmap_sf(&tmSFB, Sw, ck_nvfp4_scale_bytes(N, K));
     if (s != CK_OK) return s;
     ck::Nvfp4GemmParams p{};
     p.sfa = Sa;
@@ -562,8 +582,10 @@ ck_status nvfp4_gemm_checked(const uint8_t *Qa, const uint8_t *Sa, const float *
     p.K = static_cast<int>(K);
     p.err = st->err;
     p.wait_limit_ns = ck::kDefaultWaitLimitNs;
-    return ck::launch_gemm_nvfp4(tmA, tmB, p, st->num_sms, stream) == cudaSuccess ? CK_OK
-                                                                                  : CK_ERR_CUDA;
+    return ck::launch_gemm_nvfp4(tmA, tmB, tmSFA, tmSFB, p, st->num_sms, true, stream) ==
+                   cudaSuccess
+               ? CK_OK
+               : CK_ERR_CUDA;
 }
 }  // namespace
 

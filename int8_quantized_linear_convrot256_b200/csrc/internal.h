@@ -105,7 +105,13 @@ constexpr int kNvfp4BM = 128;      // rows of A per tile (TMA box rows)
 constexpr int kNvfp4BN = 128;      // rows of B per tile
 constexpr int kNvfp4BKBytes = 128; // packed bytes of K per stage (256 values)
 
+// The 2-SM kernel (256 x 256 tiles per CTA pair) runs when M > 128 and
+// allow_pair, else the 1-SM 128 x 128 kernel. tmA / tmB: the packed codes
+// (boxes of 128 bytes x 128 rows, 128-byte swizzle); tmSFA / tmSFB: the
+// blocked scales as rows of 256 bytes (boxes of 256 bytes x 8 rows).
 cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB,
-                              const Nvfp4GemmParams &p, int num_sms, cudaStream_t stream);
+                              const CUtensorMap &tmSFA, const CUtensorMap &tmSFB,
+                              const Nvfp4GemmParams &p, int num_sms, bool allow_pair,
+                              cudaStream_t stream);
 
 }  // namespace ck
