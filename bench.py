@@ -183,34 +183,56 @@ def oracle_inputs(cfg):
 
 
 def run_reference(args, cfg, rank, world):
+    """The oracle, as it stands, on the host cores: each step quantises a
+    bounded sample of the batch's rows and computes all N outputs of those
+    rows (the path chosen by --path)."""
     if rank != 0:
         return 0
     import oracle
 
-    X_bits, Qw, s_w, bias_bits = oracle_inputs(cfg)
+    X, W, bias = workloads.make_inputs(cfg)
+    X_bits, bias_bits = workloads.bf16_bits(X), workloads.bf16_bits(bias)
+    if args.path == "nvfp4":
+        Qw, Sw, s_tw = oracle.rotate_quant_weight_nvfp4(W.numpy())
+
+        def run(rows):
+            Qa, Sa, s_ta = oracle.quantize_rotate_nvfp4(X_bits[:rows])
+            oracle.nvfp4_linear_rows(Qa, Sa, s_ta, Qw, Sw, s_tw, bias_bits)
+        what, dtype = "ConvRot NVFP4 quantisation of those rows + their outputs", "fp4-e2m1"
+    elif args.path == "w4a4":
+        Qw4, s_w = oracle.rotate_quant_weight_int4(W.numpy())
+
+        def run(rows):
+            oracle.convrot_w4a4_linear(X_bits[:rows], Qw4, s_w, bias_bits)
+        what, dtype = "convrot_w4a4_linear of those rows", "int8"
+    else:
+        Qw, s_w = oracle.rotate_quant_weight(W.numpy())
+
+        def run(rows):
+            Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows], act=args.act)
+            oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
+        what, dtype = "quantize_and_rotate_rowwise of those rows + their outputs", "int8"
     total_budget = 150.0
     per_step = total_budget / max(1, args.steps + args.warmup)
     t_probe = time.perf_counter()
-    Qx, s_x = oracle.quantize_rows_bf16(X_bits[:4], act=args.act)
-    oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(4))
+    run(4)
     t_row = (time.perf_counter() - t_probe) / 4
     rows = int(max(1, min(cfg.M, per_step / max(t_row, 1e-9))))
     times = []
     for i in range(args.warmup + args.steps):
         t = time.perf_counter()
-        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows], act=args.act)
-        oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
+        run(rows)
         dt = time.perf_counter() - t
         if i >= args.warmup:
             times.append(dt)
     ms = 1e3 * sum(times) / len(times)
     tops = 2.0 * rows * cfg.N * cfg.K / (ms / 1e3) / 1e12
-    sample = (f"{rows} of {cfg.M} rows per step (quantize_and_rotate_rowwise of those rows + "
-              f"their {cfg.N} outputs each), oracle in plain C on host cores")
+    sample = (f"{rows} of {cfg.M} rows per step ({what}, all {cfg.N} outputs each), oracle in "
+              f"plain C on host cores")
     line = {"metric": METRIC, "value": tops, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "impl": "reference",
-            "config": config_dict(cfg, world, "weak", args.act),
+            "vs_baseline": None, "dtype": dtype, "data": "synthetic", "impl": "reference",
+            "config": config_dict(cfg, world, "weak", args.act, args.path),
             "cpu_baseline": {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": tops, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -394,13 +416,17 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
         q_bytes = 3.0 * M * K + 4.0 * M
         int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     q_gbs = q_bytes / (ms_q / 1e3) / 1e9
+    ratio = NOMINAL_FP4_OVER_BF16 if args.path == "nvfp4" else NOMINAL_INT8_OVER_BF16
+    sustained_peak = P["bf16_tflops_sustained"] * ratio
+    # DRAM bytes of one launch of the dominant kernel, from an ncu capture of
+    # this workload (profiles/<kernel>__<workload>.dram.json), if there is one
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(prof):
+    kname = ("gemm_nvfp4_pair_kernel" if args.path == "nvfp4" else "gemm_i8_pair_kernel") \
+        if M > 128 else ("gemm_nvfp4_kernel" if args.path == "nvfp4" else "gemm_i8_kernel")
+    prof = os.path.join(ROOT, "profiles", f"{kname}__{cfg.name}.dram.json")
+    if os.path.exists(prof) and args.scaling == "weak":
         try:
-            d = json.load(open(prof))
-            if d.get("workload") == cfg.name:
-                traffic = d.get("dram_bytes_per_launch")
+            traffic = float(json.load(open(prof))["dram_bytes_per_launch"])
         except Exception:
             traffic = None
 
@@ -441,6 +467,7 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                                            f"nominal int8/bf16 ratio {NOMINAL_INT8_OVER_BF16}"),
                          ("frac_of_spec_9000" if args.path == "nvfp4" else "frac_of_spec_4500"):
                              gemm_tops / (9000.0 if args.path == "nvfp4" else 4500.0),
+                         "frac_of_measured_sustained": gemm_tops / sustained_peak,
                          "ms_per_launch": ms_g},
             "quantizer": {"kernel": ("nvfp4_amax_kernel + nvfp4_quant_kernel (ConvRot256 + "
                                      "NVFP4, two passes over X)" if args.path == "nvfp4" else

@@ -232,7 +232,10 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
  * copy back, so work queued on `stream` afterwards - or a synchronize of it -
  * sees Y_host complete. Calls on one device are queued on the same internal
  * streams in the order they are made. Nothing here blocks the host (apart
- * from what the driver does for pageable memory).
+ * from what the driver does for pageable memory). Validation failures
+ * enqueue nothing; a CUDA error returned while chunks are being enqueued
+ * (CK_ERR_CUDA) can leave earlier chunks queued, and Y_host is then
+ * undefined.
  */
 size_t ck_int8_linear_host_workspace_bytes(int64_t chunk_rows, int64_t N, int64_t K);
 ck_status ck_int8_linear_host(const ck_bf16 *X_host, int64_t ldx, int act, const int8_t *Qw,
