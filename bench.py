@@ -349,7 +349,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     ms_step = sum(s_ms) / len(s_ms)
     ms_q = sum(q_ms) / len(q_ms)
     ms_g = sum(g_ms) / len(g_ms)
-    ms_step, ms_q, ms_g = max_over_ranks([ms_step, ms_q, ms_g], dev)
+    srt = sorted(s_ms)
+    spread = [srt[len(srt) // 2], srt[0], srt[-1]]  # median, min, max of the steps
+    ms_step, ms_q, ms_g, *spread = max_over_ranks([ms_step, ms_q, ms_g, *spread], dev)
 
     # ---- end to end through the public composite call, host buffers
     if args.no_e2e or args.path in ("w4a4", "nvfp4"):
@@ -357,7 +359,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
     return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
-                  clocks, t_wall0, t_wall1)
+                  clocks, t_wall0, t_wall1, spread)
 
 
 E2E_CHUNK_ROWS = 4096
@@ -398,7 +400,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
 
 
 def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
-           t_wall0, t_wall1):
+           t_wall0, t_wall1, spread=None):
     # per-rank work: the full batch (weak, replicas) or this rank's row shard
     # (strong); the job's total is world x per-rank (weak) or the whole batch
     M, N, K = X.shape[0], cfg.N, cfg.K
@@ -447,7 +449,9 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
         page_ms = PAGE_MS.get(cfg.name)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": ms_step,
+            "ms_per_step_median_min_max": spread,
+            "higher_is_better": True,
             "scaling": args.scaling,
             "vs_baseline": value / (2.0 * cfg.M * N * K / (page_ms / 1e3) / 1e12) if page_ms else None,
             "dtype": "fp4-e2m1" if args.path == "nvfp4" else "int8", "data": "synthetic",
