@@ -401,7 +401,7 @@ ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t
 
 /*
  * Fault injection for the bounded waits, host side only: with mode 1 the next
- * GEMM launch on this thread's current device runs with its TMA producer
+ * GEMM launch (INT8 or NVFP4) on this thread's current device runs with its TMA producer
  * issuing nothing, so the MMA warp's wait for the first stage can never be
  * satisfied; the kernel must then record CK_ERR_DEVICE_TIMEOUT and return
  * instead of hanging. The flag is consumed by that launch. mode 0 clears it.

@@ -582,6 +582,13 @@ ck_status nvfp4_gemm_checked(const uint8_t *Qa, const uint8_t *Sa, const float *
     p.K = static_cast<int>(K);
     p.err = st->err;
     p.wait_limit_ns = ck::kDefaultWaitLimitNs;
+    p.stall_producer = 0;
+    if (t_stall_next) {
+        p.stall_producer = 1;
+        if (t_stall_limit_ns > 0) p.wait_limit_ns = static_cast<uint64_t>(t_stall_limit_ns);
+        t_stall_next = 0;
+        t_stall_limit_ns = 0;
+    }
     return ck::launch_gemm_nvfp4(tmA, tmB, tmSFA, tmSFB, p, st->num_sms, true, stream) ==
                    cudaSuccess
                ? CK_OK

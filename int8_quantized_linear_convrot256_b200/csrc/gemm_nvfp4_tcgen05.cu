@@ -189,7 +189,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_parity = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = blockIdx.x; ok && !p.stall_producer && tile < num_tiles;
+                 tile += gridDim.x) {
                 int mt, nt;
                 tile_of(tile, num_m, num_n, mt, nt);
                 const uint8_t *sfa = p.sfa + int64_t(mt) * sf_tiles_per_row_block * kSfTileBytes;
@@ -496,7 +497,8 @@ gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_parity = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+            for (int tile = pair; ok && !p.stall_producer && tile < num_tiles;
+                 tile += num_pairs) {
                 int mt, nt;
                 tile_of_pair(tile, num_m, num_n, mt, nt);
                 const int a_row = mt * kPairBMn + int(rank) * kPairRowsN;

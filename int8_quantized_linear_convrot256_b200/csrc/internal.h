@@ -99,6 +99,7 @@ struct Nvfp4GemmParams {
     int M, N, K;
     unsigned *err;
     uint64_t wait_limit_ns;
+    int stall_producer;     // test hook: the loads are never issued
 };
 
 constexpr int kNvfp4BM = 128;      // rows of A per tile (TMA box rows)
