@@ -473,8 +473,8 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                              gemm_tops / (9000.0 if args.path == "nvfp4" else 4500.0),
                          "frac_of_measured_sustained": gemm_tops / sustained_peak,
                          "ms_per_launch": ms_g},
-            "quantizer": {"kernel": ("nvfp4_amax_kernel + nvfp4_quant_kernel (ConvRot256 + "
-                                     "NVFP4, two passes over X)" if args.path == "nvfp4" else
+            "quantizer": {"kernel": ("nvfp4_bulk_kernel<1> + <2> (ConvRot256 + NVFP4, two "
+                                     "staged passes over X)" if args.path == "nvfp4" else
                                      ("quant_rows_bulk_kernel" if K <= 28672 else
                                       "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)"),
                           "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",

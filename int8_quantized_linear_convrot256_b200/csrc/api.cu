@@ -509,6 +509,7 @@ ck_status ck_quantize_rotate_nvfp4(const ck_bf16 *X, int64_t M, int64_t K, int64
     s = device_state(&st);
     if (s != CK_OK) return s;
     return ck::launch_quant_nvfp4_bf16(X, M, K, ldx, Q, S, ck_nvfp4_scale_bytes(M, K), s_t,
+                                       st->err, st->num_sms,
                                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? CK_OK
                : CK_ERR_CUDA;
@@ -650,8 +651,8 @@ ck_status ck_convrot_nvfp4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *
     uint8_t *Sa = base + round256(size_t(M) * size_t(K / 2));
     float *s_ta = reinterpret_cast<float *>(Sa + round256(ck_nvfp4_scale_bytes(M, K)));
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    if (ck::launch_quant_nvfp4_bf16(X, M, K, ldx, Qa, Sa, ck_nvfp4_scale_bytes(M, K), s_ta, cs) !=
-        cudaSuccess)
+    if (ck::launch_quant_nvfp4_bf16(X, M, K, ldx, Qa, Sa, ck_nvfp4_scale_bytes(M, K), s_ta,
+                                    st->err, st->num_sms, cs) != cudaSuccess)
         return CK_ERR_CUDA;
     return nvfp4_gemm_checked(Qa, Sa, s_ta, Qw, Sw, s_tw, bias, Y, M, N, K, st, cs);
 }

@@ -27,7 +27,7 @@ cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int
 // bytes, per-tensor scale in *s_t) and decoding to fp32.
 cudaError_t launch_quant_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     uint8_t *Q, uint8_t *S, size_t s_bytes, float *s_t,
-                                    cudaStream_t stream);
+                                    unsigned *err, int num_sms, cudaStream_t stream);
 cudaError_t launch_quant_nvfp4_f32(const float *W, int64_t N, int64_t K, uint8_t *Q, uint8_t *S,
                                    size_t s_bytes, float *s_t, cudaStream_t stream);
 cudaError_t launch_dequant_nvfp4(const uint8_t *Q, const uint8_t *S, const float *s_t,

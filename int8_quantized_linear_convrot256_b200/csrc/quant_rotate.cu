@@ -982,6 +982,131 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
     }
 }
 
+// Staged, persistent variant of the two NVFP4 passes for bf16 rows (as
+// quant_rows_bulk_kernel: row groups arrive by cp.async.bulk into two
+// buffers, the next group landing while the current one is computed). No
+// row-wide reduction is needed, so the CTA barrier of a group comes right
+// after its values are in registers and the buffer is refilled at once.
+// kPass 1: absmax of the rotated tensor into *amax_bits; kPass 2: codes and
+// block scales (as nvfp4_quant_kernel).
+template <int kPass>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
+                  unsigned *amax_bits, uint8_t *__restrict__ Q, uint8_t *__restrict__ S,
+                  unsigned *err, uint64_t limit_ns) {
+    extern __shared__ __align__(128) uint8_t stage_raw[];
+    __shared__ unsigned s_max;
+    __shared__ __align__(8) uint64_t full[2];
+    const int tid = threadIdx.x;
+    const int t = tid & 3;
+    const int quad = tid >> 2;
+    const int nb = K >> 8;
+    const int R = rows_per_cta;
+    const int row_local = quad / nb;
+    const int blk = quad - row_local * nb;
+    const int col0 = blk * kBlock + 8 * t;
+    const int64_t ngroups = (M + R - 1) / R;
+    const uint32_t row_bytes = uint32_t(K) * 2u;
+    const uint32_t buf0 = smem_u32(stage_raw);
+    const uint32_t buf_bytes = uint32_t(R) * row_bytes;
+    const int C = K >> 4;
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        fence_mbar_init();
+        s_max = 0u;
+    }
+    __syncthreads();
+
+    auto issue = [&](int64_t g, int b) {
+        const int64_t r0 = g * R;
+        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
+        const uint32_t bar = smem_u32(&full[b]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
+        for (int r = 0; r < n; ++r) {
+            const uint16_t *src = X + (r0 + r) * ldx;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(buf0 + uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes),
+                "l"(reinterpret_cast<uint64_t>(src)), "r"(row_bytes), "r"(bar)
+                : "memory");
+        }
+    };
+
+    const int64_t g0 = blockIdx.x;
+    const int64_t step = gridDim.x;
+    if (tid == 0) {
+        if (g0 < ngroups) issue(g0, 0);
+        if (g0 + step < ngroups) issue(g0 + step, 1);
+    }
+    float s_t = 0.0f;
+    if (kPass == 2) s_t = __fdiv_rn(__fmul_rn(__uint_as_float(*amax_bits), 0.0625f), 2688.0f);
+    float local_max = 0.0f;
+    for (int i = 0; g0 + i * step < ngroups; ++i) {
+        const int64_t g = g0 + i * step;
+        const int b = i & 1;
+        const bool ok = mbar_wait_bounded(smem_u32(&full[b]), uint32_t(i >> 1) & 1u, limit_ns,
+                                          nullptr);
+        const int64_t row = g * R + row_local;
+        const bool active = ok && row_local < R && row < M;
+        float2 P[kPairs];
+        const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
+                            uint32_t(col0) * 2u;
+        if (active)
+            load_block_smem<true>(sa, 0, P);
+        else
+            zero_block(P);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicMax(err, kDevErrTimeout);
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000ull) {
+            }
+            break;
+        }
+        if (tid == 0 && g + 2 * step < ngroups) issue(g + 2 * step, b);
+        butterflies<true>(P, t);
+        if (kPass == 1) {
+            local_max = fmaxf(local_max, block_absmax(P));
+            continue;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            float y[8];
+            float m8 = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 z = P[4 * c + k];
+                y[2 * k] = __fmul_rn(z.x, 0.0625f);
+                y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
+                m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
+            }
+            const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
+            uint32_t bsc = 0;
+            if (s_t > 0.0f) bsc = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
+            const float d = __fmul_rn(e4m3_to_f32(bsc), s_t);
+            uint32_t packed = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float v = d != 0.0f ? __fdiv_rn(y[j], d) : 0.0f;
+                packed |= e2m1_rne_sat(v) << (4 * j);
+            }
+            if (active) {
+                const int e0 = col0 + 32 * c;
+                *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
+                if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(bsc);
+            }
+        }
+    }
+    if (kPass == 1) {
+        // the quads' maxima are equal within a quad; one atomic per quad
+        if (t == 0 && local_max > 0.0f) atomicMax(&s_max, __float_as_uint(local_max));
+        __syncthreads();
+        if (tid == 0 && s_max != 0u) atomicMax(amax_bits, s_max);
+    }
+}
+
 // Turns the absmax bits of z into the per-tensor scale, in place.
 __global__ void nvfp4_scale_kernel(float *s_t) {
     const float amax = __fmul_rn(__uint_as_float(*reinterpret_cast<unsigned *>(s_t)), 0.0625f);
@@ -1072,10 +1197,63 @@ cudaError_t launch_nvfp4_impl(const TIn *X, int64_t M, int64_t K, int64_t ldx, u
     return cudaGetLastError();
 }
 
+std::map<std::tuple<int, int, int, size_t>, int> g_nvfp4_bulk_occupancy;
+
+template <int kPass>
+cudaError_t nvfp4_bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
+    std::lock_guard<std::mutex> lock(g_occ_mutex);
+    const auto key = std::make_tuple(dev, kPass, threads, smem);
+    auto it = g_nvfp4_bulk_occupancy.find(key);
+    if (it != g_nvfp4_bulk_occupancy.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(nvfp4_bulk_kernel<kPass>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(kBulkSmemBudget));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_bulk_kernel<kPass>, threads,
+                                                      smem);
+    if (e != cudaSuccess) return e;
+    g_nvfp4_bulk_occupancy[key] = per_sm;
+    *out = per_sm;
+    return cudaSuccess;
+}
+
 cudaError_t launch_quant_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     uint8_t *Q, uint8_t *S, size_t s_bytes, float *s_t,
-                                    cudaStream_t stream) {
-    return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
+                                    unsigned *err, int num_sms, cudaStream_t stream) {
+    if (M <= 0) return cudaSuccess;
+    const int nb = static_cast<int>(K / kBlock);
+    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2)),
+                                  kMaxRowsPerCta);
+    if (max_rows < 1 || 4 * nb > kMaxThreads)
+        return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
+    int threads = 0;
+    const int rows = pick_rows_per_cta(nb, 4, max_rows, kMaxThreads, 256, &threads);
+    const size_t smem = 2 * size_t(rows) * size_t(K) * 2;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int per_sm1 = 0, per_sm2 = 0;
+    if ((e = nvfp4_bulk_blocks_per_sm<1>(dev, threads, smem, &per_sm1)) != cudaSuccess) return e;
+    if ((e = nvfp4_bulk_blocks_per_sm<2>(dev, threads, smem, &per_sm2)) != cudaSuccess) return e;
+    if (per_sm1 < 1 || per_sm2 < 1)
+        return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
+    const int64_t groups = (M + rows - 1) / rows;
+    const unsigned grid1 = unsigned(std::min<int64_t>(groups, int64_t(per_sm1) * num_sms));
+    const unsigned grid2 = unsigned(std::min<int64_t>(groups, int64_t(per_sm2) * num_sms));
+    e = cudaMemsetAsync(s_t, 0, sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(S, 0, s_bytes, stream);
+    if (e != cudaSuccess) return e;
+    unsigned *amax = reinterpret_cast<unsigned *>(s_t);
+    nvfp4_bulk_kernel<1><<<grid1, threads, smem, stream>>>(X, M, static_cast<int>(K), ldx, rows,
+                                                         amax, Q, S, err, kDefaultWaitLimitNs);
+    nvfp4_bulk_kernel<2><<<grid2, threads, smem, stream>>>(X, M, static_cast<int>(K), ldx, rows,
+                                                         amax, Q, S, err, kDefaultWaitLimitNs);
+    nvfp4_scale_kernel<<<1, 1, 0, stream>>>(s_t);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_nvfp4_f32(const float *W, int64_t N, int64_t K, uint8_t *Q, uint8_t *S,
