@@ -32,7 +32,8 @@ def _np(t):
     return t.cpu().numpy()
 
 
-@pytest.mark.parametrize("M,K", [(1, 256), (37, 768), (130, 5376), (5, 28672), (300, 512)])
+@pytest.mark.parametrize("M,K", [(1, 256), (37, 768), (130, 5376), (5, 28672), (300, 512),
+                                 (2, 32768)])
 def test_quantize_rotate_nvfp4_bit_exact(ck, M, K):
     cfg = workloads.custom(M, K, 8, seed=M * 7 + K)
     X, _, _ = workloads.make_inputs(cfg)
@@ -52,6 +53,18 @@ def test_rotate_quant_weight_nvfp4_bit_exact(ck, N, K):
     assert np.float32(_np(s_t)[0]) == np.float32(sr)
     assert np.array_equal(_np(S)[: Sr.size], Sr)
     assert np.array_equal(_np(Q), Qr)
+
+
+def test_quantize_nvfp4_row_stride(ck):
+    """X with a row stride larger than K (a column slice of a wider tensor)."""
+    cfg = workloads.custom(45, 1024, 8, seed=44)
+    X, _, _ = workloads.make_inputs(cfg)
+    wide = torch.zeros((45, 1024 + 512), dtype=torch.bfloat16)
+    wide[:, :1024] = X
+    Qr, Sr, sr = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X))
+    Q, S, s_t = ck.quantize_rotate_nvfp4(wide.cuda()[:, :1024])
+    assert np.float32(_np(s_t)[0]) == np.float32(sr)
+    assert np.array_equal(_np(S)[: Sr.size], Sr) and np.array_equal(_np(Q), Qr)
 
 
 def test_quantize_nvfp4_zero_and_scaled_tensors(ck):
