@@ -51,21 +51,59 @@ MUTATIONS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_pins_catch_planted_mistake(tmp_path, name):
+# Which pin file is meant to catch each kind of mistake (the others are not
+# run for it, to keep the suite short).
+PIN_FILES = {
+    "act": ["test_oracle_act_pins.py"],
+    "int4": ["test_oracle_w4a4_pins.py"],
+    "nvfp4": ["test_oracle_nvfp4_pins.py"],
+    "core": ["test_oracle_pins.py"],
+}
+
+
+def _pins_for(name: str):
+    if name.startswith(("gelu", "silu", "exp_", "act_")):
+        return PIN_FILES["act"]
+    if name.startswith("int4"):
+        return PIN_FILES["int4"]
+    if name.startswith(("e2m1", "e4m3", "nvfp4")):
+        return PIN_FILES["nvfp4"]
+    return PIN_FILES["core"]
+
+
+def _run_mutant(workdir: str, name: str):
     old, new = MUTATIONS[name]
     src = open(oracle._SRC).read()
-    assert old in src, f"mutation {name} no longer applies"
-    mut = tmp_path / "mut.c"
-    mut.write_text(src.replace(old, new, 1))
-    so = tmp_path / "libmut.so"
-    subprocess.check_call(["gcc", *oracle.CFLAGS, str(mut), "-o", str(so), "-lm"],
+    if old not in src:
+        return name, None, f"mutation {name} no longer applies"
+    mut = os.path.join(workdir, f"{name}.c")
+    with open(mut, "w") as f:
+        f.write(src.replace(old, new, 1))
+    so = os.path.join(workdir, f"lib{name}.so")
+    subprocess.check_call(["gcc", *oracle.CFLAGS, mut, "-o", so, "-lm"],
                           stderr=subprocess.DEVNULL)
-    env = dict(os.environ, CONVROT_ORACLE_LIB=str(so))
+    env = dict(os.environ, CONVROT_ORACLE_LIB=so, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_act_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_w4a4_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_nvfp4_pins.py")],
+                        *[os.path.join(ROOT, "tests", f) for f in _pins_for(name)]],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
+    return name, r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Every mutant built and its pins run once, several at a time (each run
+    is a separate process that loads that mutant's library)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        results = list(ex.map(lambda n: _run_mutant(workdir, n), sorted(MUTATIONS)))
+    return {name: (rc, out) for name, rc, out in results}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(mutant_runs, name):
+    rc, out = mutant_runs[name]
+    assert rc is not None, out
+    assert rc != 0, f"pins did not catch {name}:\n{out}"
