@@ -866,9 +866,9 @@ __global__ void unpack_int4_kernel(const uint4 *__restrict__ in, uint4 *__restri
 //   s_t = amax(tensor) / 2688, b = E4M3_rne_sat((amax(block) / 6) / s_t),
 //   d = float(b) * s_t, q = E2M1_rne_sat(y / d) (+0 when d == 0),
 // two codes per byte with the lower element in the low nibble. The
-// conversions use the hardware's round-to-nearest-even, saturating cvt; each
-// cvt gets the same value twice, so the result does not depend on which half
-// of the packed pair an operand lands in.
+// conversions use the hardware's round-to-nearest-even, saturating cvt (the
+// E4M3 one gets the same value twice, so its result does not depend on which
+// half of the packed pair an operand lands in).
 
 __device__ __forceinline__ uint32_t e4m3_rne_sat(float v) {
     uint16_t r;
@@ -883,11 +883,76 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
     return __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
 }
 
-__device__ __forceinline__ uint32_t e2m1_rne_sat(float v) {
+// Two E2M1 codes in one byte, the first argument's in the low nibble
+// (cvt puts its first source in the upper half of the pair).
+__device__ __forceinline__ uint32_t e2m1x2_rne_sat(float lo, float hi) {
     uint16_t r;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u16.u8 %0, t;\n\t}"
-        : "=h"(r) : "f"(v));
-    return uint32_t(r) & 0xFu;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+        : "=h"(r) : "f"(hi), "f"(lo));
+    return uint32_t(r) & 0xFFu;
+}
+
+// Codes of 8 consecutive values y (one half of a 16-value scale block) with
+// divisor d = float(b) * s_t, packed into 4 bytes (element 2j in the low
+// nibble of byte j). The definition's code is E2M1_rne_sat(fl(y / d)). With
+// r4 = 4 fl(1/d), u = fl(y r4) is within 2^-16 of 4 fl(y / d) (|y / d| < 10:
+// the block scale's rounding in E4M3's subnormal range leaves at most 1.5x
+// headroom over 6), and the E2M1 rounding boundaries 0.25, 0.75, ..., 5 are
+// integers in units of u. So unless some u lies within 2^-14 of an integer,
+// u / 4 (exact) rounds to the same codes as the IEEE quotients; otherwise the
+// 8 values take the IEEE division. That includes y = +-0 (whose sign the code
+// keeps) and a d so small that 4 / d overflows.
+__device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) {
+    if (d == 0.0f) return 0u;
+    const float r4 = __fmul_rn(__frcp_rn(d), 4.0f);
+    const float2 r4v = make_float2(r4, r4);
+    const float2 mg = make_float2(kMagic, kMagic);
+    const float2 nmg = make_float2(-kMagic, -kMagic);
+    const float2 quarter = make_float2(0.25f, 0.25f);
+    float v[8];
+    float dmin = r4 <= 3.0e38f ? 1.0f : 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 u = __fmul2_rn(make_float2(y[2 * k], y[2 * k + 1]), r4v);
+        const float2 r = __fadd2_rn(__fadd2_rn(u, mg), nmg);
+        const float2 du = __ffma2_rn(r, make_float2(-1.0f, -1.0f), u);
+        float m;
+        asm("min.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(dmin), "f"(fabsf(du.x)), "f"(fabsf(du.y)));
+        dmin = m;
+        const float2 w = __fmul2_rn(u, quarter);
+        v[2 * k] = w.x;
+        v[2 * k + 1] = w.y;
+    }
+    if (dmin < 6.103515625e-05f) {  // 2^-14
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = __fdiv_rn(y[k], d);
+    }
+    uint32_t out = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out |= e2m1x2_rne_sat(v[2 * k], v[2 * k + 1]) << (8 * k);
+    return out;
+}
+
+// Scale block c of a lane's 64 rotated (unnormalised) values: the 8 values
+// y = z / 16 this lane holds, the block scale b = E4M3_rne_sat((amax16 / 6) /
+// s_t) over the 16 values it shares with its neighbour lane (t ^ 1), and the
+// 8 codes, packed. The lanes of a quad call this together (one shuffle).
+__device__ __forceinline__ uint32_t nvfp4_block_codes(const float2 (&P)[kPairs], int c, float s_t,
+                                                      uint32_t *bsc) {
+    float y[8];
+    float m8 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 z = P[4 * c + k];
+        y[2 * k] = __fmul_rn(z.x, 0.0625f);
+        y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
+        m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
+    }
+    const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
+    uint32_t b = 0;
+    if (s_t > 0.0f) b = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
+    *bsc = b;
+    return nvfp4_encode8(y, __fmul_rn(e4m3_to_f32(b), s_t));
 }
 
 // Offset of the scale of row r, scale column c (of C) in the blocked layout:
@@ -955,25 +1020,8 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
     const int C = K >> 4;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        float y[8];
-        float m8 = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 z = P[4 * i + k];
-            y[2 * k] = __fmul_rn(z.x, 0.0625f);
-            y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
-            m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
-        }
-        const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
-        uint32_t b = 0;
-        if (s_t > 0.0f) b = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
-        const float d = __fmul_rn(e4m3_to_f32(b), s_t);
-        uint32_t packed = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float v = d != 0.0f ? __fdiv_rn(y[j], d) : 0.0f;
-            packed |= e2m1_rne_sat(v) << (4 * j);
-        }
+        uint32_t b;
+        const uint32_t packed = nvfp4_block_codes(P, i, s_t, &b);
         if (active) {
             const int e0 = col0 + 32 * i;
             *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
@@ -1067,35 +1115,18 @@ nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
         }
         if (tid == 0 && g + 2 * step < ngroups) issue(g + 2 * step, b);
         butterflies<true>(P, t);
-        if (kPass == 1) {
+        if constexpr (kPass == 1) {
             local_max = fmaxf(local_max, block_absmax(P));
-            continue;
-        }
+        } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float y[8];
-            float m8 = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 z = P[4 * c + k];
-                y[2 * k] = __fmul_rn(z.x, 0.0625f);
-                y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
-                m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
-            }
-            const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
-            uint32_t bsc = 0;
-            if (s_t > 0.0f) bsc = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
-            const float d = __fmul_rn(e4m3_to_f32(bsc), s_t);
-            uint32_t packed = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float v = d != 0.0f ? __fdiv_rn(y[j], d) : 0.0f;
-                packed |= e2m1_rne_sat(v) << (4 * j);
-            }
-            if (active) {
-                const int e0 = col0 + 32 * c;
-                *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
-                if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(bsc);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t bsc;
+                const uint32_t packed = nvfp4_block_codes(P, c, s_t, &bsc);
+                if (active) {
+                    const int e0 = col0 + 32 * c;
+                    *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
+                    if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(bsc);
+                }
             }
         }
     }
