@@ -933,26 +933,59 @@ __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) 
     return out;
 }
 
-// Scale block c of a lane's 64 rotated (unnormalised) values: the 8 values
-// y = z / 16 this lane holds, the block scale b = E4M3_rne_sat((amax16 / 6) /
-// s_t) over the 16 values it shares with its neighbour lane (t ^ 1), and the
-// 8 codes, packed. The lanes of a quad call this together (one shuffle).
-__device__ __forceinline__ uint32_t nvfp4_block_codes(const float2 (&P)[kPairs], int c, float s_t,
-                                                      uint32_t *bsc) {
-    float y[8];
-    float m8 = 0.0f;
+// fl(1 / fl(6 s_t)) for nvfp4_block_scale, or 0 when s_t is 0 or the
+// reciprocal is not finite (every block then takes the exact divisions).
+__device__ __forceinline__ float nvfp4_scale_rcp(float s_t) {
+    if (!(s_t > 0.0f)) return 0.0f;
+    const float c = __frcp_rn(__fmul_rn(6.0f, s_t));
+    return c <= 3.0e38f ? c : 0.0f;
+}
+
+// Block scale b = E4M3_rne_sat(fl(fl(m / 6) / s_t)) of a block with absmax m.
+// q = fl(m c6) is within 5 units in the last place of the two divisions'
+// result (five roundings of relative size 2^-24 between them). In E4M3's
+// normal range [2^-6, 448] the rounding keeps 3 of fp32's 23 mantissa bits,
+// so q rounds as that result does unless its low 20 mantissa bits lie within
+// 8 units of the half-way pattern 0x80000. Those blocks, values below 2^-6
+// (E4M3's subnormal range, where the rounding position moves) and c6 = 0
+// take the two IEEE divisions.
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float m, float s_t, float c6) {
+    if (!(s_t > 0.0f)) return 0u;
+    const float q = __fmul_rn(m, c6);
+    const uint32_t low = __float_as_uint(q) & 0xFFFFFu;
+    if (q >= 0.0156265625f && low - 0x7FFF8u >= 16u) return e4m3_rne_sat(q);
+    return e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m, 6.0f), s_t));
+}
+
+// Scale blocks of register groups c and c + 1 (c even) of a lane. The lanes
+// t and t ^ 1 each hold 8 of a block's 16 values; the lane with t & 1 = 0
+// computes the scale of group c's block and the other that of group c + 1's,
+// and they swap the results. Returns the two packed code words (8 codes
+// each); *b_own is the scale this lane computed, which it stores.
+__device__ __forceinline__ uint2 nvfp4_codes_pair(const float2 (&P)[kPairs], int c, int t,
+                                                  float s_t, float c6, uint32_t *b_own) {
+    float y[2][8];
+    float m8[2] = {0.0f, 0.0f};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float2 z = P[4 * c + k];
-        y[2 * k] = __fmul_rn(z.x, 0.0625f);
-        y[2 * k + 1] = __fmul_rn(z.y, 0.0625f);
-        m8 = max3(m8, fabsf(y[2 * k]), fabsf(y[2 * k + 1]));
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 z = P[4 * (c + h) + k];
+            y[h][2 * k] = __fmul_rn(z.x, 0.0625f);
+            y[h][2 * k + 1] = __fmul_rn(z.y, 0.0625f);
+            m8[h] = max3(m8[h], fabsf(y[h][2 * k]), fabsf(y[h][2 * k + 1]));
+        }
     }
-    const float m16 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, 1));
-    uint32_t b = 0;
-    if (s_t > 0.0f) b = e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m16, 6.0f), s_t));
-    *bsc = b;
-    return nvfp4_encode8(y, __fmul_rn(e4m3_to_f32(b), s_t));
+    const float m0 = fmaxf(m8[0], __shfl_xor_sync(0xFFFFFFFFu, m8[0], 1));
+    const float m1 = fmaxf(m8[1], __shfl_xor_sync(0xFFFFFFFFu, m8[1], 1));
+    const bool odd = (t & 1) != 0;
+    const uint32_t mine = nvfp4_block_scale(odd ? m1 : m0, s_t, c6);
+    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+    const uint32_t b0 = odd ? other : mine;
+    const uint32_t b1 = odd ? mine : other;
+    *b_own = mine;
+    return make_uint2(nvfp4_encode8(y[0], __fmul_rn(e4m3_to_f32(b0), s_t)),
+                      nvfp4_encode8(y[1], __fmul_rn(e4m3_to_f32(b1), s_t)));
 }
 
 // Offset of the scale of row r, scale column c (of C) in the blocked layout:
@@ -1017,15 +1050,18 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
     butterflies(P, t);
     const float amax = __fmul_rn(__uint_as_float(*amax_bits), 0.0625f);
     const float s_t = __fdiv_rn(amax, 2688.0f);
+    const float c6 = nvfp4_scale_rcp(s_t);
     const int C = K >> 4;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 8; i += 2) {
         uint32_t b;
-        const uint32_t packed = nvfp4_block_codes(P, i, s_t, &b);
+        const uint2 packed = nvfp4_codes_pair(P, i, t, s_t, c6, &b);
         if (active) {
             const int e0 = col0 + 32 * i;
-            *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
-            if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(b);
+            uint8_t *qr = Q + row * int64_t(K / 2);
+            *reinterpret_cast<uint32_t *>(qr + e0 / 2) = packed.x;
+            *reinterpret_cast<uint32_t *>(qr + (e0 + 32) / 2) = packed.y;
+            S[nvfp4_sf_offset(row, (e0 + 32 * (t & 1)) >> 4, C)] = uint8_t(b);
         }
     }
 }
@@ -1091,6 +1127,7 @@ nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
     }
     float s_t = 0.0f;
     if (kPass == 2) s_t = __fdiv_rn(__fmul_rn(__uint_as_float(*amax_bits), 0.0625f), 2688.0f);
+    const float c6 = nvfp4_scale_rcp(s_t);
     float local_max = 0.0f;
     for (int i = 0; g0 + i * step < ngroups; ++i) {
         const int64_t g = g0 + i * step;
@@ -1119,13 +1156,15 @@ nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
             local_max = fmaxf(local_max, block_absmax(P));
         } else {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 8; c += 2) {
                 uint32_t bsc;
-                const uint32_t packed = nvfp4_block_codes(P, c, s_t, &bsc);
+                const uint2 packed = nvfp4_codes_pair(P, c, t, s_t, c6, &bsc);
                 if (active) {
                     const int e0 = col0 + 32 * c;
-                    *reinterpret_cast<uint32_t *>(Q + row * int64_t(K / 2) + e0 / 2) = packed;
-                    if ((t & 1) == 0) S[nvfp4_sf_offset(row, e0 >> 4, C)] = uint8_t(bsc);
+                    uint8_t *qr = Q + row * int64_t(K / 2);
+                    *reinterpret_cast<uint32_t *>(qr + e0 / 2) = packed.x;
+                    *reinterpret_cast<uint32_t *>(qr + (e0 + 32) / 2) = packed.y;
+                    S[nvfp4_sf_offset(row, (e0 + 32 * (t & 1)) >> 4, C)] = uint8_t(bsc);
                 }
             }
         }

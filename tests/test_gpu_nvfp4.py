@@ -78,6 +78,37 @@ def test_quantize_nvfp4_zero_and_scaled_tensors(ck):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and float(b[2][0]) == 4 * float(a[2][0])
 
 
+def test_quantize_nvfp4_rounding_ties(ck):
+    """Inputs whose rotated values hit the E4M3 and E2M1 rounding ties exactly.
+
+    Row 0 holds A = 258048 in column 0: every rotated value is A / 16, so the
+    tensor's absmax is 16128 and s_t = 16128 / 2688 = 6. A row with one value
+    a has the block absmax m = a / 16 and the block-scale quotient m / 36:
+    a = 612 gives 1.0625, half-way between the E4M3 values 1 and 1.125 (ties
+    to 1.0, byte 0x38); a = 8 and a = 1 fall in E4M3's subnormal range. A row
+    a e_0 + b e_1 rotates to (a + b) / 16 and (a - b) / 16 in alternate
+    places; with a + b = 576 the block scale is exactly 1 (d = 6), and
+    a - b = 24, 72, 240, 480 puts (a - b) / 96 on the E2M1 ties 0.25, 0.75,
+    2.5 and 5. Every tie must round to even, as the oracle does."""
+    rows = [[(0, 258048.0)], [(0, 612.0)], [(0, 8.0)], [(0, 1.0)],
+            [(0, 300.0), (1, 276.0)], [(0, 324.0), (1, 252.0)], [(0, 408.0), (1, 168.0)],
+            [(0, 528.0), (1, 48.0)], [(0, -612.0)], [(3, 612.0), (200, -300.0)]]
+    X = torch.zeros((len(rows), 256), dtype=torch.float32)
+    for r, entries in enumerate(rows):
+        for c, v in entries:
+            X[r, c] = v
+    X = X.to(torch.bfloat16)
+    assert torch.equal(X.float(), X.to(torch.float32))
+    Qr, Sr, sr = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X))
+    assert np.float32(sr) == np.float32(6.0)
+    # the a = 612 row: every block's scale ties to E4M3 1.0
+    assert all(Sr[oracle.nvfp4_sf_offset(1, c, 16)] == 0x38 for c in range(16))
+    Q, S, s_t = ck.quantize_rotate_nvfp4(X.cuda())
+    assert np.float32(_np(s_t)[0]) == np.float32(sr)
+    assert np.array_equal(_np(S)[: Sr.size], Sr)
+    assert np.array_equal(_np(Q), Qr)
+
+
 @pytest.mark.parametrize("hi_first", [False, True])
 def test_dequantize_nvfp4_bit_exact(ck, hi_first):
     cfg = workloads.custom(33, 768, 8, seed=21)

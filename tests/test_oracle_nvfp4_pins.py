@@ -200,3 +200,35 @@ def test_linear_rows_match_fp64_products():
     got = workloads.from_bf16_bits(Y).double().numpy()
     assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
     assert np.all(mag >= np.abs(acc * sa * sw) * (1 - 1e-6))
+
+
+def test_rounding_ties_worked_by_hand():
+    """Inputs whose rotated values land on rounding ties, with the results
+    worked out by hand from the definition (ConvRot256 of a row with one or
+    two non-zeros is known in closed form: H e_0 = all ones, H e_1 alternates
+    signs, then x 1/16).
+
+    Row 0 = 258048 e_0: every rotated value is 16128, so s_t = 16128 / 2688 = 6
+    and the block scale quotient is 448 (E4M3 0x7E). Row a e_0: block absmax
+    a / 16, quotient a / 576: a = 612 gives 1.0625, the tie between E4M3 1 and
+    1.125 (even: 1.0, byte 0x38); a = 8 and a = 1 give 0.01389 and 0.001736,
+    E4M3 subnormals 7 x 2^-9 and 1 x 2^-9. Row a e_0 + b e_1 with a + b = 576:
+    scale 1.0, divisor 6; even places hold 36 / 6 = 6 (code 7), odd places
+    (a - b) / 96, the E2M1 ties 0.25 -> 0, 0.75 -> 1.0 (code 2), 2.5 -> 2
+    (code 4), 5 -> 4 (code 6). Element 2j sits in the low nibble of byte j."""
+    rows = [[(0, 258048.0)], [(0, 612.0)], [(0, 8.0)], [(0, 1.0)],
+            [(0, 300.0), (1, 276.0)], [(0, 324.0), (1, 252.0)], [(0, 408.0), (1, 168.0)],
+            [(0, 528.0), (1, 48.0)]]
+    X = torch.zeros((len(rows), 256), dtype=torch.float32)
+    for r, entries in enumerate(rows):
+        for c, v in entries:
+            X[r, c] = v
+    Q, S, s_t = oracle.quantize_rotate_nvfp4(workloads.bf16_bits(X.to(torch.bfloat16)))
+    assert np.float32(s_t) == np.float32(6.0)
+    want_scale = [0x7E, 0x38, 0x07, 0x01, 0x38, 0x38, 0x38, 0x38]
+    for r, b in enumerate(want_scale):
+        assert [int(S[oracle.nvfp4_sf_offset(r, c, 16)]) for c in range(16)] == [b] * 16
+    for r, byte in zip(range(4, 8), [0x07, 0x27, 0x47, 0x67]):
+        assert np.all(Q[r] == byte), (r, Q[r][:4])
+    # row 0: every value is 16128 and the divisor 448 x 6 = 2688, so every code is +6 (7)
+    assert np.all(Q[0] == 0x77)
