@@ -77,6 +77,7 @@ constexpr int kMaxThreads = 512;
 constexpr int kMaxRowsPerCta = kMaxThreads / 4;
 constexpr int kTwoPassQuads = 128;                   // quads per row in the two-pass variant
 constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
+constexpr float kMagic4 = 3145728.0f;                // 1.5 * 2^21 (spacing 1/4 around it)
 constexpr float kNearHalf = 0.4999847412109375f;     // 0.5 - 2^-16
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
 constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
@@ -876,60 +877,62 @@ __device__ __forceinline__ uint32_t e4m3_rne_sat(float v) {
     return uint32_t(r) & 0xFFu;
 }
 
+// An E4M3 byte's value (sign clear, not NaN): its exponent and mantissa bits
+// shifted into fp32's places (b << 20) read as 2^(e - 127) (1 + m / 8), or
+// as the subnormal m 2^-129 when e = 0; the exact product with 2^120 gives
+// 2^(e - 7) (1 + m / 8) and m 2^-9, E4M3's normal and subnormal values.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-    const uint16_t pair = uint16_t(b | (b << 8));
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-    return __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
-}
-
-// Two E2M1 codes in one byte, the first argument's in the low nibble
-// (cvt puts its first source in the upper half of the pair).
-__device__ __forceinline__ uint32_t e2m1x2_rne_sat(float lo, float hi) {
-    uint16_t r;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
-        : "=h"(r) : "f"(hi), "f"(lo));
-    return uint32_t(r) & 0xFFu;
+    return __fmul_rn(__uint_as_float(b << 20), 1.329227995784916e36f);  // 2^120
 }
 
 // Codes of 8 consecutive values y (one half of a 16-value scale block) with
 // divisor d = float(b) * s_t, packed into 4 bytes (element 2j in the low
-// nibble of byte j). The definition's code is E2M1_rne_sat(fl(y / d)). With
-// r4 = 4 fl(1/d), u = fl(y r4) is within 2^-16 of 4 fl(y / d) (|y / d| < 10:
-// the block scale's rounding in E4M3's subnormal range leaves at most 1.5x
-// headroom over 6), and the E2M1 rounding boundaries 0.25, 0.75, ..., 5 are
-// integers in units of u. So unless some u lies within 2^-14 of an integer,
-// u / 4 (exact) rounds to the same codes as the IEEE quotients; otherwise the
-// 8 values take the IEEE division. That includes y = +-0 (whose sign the code
-// keeps) and a d so small that 4 / d overflows.
+// nibble of byte j). The definition's code is E2M1_rne_sat(fl(y / d)).
+// r = rcp.approx(d) is within a few units in the last place of 1 / d (taken
+// as at most 2^-21 relative here; the instruction's documented bound is
+// tighter), so u = fl(y r) lies within 2^-17.3 of fl(y / d) for |y / d| < 10
+// (the block scale's rounding in E4M3's subnormal range leaves at most 1.5x
+// headroom over 6). The E2M1 rounding boundaries 0.25, 0.75, ..., 5 are
+// multiples of 1/4, so unless some u lies within 2^-16 of a multiple of 1/4,
+// u converts to the same codes as the IEEE quotients; otherwise the 8 values
+// take the IEEE division. That includes y = +-0 (whose sign the code keeps)
+// and a d in fp32's subnormal range (flushed by the approximation: r = inf).
+// cvt.e2m1x2 puts its first source in the upper nibble; mov packs the four
+// bytes low byte first.
 __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) {
     if (d == 0.0f) return 0u;
-    const float r4 = __fmul_rn(__frcp_rn(d), 4.0f);
-    const float2 r4v = make_float2(r4, r4);
-    const float2 mg = make_float2(kMagic, kMagic);
-    const float2 nmg = make_float2(-kMagic, -kMagic);
-    const float2 quarter = make_float2(0.25f, 0.25f);
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    const float2 rv = make_float2(r, r);
+    const float2 mg = make_float2(kMagic4, kMagic4);
+    const float2 nmg = make_float2(-kMagic4, -kMagic4);
     float v[8];
-    float dmin = r4 <= 3.0e38f ? 1.0f : 0.0f;
+    float dmin = r <= 3.0e38f ? 1.0f : 0.0f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float2 u = __fmul2_rn(make_float2(y[2 * k], y[2 * k + 1]), r4v);
-        const float2 r = __fadd2_rn(__fadd2_rn(u, mg), nmg);
-        const float2 du = __ffma2_rn(r, make_float2(-1.0f, -1.0f), u);
+        const float2 u = __fmul2_rn(make_float2(y[2 * k], y[2 * k + 1]), rv);
+        const float2 q = __fadd2_rn(__fadd2_rn(u, mg), nmg);  // nearest multiple of 1/4
+        const float2 du = __ffma2_rn(q, make_float2(-1.0f, -1.0f), u);
         float m;
         asm("min.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(dmin), "f"(fabsf(du.x)), "f"(fabsf(du.y)));
         dmin = m;
-        const float2 w = __fmul2_rn(u, quarter);
-        v[2 * k] = w.x;
-        v[2 * k + 1] = w.y;
+        v[2 * k] = u.x;
+        v[2 * k + 1] = u.y;
     }
-    if (dmin < 6.103515625e-05f) {  // 2^-14
+    if (dmin < 1.52587890625e-05f) {  // 2^-16
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = __fdiv_rn(y[k], d);
     }
-    uint32_t out = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) out |= e2m1x2_rne_sat(v[2 * k], v[2 * k + 1]) << (8 * k);
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
     return out;
 }
 
@@ -970,10 +973,10 @@ __device__ __forceinline__ uint2 nvfp4_codes_pair(const float2 (&P)[kPairs], int
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 z = P[4 * (c + h) + k];
-            y[h][2 * k] = __fmul_rn(z.x, 0.0625f);
-            y[h][2 * k + 1] = __fmul_rn(z.y, 0.0625f);
-            m8[h] = max3(m8[h], fabsf(y[h][2 * k]), fabsf(y[h][2 * k + 1]));
+            const float2 z = __fmul2_rn(P[4 * (c + h) + k], make_float2(0.0625f, 0.0625f));
+            y[h][2 * k] = z.x;
+            y[h][2 * k + 1] = z.y;
+            m8[h] = max3(m8[h], fabsf(z.x), fabsf(z.y));
         }
     }
     const float m0 = fmaxf(m8[0], __shfl_xor_sync(0xFFFFFFFFu, m8[0], 1));

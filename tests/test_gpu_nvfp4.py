@@ -119,6 +119,29 @@ def test_dequantize_nvfp4_bit_exact(ck, hi_first):
     assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
 
 
+def test_dequantize_nvfp4_every_scale_byte(ck):
+    """Every non-NaN positive E4M3 byte (subnormals included) as a block scale
+    with E2M1 code 2 (= 1.0) and s_t = 1: the decoded values are the scales
+    themselves, compared with the oracle and with PyTorch's float8_e4m3fn."""
+    rows, K = 128, 2048
+    C = K // 16
+    S = np.zeros(ck.nvfp4_scale_bytes(rows, K), np.uint8)
+    byte_of = np.zeros((rows, C), np.uint8)
+    for r in range(rows):
+        for c in range(C):
+            b = (r * C + c) % 127
+            byte_of[r, c] = b
+            S[oracle.nvfp4_sf_offset(r, c, C)] = b
+    Q = np.full((rows, K // 2), 0x22, np.uint8)
+    s_t = np.ones(1, np.float32)
+    got = _np(ck.dequantize_nvfp4(torch.from_numpy(Q).cuda(), torch.from_numpy(S).cuda(),
+                                  torch.from_numpy(s_t).cuda()))
+    want = oracle.dequantize_nvfp4(Q, S, 1.0)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    e4m3 = torch.from_numpy(byte_of).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(got.reshape(rows, C, 16), np.repeat(e4m3[:, :, None], 16, axis=2))
+
+
 def _bf16_val(bits):
     return workloads.from_bf16_bits(bits).double().numpy()
 
