@@ -167,9 +167,15 @@ def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float, act: str = "n
         return time.perf_counter() - t
 
     probe = 8
+    target = 1.25 * seconds
+    run(probe)  # first touch of the weights, thread start-up
     dt = run(probe)
-    rows = int(max(probe, min(cfg.M, probe * seconds / max(dt, 1e-6))))
+    rows = int(max(probe, min(cfg.M, probe * target / max(dt, 1e-6))))
     dt = run(rows)
+    if dt < seconds and rows < cfg.M:
+        # a probe of 8 rows leaves most host threads idle: size again from this run
+        rows = int(max(probe, min(cfg.M, rows * target / max(dt, 1e-6))))
+        dt = run(rows)
     tops = 2.0 * rows * cfg.N * cfg.K / dt / 1e12
     return tops, rows, dt, oracle.num_threads()
 
@@ -214,9 +220,10 @@ def run_reference(args, cfg, rank, world):
         what, dtype = "quantize_and_rotate_rowwise of those rows + their outputs", "int8"
     total_budget = 150.0
     per_step = total_budget / max(1, args.steps + args.warmup)
+    run(4)  # first touch of the weights, thread start-up
     t_probe = time.perf_counter()
-    run(4)
-    t_row = (time.perf_counter() - t_probe) / 4
+    run(16)
+    t_row = (time.perf_counter() - t_probe) / 16
     rows = int(max(1, min(cfg.M, per_step / max(t_row, 1e-9))))
     times = []
     for i in range(args.warmup + args.steps):
