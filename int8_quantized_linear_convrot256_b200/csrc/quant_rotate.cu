@@ -78,6 +78,7 @@ constexpr int kMaxRowsPerCta = kMaxThreads / 4;
 constexpr int kTwoPassQuads = 128;                   // quads per row in the two-pass variant
 constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
 constexpr float kMagic4 = 3145728.0f;                // 1.5 * 2^21 (spacing 1/4 around it)
+constexpr float kNearQuarter = 1.52587890625e-05f;   // 2^-16
 constexpr float kNearHalf = 0.4999847412109375f;     // 0.5 - 2^-16
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
 constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
@@ -894,9 +895,10 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
 // (the block scale's rounding in E4M3's subnormal range leaves at most 1.5x
 // headroom over 6). The E2M1 rounding boundaries 0.25, 0.75, ..., 5 are
 // multiples of 1/4, so unless some u lies within 2^-16 of a multiple of 1/4,
-// u converts to the same codes as the IEEE quotients; otherwise the 8 values
-// take the IEEE division. That includes y = +-0 (whose sign the code keeps)
-// and a d in fp32's subnormal range (flushed by the approximation: r = inf).
+// u converts to the same codes as the IEEE quotients; the values that are
+// that close take the IEEE division. That includes y = +-0 (whose sign the
+// code keeps) and, for all 8, a d in fp32's subnormal range (flushed by the
+// approximation: r = inf).
 // cvt.e2m1x2 puts its first source in the upper nibble; mov packs the four
 // bytes low byte first.
 __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) {
@@ -919,9 +921,15 @@ __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) 
         v[2 * k] = u.x;
         v[2 * k + 1] = u.y;
     }
-    if (dmin < 1.52587890625e-05f) {  // 2^-16
+    if (dmin < kNearQuarter) {
+        // only the values near a multiple of 1/4 take the division (all of
+        // them when r is not finite: |du| is then NaN)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = __fdiv_rn(y[k], d);
+        for (int k = 0; k < 8; ++k) {
+            const float u = __fmul_rn(y[k], r);
+            const float q = __fadd_rn(__fadd_rn(u, kMagic4), -kMagic4);
+            if (!(fabsf(__fadd_rn(u, -q)) >= kNearQuarter)) v[k] = __fdiv_rn(y[k], d);
+        }
     }
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
