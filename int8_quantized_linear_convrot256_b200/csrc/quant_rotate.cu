@@ -542,9 +542,22 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const 
         store_group<kPack4>(u, i, dst);
     }
     if (redo) {
+        // In a flagged group only the values near a half-integer take the
+        // exact path; the others keep their fast codes (recomputed).
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (redo & (1u << i)) store_group_exact<kPack4>(P, i, rq, dst);
+        for (int i = 0; i < 8; ++i) {
+            if (redo & (1u << i)) {
+                uint32_t u[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float z = (k & 1) ? P[4 * i + (k >> 1)].y : P[4 * i + (k >> 1)].x;
+                    const float m = __fmaf_rn(z, rq.rc, kMagic);
+                    const float d = __fmaf_rn(z, -rq.rc, __fadd_rn(m, -kMagic));
+                    u[k] = fabsf(d) >= kNearHalf ? code_exact(z, rq) : __float_as_uint(m);
+                }
+                store_group<kPack4>(u, i, dst);
+            }
+        }
     }
 }
 
