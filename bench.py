@@ -369,7 +369,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                   clocks, t_wall0, t_wall1, spread)
 
 
-E2E_CHUNK_ROWS = 4096
+E2E_CHUNK_ROWS = 2048
 
 
 def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):

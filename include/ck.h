@@ -220,8 +220,10 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
  *           memory gives the same results without the overlap)
  *   Qw, s_w, bias: device memory, as for ck_int8_linear.
  *   Y_host  [M, N] bf16, row stride N, host memory.   (output)
- *   chunk_rows  rows per chunk (> 0); 4096 keeps a chunk's GEMM several
- *           waves long on a B200 for the N of the pages' workloads.
+ *   chunk_rows  rows per chunk (> 0). 2048 keeps a chunk's GEMM a few waves
+ *           long on a B200 for the N of the pages' workloads while the
+ *           first copy in and the last copy out, which nothing overlaps,
+ *           stay short.
  *   workspace   >= ck_int8_linear_host_workspace_bytes(chunk_rows, N, K)
  *           bytes of device memory, 256-B aligned (two input and two output
  *           chunk buffers, the chunk's codes and row scales).

@@ -245,7 +245,7 @@ def host_workspace_bytes(chunk_rows: int, N: int, K: int) -> int:
 
 def int8_linear_host(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
                      bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                     chunk_rows: int = 4096, workspace: torch.Tensor | None = None, stream=None,
+                     chunk_rows: int = 2048, workspace: torch.Tensor | None = None, stream=None,
                      input_act: str = "none") -> torch.Tensor:
     """int8_linear for X and Y in host memory (ck_int8_linear_host): the rows
     go through the GPU in chunks with the copies in and out overlapped with the
