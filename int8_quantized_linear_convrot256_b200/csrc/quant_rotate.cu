@@ -266,16 +266,17 @@ __device__ __forceinline__ void act_in_smem(uint32_t saddr) {
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
                      : "r"(saddr + 64u * i));
-        bool exact = false;
-        uint32_t ax = act_bf16x2<kAct>(x, exact);
-        uint32_t ay = act_bf16x2<kAct>(y, exact);
-        uint32_t az = act_bf16x2<kAct>(z, exact);
-        uint32_t aw = act_bf16x2<kAct>(w, exact);
-        if (exact) {
-            ax = act_bf16x2_exact<kAct>(x);
-            ay = act_bf16x2_exact<kAct>(y);
-            az = act_bf16x2_exact<kAct>(z);
-            aw = act_bf16x2_exact<kAct>(w);
+        // one flag per word: only a flagged word is redone
+        bool ex = false, ey = false, ez = false, ew = false;
+        uint32_t ax = act_bf16x2<kAct>(x, ex);
+        uint32_t ay = act_bf16x2<kAct>(y, ey);
+        uint32_t az = act_bf16x2<kAct>(z, ez);
+        uint32_t aw = act_bf16x2<kAct>(w, ew);
+        if (ex | ey | ez | ew) {
+            if (ex) ax = act_bf16x2_exact<kAct>(x);
+            if (ey) ay = act_bf16x2_exact<kAct>(y);
+            if (ez) az = act_bf16x2_exact<kAct>(z);
+            if (ew) aw = act_bf16x2_exact<kAct>(w);
         }
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr + 64u * i), "r"(ax),
                      "r"(ay), "r"(az), "r"(aw)
