@@ -133,6 +133,9 @@ def lib():
                                                    _P(ctypes.c_int64), i64, u16p,
                                                    _P(ctypes.c_double)]
             L.oracle_nvfp4_linear_rows.restype = None
+            L.oracle_rmsnorm_rows.argtypes = [u16p, i64, u16p, i64, u16p, ctypes.c_float, i64,
+                                              i64, u16p, u16p]
+            L.oracle_rmsnorm_rows.restype = ctypes.c_int
             L.oracle_num_threads.argtypes = []
             L.oracle_num_threads.restype = ctypes.c_int
             _lib = L
@@ -354,6 +357,44 @@ def int8_linear(X_bits, Qw, s_w, bias_bits=None, act: str = "none"):
     Qx, s_x = quantize_rows_bf16(X_bits, rotate=True, act=act)
     acc = gemm_i32(Qx, Qw)
     return epilogue(acc, s_x, s_w, bias_bits), Qx, s_x, acc
+
+
+# --------------------------------------------------------- input RMSNorm
+
+def rmsnorm_rows(X_bits, residual_bits=None, g_bits=None, eps: float = 1e-6):
+    """The input RMSNorm with an optional residual (the C oracle's reading:
+    h = bf16(x + r), y = bf16((h / sqrt(mean(h^2) + eps)) * g), the sum of
+    squares in the order stated there). Returns (Y bits [M, K], h bits)."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    Y = np.empty((M, K), np.uint16)
+    H = np.empty((M, K), np.uint16)
+    rp = gp = None
+    ldr = K
+    if residual_bits is not None:
+        residual_bits = np.ascontiguousarray(residual_bits, dtype=np.uint16)
+        assert residual_bits.shape == (M, K)
+        rp = _ptr(residual_bits, ctypes.c_uint16)
+    if g_bits is not None:
+        g_bits = np.ascontiguousarray(g_bits, dtype=np.uint16)
+        assert g_bits.shape == (K,)
+        gp = _ptr(g_bits, ctypes.c_uint16)
+    rc = lib().oracle_rmsnorm_rows(_ptr(X_bits, ctypes.c_uint16), K, rp, ldr, gp, float(eps), M,
+                                   K, _ptr(Y, ctypes.c_uint16), _ptr(H, ctypes.c_uint16))
+    if rc != 0:
+        raise ValueError(f"oracle_rmsnorm_rows failed ({rc}); K must be a multiple of 256")
+    return Y, H
+
+
+def int8_linear_norm(X_bits, Qw, s_w, bias_bits=None, residual_bits=None, g_bits=None,
+                     eps: float = 1e-6):
+    """int8_linear after the input RMSNorm (and residual): the normalised bf16
+    rows go through quantize_and_rotate_rowwise, the INT32 GEMM and the
+    epilogue. Returns (Y bits [M, N], h bits, Qx, s_x)."""
+    Yn, H = rmsnorm_rows(X_bits, residual_bits, g_bits, eps)
+    Qx, s_x = quantize_rows_bf16(Yn, rotate=True)
+    acc = gemm_i32(Qx, Qw)
+    return epilogue(acc, s_x, s_w, bias_bits), H, Qx, s_x
 
 
 # ----------------------------------------------------------------- NVFP4

@@ -427,6 +427,72 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* ============================================================ input RMSNorm
+ * comfy-kitchen 0.2.40 (PyPI page), "Huawei Ascend backend": int8_linear
+ * accepts the input RMSNorm and residual arguments and applies them with the
+ * shared device-side helpers, apart from its GEMM. The page prints no
+ * formula. The reading here is the usual add-then-normalise form, each step
+ * an IEEE fp32 operation:
+ *   h   = bf16_rne(float(x) + float(r))      (h = x when there is no residual)
+ *   the residual output is h
+ *   ss  = the sum of h_k^2 over the row, in this order: 32 partial sums p_l
+ *         (l = 0..31), p_l taking, for i = 0, 1, ... and then j = 0..7, the
+ *         element k = 256 i + 8 l + j with one fused multiply-add each
+ *         (p_l = fma(h_k, h_k, p_l), from +0); then five butterfly levels
+ *         p_l = p_l + p_(l xor m) for m = 16, 8, 4, 2, 1 (every l ends with
+ *         the same value, the sum)
+ *   inv = 1 / sqrt(ss / K + eps)
+ *   y   = bf16_rne((h * inv) * float(g_k))   (bf16_rne(h * inv) without g)
+ * The order of the sum is part of the reading: the pages give none, and any
+ * fixed order defines the same function up to fp32 rounding. */
+int oracle_rmsnorm_rows(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t ldr,
+                        const uint16_t *g, float eps, int64_t M, int64_t K, uint16_t *Y,
+                        uint16_t *Rout) {
+    if (K % ROT_N != 0) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        uint16_t *h = (uint16_t *)malloc((size_t)K * sizeof(uint16_t));
+        if (!h) {
+#pragma omp atomic write
+            err = -2;
+        }
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            if (!h) continue;
+            for (int64_t k = 0; k < K; ++k) {
+                float x = oracle_bf16_to_f32(X[m * ldx + k]);
+                h[k] = R ? oracle_f32_to_bf16_rne(x + oracle_bf16_to_f32(R[m * ldr + k]))
+                         : X[m * ldx + k];
+            }
+            if (Rout)
+                for (int64_t k = 0; k < K; ++k) Rout[m * K + k] = h[k];
+            float p[32], q[32];
+            for (int l = 0; l < 32; ++l) {
+                p[l] = 0.0f;
+                for (int64_t i = 0; i < K / ROT_N; ++i)
+                    for (int j = 0; j < 8; ++j) {
+                        float v = oracle_bf16_to_f32(h[ROT_N * i + 8 * l + j]);
+                        p[l] = fmaf(v, v, p[l]);
+                    }
+            }
+            for (int mm = 16; mm >= 1; mm >>= 1) {
+                for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ mm];
+                for (int l = 0; l < 32; ++l) p[l] = q[l];
+            }
+            float ss = p[0];
+            float inv = 1.0f / sqrtf(ss / (float)K + eps);
+            for (int64_t k = 0; k < K; ++k) {
+                float v = oracle_bf16_to_f32(h[k]) * inv;
+                if (g) v = v * oracle_bf16_to_f32(g[k]);
+                Y[m * K + k] = oracle_f32_to_bf16_rne(v);
+            }
+        }
+        free(h);
+    }
+    return err;
+}
+
 /* ===================================================================== NVFP4
  * ConvRot NVFP4 (ComfyUI-HSWQ-Loader-and-Tools, "NVFP4 torch.compile Fix",
  * section 5-1, nvfp4_gemm.py): FP4 E2M1 codes with one scale per 16 values

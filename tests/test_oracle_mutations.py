@@ -48,6 +48,15 @@ MUTATIONS = {
                                 "                        if (y[i] > ab)\n                            ab = y[i];"),
     "act_not_rounded_to_bf16": ("v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));",
                                 "v = oracle_act(act, v);"),
+    "rmsnorm_eps_outside_sqrt": ("float inv = 1.0f / sqrtf(ss / (float)K + eps);",
+                                 "float inv = 1.0f / (sqrtf(ss / (float)K) + eps);"),
+    "rmsnorm_sum_not_mean": ("float inv = 1.0f / sqrtf(ss / (float)K + eps);",
+                             "float inv = 1.0f / sqrtf(ss + eps);"),
+    "rmsnorm_skips_a_partial": ("for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ mm];",
+                                "for (int l = 0; l < 32; ++l) q[l] = mm == 1 ? p[l] + p[l] : p[l] + p[l ^ mm];"),
+    "rmsnorm_weight_dropped": ("if (g) v = v * oracle_bf16_to_f32(g[k]);", "(void)g;"),
+    "rmsnorm_residual_subtracted": ("h[k] = R ? oracle_f32_to_bf16_rne(x + oracle_bf16_to_f32(R[m * ldr + k]))",
+                                    "h[k] = R ? oracle_f32_to_bf16_rne(x - oracle_bf16_to_f32(R[m * ldr + k]))"),
 }
 
 
@@ -58,6 +67,7 @@ PIN_FILES = {
     "int4": ["test_oracle_w4a4_pins.py"],
     "nvfp4": ["test_oracle_nvfp4_pins.py"],
     "core": ["test_oracle_pins.py"],
+    "rmsnorm": ["test_oracle_rmsnorm_pins.py"],
 }
 
 
@@ -68,6 +78,8 @@ def _pins_for(name: str):
         return PIN_FILES["int4"]
     if name.startswith(("e2m1", "e4m3", "nvfp4")):
         return PIN_FILES["nvfp4"]
+    if name.startswith("rmsnorm"):
+        return PIN_FILES["rmsnorm"]
     return PIN_FILES["core"]
 
 
