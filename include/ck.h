@@ -206,6 +206,48 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
                              ck_stream_t stream);
 
 /*
+ * Input RMSNorm with a residual (comfy-kitchen 0.2.40, "Huawei Ascend backend":
+ * int8_linear accepts the input RMSNorm and residual arguments and applies
+ * them with shared helpers apart from its GEMM; the page prints no formula).
+ * Reading, every step an IEEE fp32 operation:
+ *   h   = bf16_rne(x + r), or h = x when residual is NULL;
+ *   residual_out = h (when residual_out is not NULL);
+ *   ss  = sum over the row of h^2 in this order: 32 partial sums p_l, p_l
+ *         taking, for i = 0, 1, ... and then j = 0..7, element 256 i + 8 l + j
+ *         with one fused multiply-add each; then p_l = p_l + p_(l xor m) for
+ *         m = 16, 8, 4, 2, 1;
+ *   inv = 1 / sqrt(ss / K + eps);
+ *   Y   = bf16_rne((h * inv) * g), or bf16_rne(h * inv) when g is NULL.
+ *   X            [M, K] bf16, row stride ldx (>= K, % 8 == 0), 16-B aligned.
+ *   residual     [M, K] bf16, row stride ldr, or NULL.
+ *   residual_out [M, K] bf16, row stride ldo, or NULL (output); it may alias
+ *                X or residual (in-place update of the residual stream).
+ *   g            [K] bf16 weight, or NULL.
+ *   eps          > 0 and finite.
+ *   Y            [M, K] bf16, row stride K (output; must not overlap the inputs).
+ * All pointers 16-B aligned, strides multiples of 8; K % 256 == 0,
+ * K <= CK_MAX_K. One kernel on `stream`, one warp per row.
+ */
+ck_status ck_rmsnorm_residual(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual, int64_t ldr,
+                              ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g, float eps,
+                              int64_t M, int64_t K, ck_bf16 *Y, ck_stream_t stream);
+
+/*
+ * ck_int8_linear on the input RMSNorm of X (with an optional residual), as
+ * the page's int8_linear takes them: ck_rmsnorm_residual into the workspace,
+ * then the ConvRot quantiser and the INT8 GEMM on the normalised rows.
+ * Arguments as in ck_rmsnorm_residual and ck_int8_linear. Workspace:
+ * ck_int8_linear_norm_workspace_bytes(M, K) bytes, 256-B aligned (the
+ * normalised rows, then the codes and row scales).
+ */
+size_t ck_int8_linear_norm_workspace_bytes(int64_t M, int64_t K);
+ck_status ck_int8_linear_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual,
+                              int64_t ldr, ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g,
+                              float eps, const int8_t *Qw, const float *s_w, const ck_bf16 *bias,
+                              ck_bf16 *Y, int64_t M, int64_t N, int64_t K, void *workspace,
+                              size_t workspace_bytes, ck_stream_t stream);
+
+/*
  * ck_int8_linear_act for activations and outputs in HOST memory, with the
  * PCIe copies overlapped with the kernels. The rows are processed in chunks of
  * chunk_rows (the last one ragged): chunk c is copied to the device while

@@ -62,6 +62,11 @@ _SIGS = {
     "ck_quantize_rotate_rowwise_act": (_st, [_vp, _i64, _i64, _i64, _st, _vp, _vp, _vp]),
     "ck_int8_linear_act": (_st, [_vp, _i64, _st, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                  ctypes.c_size_t, _vp]),
+    "ck_rmsnorm_residual": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, ctypes.c_float, _i64,
+                                  _i64, _vp, _vp]),
+    "ck_int8_linear_norm_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "ck_int8_linear_norm": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, ctypes.c_float, _vp, _vp,
+                                  _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "ck_rotate_quant_weight_int4": (_st, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "ck_unpack_int4": (_st, [_vp, _i64, _i64, _vp, _vp]),
     "ck_quantize_rotate_rowwise_int4": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -236,6 +241,83 @@ def int8_linear(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
         _check(lib.ck_int8_linear_act(_ptr(X), ldx, ACTS[input_act], _ptr(Qw), _ptr(s_w),
                                       _ptr(bias), _ptr(out), M, N, K, _ptr(workspace), ws_bytes,
                                       _stream(stream)), "ck_int8_linear_act")
+    return out
+
+
+def _row_stride(t: torch.Tensor, K: int) -> int:
+    return t.stride(0) if t.shape[0] > 1 else max(K, t.stride(0))
+
+
+def _norm_args(X, residual, residual_out, g):
+    _need(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if X.stride(1) != 1:
+        raise ValueError("X must have a unit column stride")
+    for name, t in (("residual", residual), ("residual_out", residual_out)):
+        if t is not None:
+            _need(t, name, torch.bfloat16, 2)
+            if tuple(t.shape) != (M, K) or t.stride(1) != 1:
+                raise ValueError(f"{name} must be [M, K] bf16 with unit column stride")
+    if g is not None:
+        _need(g, "g", torch.bfloat16, 1)
+        if g.shape[0] != K or not g.is_contiguous():
+            raise ValueError("g must be a contiguous [K] bf16 tensor")
+    ldr = _row_stride(residual, K) if residual is not None else K
+    ldo = _row_stride(residual_out, K) if residual_out is not None else K
+    return M, K, ldr, ldo
+
+
+def rmsnorm_residual(X: torch.Tensor, residual: torch.Tensor | None = None,
+                     g: torch.Tensor | None = None, eps: float = 1e-6,
+                     residual_out: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """The input RMSNorm of int8_linear (ck_rmsnorm_residual): h = bf16(X +
+    residual) (h = X without one), written to ``residual_out`` when given (it
+    may be ``residual`` itself); returns bf16((h / sqrt(mean(h^2) + eps)) * g)."""
+    M, K, ldr, ldo = _norm_args(X, residual, residual_out, g)
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    _check(lib.ck_rmsnorm_residual(_ptr(X), _row_stride(X, K), _ptr(residual), ldr,
+                                   _ptr(residual_out), ldo, _ptr(g), float(eps), M, K, _ptr(out),
+                                   _stream(stream)), "ck_rmsnorm_residual")
+    return out
+
+
+def norm_workspace_bytes(M: int, K: int) -> int:
+    return int(lib.ck_int8_linear_norm_workspace_bytes(M, K))
+
+
+def int8_linear_norm(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                     bias: torch.Tensor | None = None, residual: torch.Tensor | None = None,
+                     g: torch.Tensor | None = None, eps: float = 1e-6,
+                     residual_out: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """int8_linear on the input RMSNorm (and residual) of X (ck_int8_linear_norm)."""
+    M, K, ldr, ldo = _norm_args(X, residual, residual_out, g)
+    _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
+    _need(s_w, "s_w", torch.float32, 1)
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, Qw {tuple(Qw.shape)}, s_w {tuple(s_w.shape)}")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    need = norm_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.ck_int8_linear_norm(_ptr(X), _row_stride(X, K), _ptr(residual), ldr,
+                                   _ptr(residual_out), ldo, _ptr(g), float(eps), _ptr(Qw),
+                                   _ptr(s_w), _ptr(bias), _ptr(out), M, N, K, _ptr(workspace),
+                                   ws_bytes, _stream(stream)), "ck_int8_linear_norm")
     return out
 
 

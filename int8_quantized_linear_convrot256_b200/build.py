@@ -36,7 +36,7 @@ PER_FILE = {
     "dequant.cu": ["-fmad=false"],
 }
 SOURCES = ["api.cu", "quant_rotate.cu", "gemm_i8_tcgen05.cu", "gemm_nvfp4_tcgen05.cu", "noalloc.cu",
-           "dequant.cu"]
+           "dequant.cu", "rmsnorm.cu"]
 HEADERS = ["ck_device.cuh", "internal.h", "libck.map"]
 
 

@@ -384,6 +384,80 @@ ck_status ck_int8_linear(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const 
                               workspace_bytes, stream);
 }
 
+// Arguments of the input RMSNorm (ck_rmsnorm_residual's rules), M > 0.
+static ck_status check_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual, int64_t ldr,
+                            const ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g, float eps,
+                            int64_t K) {
+    if (!X || ldx < K || (residual && ldr < K) || (residual_out && ldo < K) ||
+        !(eps > 0.0f) || !(eps <= 3.4e38f))
+        return CK_ERR_INVALID_VALUE;
+    if (!aligned16(X) || ldx % 8 != 0 || (residual && (!aligned16(residual) || ldr % 8 != 0)) ||
+        (residual_out && (!aligned16(residual_out) || ldo % 8 != 0)) || (g && !aligned16(g)))
+        return CK_ERR_MISALIGNED;
+    return CK_OK;
+}
+
+ck_status ck_rmsnorm_residual(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual, int64_t ldr,
+                              ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g, float eps,
+                              int64_t M, int64_t K, ck_bf16 *Y, ck_stream_t stream) {
+    if (M < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s != CK_OK) return s;
+    if (M == 0) return CK_OK;
+    if (!Y) return CK_ERR_INVALID_VALUE;
+    s = check_norm(X, ldx, residual, ldr, residual_out, ldo, g, eps, K);
+    if (s != CK_OK) return s;
+    if (!aligned16(Y)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_rmsnorm_rows(X, ldx, residual, ldr, residual_out, ldo, g, eps, M, K,
+                                            Y, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+size_t ck_int8_linear_norm_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return round256(size_t(M) * size_t(K) * 2) + ck_int8_linear_workspace_bytes(M, K);
+}
+
+ck_status ck_int8_linear_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual,
+                              int64_t ldr, ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g,
+                              float eps, const int8_t *Qw, const float *s_w, const ck_bf16 *bias,
+                              ck_bf16 *Y, int64_t M, int64_t N, int64_t K, void *workspace,
+                              size_t workspace_bytes, ck_stream_t stream) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (M > 0 && N > 0 && (!X || !Qw || !s_w || !Y || !workspace)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    s = check_norm(X, ldx, residual, ldr, residual_out, ldo, g, eps, K);
+    if (s != CK_OK) return s;
+    if (!aligned16(Qw) || !aligned16(s_w) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CK_ERR_MISALIGNED;
+    if (workspace_bytes < ck_int8_linear_norm_workspace_bytes(M, K)) return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    ck_bf16 *Xn = reinterpret_cast<ck_bf16 *>(base);
+    int8_t *Qx = reinterpret_cast<int8_t *>(base + round256(size_t(M) * size_t(K) * 2));
+    float *s_x = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Qx) +
+                                           round256(size_t(M) * size_t(K)));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = ck::launch_rmsnorm_rows(X, ldx, residual, ldr, residual_out, ldo, g, eps, M, K,
+                                            Xn, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    e = ck::launch_quant_rows_bf16(Xn, M, K, K, true, CK_ACT_NONE, 127, Qx, s_x, st->err,
+                                   st->num_sms, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
+}
+
 size_t ck_int8_linear_host_workspace_bytes(int64_t chunk_rows, int64_t N, int64_t K) {
     if (chunk_rows <= 0 || N <= 0 || K <= 0) return 0;
     const size_t r = size_t(chunk_rows);

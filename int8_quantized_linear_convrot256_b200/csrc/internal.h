@@ -37,6 +37,13 @@ cudaError_t launch_dequant_nvfp4(const uint8_t *Q, const uint8_t *S, const float
 cudaError_t launch_unpack_int4(const uint8_t *Q4, int64_t rows, int64_t K, int8_t *Q8,
                                int num_sms, cudaStream_t stream);
 
+// ---- input RMSNorm with a residual (rmsnorm.cu): Y [M, K] (row stride K) =
+// bf16((h * inv) * g), h = bf16(x + r) (x without R) also written to Rout
+// when given (row stride ldo; it may alias X or R).
+cudaError_t launch_rmsnorm_rows(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t ldr,
+                                uint16_t *Rout, int64_t ldo, const uint16_t *g, float eps,
+                                int64_t M, int64_t K, uint16_t *Y, cudaStream_t stream);
+
 // ---- dequantize_int8_simple(_dtype), quantize_int8_tensorwise (dequant.cu)
 
 cudaError_t launch_dequantize_int8(const int8_t *Q, const float *S, int64_t rows, int64_t K,

@@ -192,3 +192,65 @@ def test_nvfp4_validation(call, status):
         assert got in (ck.CK_ERR_CUDA, ck.CK_ERR_ARCH)
     else:
         assert got == status
+
+
+def norm(X=FAKE, ldx=512, R=None, ldr=512, Ro=None, ldo=512, g=None, eps=1e-6, M=4, K=512, Y=FAKE):
+    return ck.lib.ck_rmsnorm_residual(X, ldx, R, ldr, Ro, ldo, g, eps, M, K, Y, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(X=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(Y=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(M=-1), ck.CK_ERR_INVALID_VALUE),
+    (dict(K=0), ck.CK_ERR_INVALID_VALUE),
+    (dict(ldx=256), ck.CK_ERR_INVALID_VALUE),
+    (dict(R=FAKE, ldr=256), ck.CK_ERR_INVALID_VALUE),
+    (dict(Ro=FAKE, ldo=256), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=0.0), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=-1e-6), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=float("nan")), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=float("inf")), ck.CK_ERR_INVALID_VALUE),
+    (dict(K=300, ldx=512), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(X=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(ldx=516), ck.CK_ERR_MISALIGNED),
+    (dict(R=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(R=FAKE, ldr=516), ck.CK_ERR_MISALIGNED),
+    (dict(Ro=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(g=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(Y=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(M=0), ck.CK_OK),
+])
+def test_rmsnorm_validation(kw, status):
+    assert norm(**kw) == status
+
+
+def lin_norm(X=FAKE, ldx=512, R=None, ldr=512, Ro=None, ldo=512, g=None, eps=1e-6, Qw=FAKE,
+             s_w=FAKE, bias=None, Y=FAKE, M=4, N=8, K=512, ws=FAKE, ws_bytes=1 << 30):
+    return ck.lib.ck_int8_linear_norm(X, ldx, R, ldr, Ro, ldo, g, eps, Qw, s_w, bias, Y, M, N, K,
+                                      ws, ws_bytes, None)
+
+
+def test_norm_workspace_bytes():
+    assert ck.norm_workspace_bytes(0, 256) == 0
+    assert ck.norm_workspace_bytes(3, 256) == 3 * 256 * 2 + 768 + 256
+    M, K = 32700, 5376
+    assert ck.norm_workspace_bytes(M, K) == M * K * 2 + ck.workspace_bytes(M, K)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(X=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(Y=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(ws=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=0.0), ck.CK_ERR_INVALID_VALUE),
+    (dict(ldx=256), ck.CK_ERR_INVALID_VALUE),
+    (dict(K=300, ldx=512), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(N=12), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(g=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(Qw=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(ws=FAKE + 16), ck.CK_ERR_MISALIGNED),
+    (dict(ws_bytes=4096), ck.CK_ERR_WORKSPACE),
+    (dict(M=0), ck.CK_OK),
+    (dict(N=0), ck.CK_OK),
+])
+def test_int8_linear_norm_validation(kw, status):
+    assert lin_norm(**kw) == status
