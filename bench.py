@@ -155,14 +155,33 @@ class ClockSampler:
 # ---------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float, act: str = "none"):
-    """Time the oracle on a bounded sample of rows (quantise + linear rows).
+NORM_EPS = 1e-6
+
+
+def norm_inputs(cfg, M):
+    """Residual [M, K] and RMSNorm weight [K] of the --path norm workload
+    (bf16, seeded from the config's seed)."""
+    import torch
+
+    g = torch.Generator().manual_seed(cfg.seed + 1000)
+    R = torch.randn(M, cfg.K, generator=g).to(torch.bfloat16)
+    w = (1.0 + 0.25 * torch.randn(cfg.K, generator=g)).to(torch.bfloat16)
+    return R, w
+
+
+def oracle_sample(cfg, X_bits, Qw, s_w, bias_bits, seconds: float, act: str = "none",
+                  norm=None):
+    """Time the oracle on a bounded sample of rows (quantise + linear rows;
+    with ``norm`` = (residual bits, weight bits) the input RMSNorm first).
     Returns (TOPS, rows, seconds, threads)."""
     import oracle
 
     def run(rows):
         t = time.perf_counter()
-        Qx, s_x = oracle.quantize_rows_bf16(X_bits[:rows], act=act)
+        Xs = X_bits[:rows]
+        if norm is not None:
+            Xs, _ = oracle.rmsnorm_rows(Xs, norm[0][:rows], norm[1], NORM_EPS)
+        Qx, s_x = oracle.quantize_rows_bf16(Xs, act=act)
         oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
         return time.perf_counter() - t
 
@@ -211,6 +230,17 @@ def run_reference(args, cfg, rank, world):
         def run(rows):
             oracle.convrot_w4a4_linear(X_bits[:rows], Qw4, s_w, bias_bits)
         what, dtype = "convrot_w4a4_linear of those rows", "int8"
+    elif args.path == "norm":
+        Qw, s_w = oracle.rotate_quant_weight(W.numpy())
+        R, w = norm_inputs(cfg, cfg.M)
+        R_bits, w_bits = workloads.bf16_bits(R), workloads.bf16_bits(w)
+
+        def run(rows):
+            Xn, _ = oracle.rmsnorm_rows(X_bits[:rows], R_bits[:rows], w_bits, NORM_EPS)
+            Qx, s_x = oracle.quantize_rows_bf16(Xn)
+            oracle.linear_rows(Qx, s_x, Qw, s_w, bias_bits, np.arange(rows))
+        what, dtype = ("input RMSNorm with residual, quantize_and_rotate_rowwise and the outputs "
+                       "of those rows"), "int8"
     else:
         Qw, s_w = oracle.rotate_quant_weight(W.numpy())
 
@@ -256,7 +286,10 @@ def config_dict(cfg, world, scaling="weak", act="none", path="int8"):
             "parallelism": par + " (rows are independent: no collective on the data path)",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); X is also larger than L2",
             "weights": "rotated + quantised once before timing (offline)",
-            "input_act": act, "path": path}
+            "input_act": act, "path": path,
+            **({"input_norm": f"RMSNorm with a residual and a weight, eps {NORM_EPS} (residual "
+                              f"~ N(0, 1), weight ~ 1 + N(0, 0.25^2), seed + 1000)"}
+               if path == "norm" else {})}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -293,6 +326,13 @@ def run_ours(args, cfg, rank, world, local_rank):
         Qx = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
         Sx = torch.empty((ck.nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
         s_x = torch.empty((1,), dtype=torch.float32, device=dev)
+    if args.path == "norm":
+        R, w_norm = norm_inputs(cfg, cfg.M)
+        if args.scaling == "strong":
+            R = R[lo:hi].contiguous()
+        Rd, gd = R.to(dev), w_norm.to(dev)
+        Ro = torch.empty_like(Rd)  # the residual output (a separate buffer: steps stay equal)
+        Xn = torch.empty_like(Xd)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
@@ -306,6 +346,10 @@ def run_ours(args, cfg, rank, world, local_rank):
             ck.unpack_int4(Qw4, out=Qw)
         elif args.path == "nvfp4":
             ck.quantize_rotate_nvfp4(Xd, Qx, Sx, s_x)
+        elif args.path == "norm":
+            # int8_linear's input RMSNorm and residual, then the quantiser
+            ck.rmsnorm_residual(Xd, Rd, gd, NORM_EPS, residual_out=Ro, out=Xn)
+            ck.quantize_rotate_rowwise(Xn, Qx, s_x)
         elif args.act == "none":
             ck.quantize_rotate_rowwise(Xd, Qx, s_x)
         else:
@@ -361,7 +405,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     ms_step, ms_q, ms_g, *spread = max_over_ranks([ms_step, ms_q, ms_g, *spread], dev)
 
     # ---- end to end through the public composite call, host buffers
-    if args.no_e2e or args.path in ("w4a4", "nvfp4"):
+    if args.no_e2e or args.path in ("w4a4", "nvfp4", "norm"):
         ms_e2e = float("nan")
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
@@ -421,6 +465,12 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
         # FP4 codes and one E4M3 scale per 16 values written
         q_bytes = 2.0 * M * K + 0.5 * M * K + M * K / 16.0 + 4.0
         int8_peak = P["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    elif args.path == "norm":
+        # the input RMSNorm (X and the residual read, residual output and the
+        # normalised rows written) and the quantiser (those rows read, codes
+        # and row scales written)
+        q_bytes = 8.0 * M * K + 3.0 * M * K + 4.0 * M
+        int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     else:
         q_bytes = 3.0 * M * K + 4.0 * M
         int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
@@ -442,17 +492,24 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
     line = None
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        # (the w4a4 and nvfp4 paths have their oracle in the reference arm only)
+        if world == 1 and not args.no_cpu_baseline and args.path in ("int8", "norm"):
             X_bits = workloads.bf16_bits(X)
             import oracle
 
             Qw_o, s_w_o = oracle.rotate_quant_weight(Wcpu.numpy())
+            norm = None
+            if args.path == "norm":
+                R_o, w_o = norm_inputs(cfg, cfg.M)  # the same seeded values as on the device
+                norm = (workloads.bf16_bits(R_o), workloads.bf16_bits(w_o))
             tops, rows, dt, cores = oracle_sample(cfg, X_bits, Qw_o, s_w_o,
                                                   workloads.bf16_bits(bias), args.cpu_seconds,
-                                                  args.act)
+                                                  args.act, norm)
+            what = "input RMSNorm, " if norm is not None else ""
             cpu = {"value": tops, "unit": UNIT, "cores": cores, "kind": "oracle",
-                   "sample": f"{rows} of {cfg.M} rows (rotate+quantise and all {cfg.N} outputs of "
-                             f"those rows) in {dt:.1f} s, plain C oracle, OpenMP over rows"}
+                   "sample": f"{rows} of {cfg.M} rows ({what}rotate+quantise and all {cfg.N} "
+                             f"outputs of those rows) in {dt:.1f} s, plain C oracle, OpenMP over "
+                             f"rows"}
         page_ms = PAGE_MS.get(cfg.name)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -482,17 +539,20 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                          "ms_per_launch": ms_g},
             "quantizer": {"kernel": ("nvfp4_bulk_kernel<1> + <2> (ConvRot256 + NVFP4, two "
                                      "staged passes over X)" if args.path == "nvfp4" else
+                                     "rmsnorm_rows_kernel + quant_rows_bulk_kernel (input "
+                                     "RMSNorm with residual, then ConvRot256 + per-row INT8)"
+                                     if args.path == "norm" else
                                      ("quant_rows_bulk_kernel" if K <= 28672 else
                                       "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)"),
                           "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",
                           "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
                           "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},
             "cpu_baseline": cpu,
-            "e2e": None if (args.no_e2e or args.path in ("w4a4", "nvfp4")) else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
+            "e2e": None if (args.no_e2e or args.path in ("w4a4", "nvfp4", "norm")) else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
                     "call": f"ck_int8_linear_host: X from and Y to pinned host memory, chunks of "
                             f"{min(E2E_CHUNK_ROWS, M)} rows with copies overlapped with the kernels"},
-            "gpu_launches": {"w4a4": 3, "nvfp4": 4}.get(args.path, 2) * args.steps,
+            "gpu_launches": {"w4a4": 3, "nvfp4": 4, "norm": 3}.get(args.path, 2) * args.steps,
             "clocks": clocks.summary(t_wall0, t_wall1),
         }
     return line
@@ -508,10 +568,11 @@ def main(argv=None):
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: every rank runs the whole batch (replicas); strong: the "
                          "batch's rows are split over the ranks")
-    ap.add_argument("--path", default="int8", choices=["int8", "w4a4", "nvfp4"],
+    ap.add_argument("--path", default="int8", choices=["int8", "w4a4", "nvfp4", "norm"],
                     help="int8: int8_linear; w4a4: convrot_w4a4_linear (INT4 codes, packed "
                          "INT4 weights unpacked per step); nvfp4: ConvRot NVFP4 (two-pass "
-                         "FP4 quantiser + block-scaled FP4 GEMM)")
+                         "FP4 quantiser + block-scaled FP4 GEMM); norm: int8_linear with its "
+                         "input RMSNorm and a residual (ck_rmsnorm_residual first)")
     ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
