@@ -6,7 +6,8 @@ The CUDA product path never imports this package, and this package imports
 nothing from the product.
 
 The arithmetic lives in ``convrot_oracle.c`` (plain C, IEEE fp32, no
-contraction); this module compiles it with gcc on first use and wraps it with
+contraction; double precision where a step is defined as the bf16 rounding of
+an exact value); this module compiles it with gcc on first use and wraps it with
 numpy arrays. BF16 values travel as numpy ``uint16`` bit patterns.
 
 What each function follows (page title, section):
@@ -20,6 +21,13 @@ What each function follows (page title, section):
   - ``gemm_i32`` / ``epilogue`` / ``int8_linear``: ComfyUI-AppleSilicon-FP8
     README row 17 (INT8 x INT8 -> INT32, per-row rescale + bias in the store
     epilogue) and comfy-kitchen "int8_linear".
+  - ``act_bf16`` (input_act): comfy-kitchen 0.2.40, "HIP backend"
+    (int8_linear(input_act=...) folded into the quantiser's load); each bf16
+    input becomes the bf16 value nearest to the exact relu / silu / tanh-form
+    gelu of it, evaluated in double precision.
+  - ``rmsnorm_rows``: comfy-kitchen 0.2.40, "Huawei Ascend backend"
+    (int8_linear's input RMSNorm and residual arguments): h = bf16(x + r),
+    y = the bf16 value nearest to the exact h g / sqrt(mean(h^2) + eps).
   - ``e2m1_*``, ``e4m3_*``, ``nvfp4_*``: ComfyUI-HSWQ-Loader-and-Tools, "NVFP4
     torch.compile Fix", section 5-1 (nvfp4_gemm.py): the E2M1 value table,
     16-value blocks, the blocked scale layout that from_blocked undoes, a
@@ -96,10 +104,12 @@ def lib():
             L.oracle_dequantize_int8.restype = None
             L.oracle_quantize_int8_tensorwise.argtypes = [u16p, i64, i64, i64, i8p, f32p]
             L.oracle_quantize_int8_tensorwise.restype = None
-            L.oracle_exp.argtypes = [ctypes.c_float]
-            L.oracle_exp.restype = ctypes.c_float
-            L.oracle_act.argtypes = [ctypes.c_int, ctypes.c_float]
-            L.oracle_act.restype = ctypes.c_float
+            L.oracle_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+            L.oracle_f64_to_bf16_rne.restype = ctypes.c_uint16
+            L.oracle_act_f64.argtypes = [ctypes.c_int, ctypes.c_double]
+            L.oracle_act_f64.restype = ctypes.c_double
+            L.oracle_act_bf16_array.argtypes = [ctypes.c_int, u16p, i64, u16p]
+            L.oracle_act_bf16_array.restype = None
             L.oracle_rotate_quant_weight.argtypes = [f32p, i64, i64, i8p, f32p]
             L.oracle_rotate_quant_weight.restype = ctypes.c_int
             L.oracle_gemm_i32.argtypes = [i8p, i8p, i64, i64, i64, i32p]
@@ -134,7 +144,7 @@ def lib():
                                                    _P(ctypes.c_double)]
             L.oracle_nvfp4_linear_rows.restype = None
             L.oracle_rmsnorm_rows.argtypes = [u16p, i64, u16p, i64, u16p, ctypes.c_float, i64,
-                                              i64, u16p, u16p]
+                                              i64, u16p, u16p, u16p]
             L.oracle_rmsnorm_rows.restype = ctypes.c_int
             L.oracle_num_threads.argtypes = []
             L.oracle_num_threads.restype = ctypes.c_int
@@ -202,19 +212,31 @@ def quant_rows(y, qmax: float = 127.0) -> tuple[np.ndarray, np.ndarray]:
 ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu_tanh": 3}
 
 
-def exp(x) -> np.ndarray:
-    """The oracle's own fp32 e^x (used by the activations), element-wise."""
-    x = np.asarray(x, dtype=np.float32)
+def f64_to_bf16(v) -> np.ndarray:
+    """float64 -> bf16 bits, round-to-nearest-even from the double value directly."""
+    v = np.asarray(v, dtype=np.float64)
     L = lib()
-    return np.array([L.oracle_exp(float(v)) for v in x.reshape(-1)], np.float32).reshape(x.shape)
+    return np.array([L.oracle_f64_to_bf16_rne(float(t)) for t in v.reshape(-1)],
+                    np.uint16).reshape(v.shape)
 
 
-def act(name: str, x) -> np.ndarray:
-    """fp32 activation (before the bf16 rounding), element-wise."""
-    x = np.asarray(x, dtype=np.float32)
+def act_f64(name: str, x) -> np.ndarray:
+    """The activation evaluated in double precision (before any rounding)."""
+    x = np.asarray(x, dtype=np.float64)
     L = lib()
     a = ACTS[name]
-    return np.array([L.oracle_act(a, float(v)) for v in x.reshape(-1)], np.float32).reshape(x.shape)
+    return np.array([L.oracle_act_f64(a, float(t)) for t in x.reshape(-1)],
+                    np.float64).reshape(x.shape)
+
+
+def act_bf16(name: str, x_bits) -> np.ndarray:
+    """input_act as the quantiser applies it: each bf16 input (uint16 bits)
+    becomes the bf16 value nearest to the exact act(x), ties to even."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    y = np.empty_like(x)
+    lib().oracle_act_bf16_array(ACTS[name], _ptr(x.reshape(-1), ctypes.c_uint16), x.size,
+                                _ptr(y.reshape(-1), ctypes.c_uint16))
+    return y
 
 
 def quantize_rows_bf16(X_bits: np.ndarray, rotate: bool = True, K: int | None = None,
@@ -361,14 +383,18 @@ def int8_linear(X_bits, Qw, s_w, bias_bits=None, act: str = "none"):
 
 # --------------------------------------------------------- input RMSNorm
 
-def rmsnorm_rows(X_bits, residual_bits=None, g_bits=None, eps: float = 1e-6):
+def rmsnorm_rows(X_bits, residual_bits=None, g_bits=None, eps: float = 1e-6,
+                 with_alt: bool = False):
     """The input RMSNorm with an optional residual (the C oracle's reading:
-    h = bf16(x + r), y = bf16((h / sqrt(mean(h^2) + eps)) * g), the sum of
-    squares in the order stated there). Returns (Y bits [M, K], h bits)."""
+    h = bf16(x + r), y = the bf16 value nearest to h g / sqrt(mean(h^2) + eps)).
+    Returns (Y bits [M, K], h bits), and with ``with_alt`` also Yalt: the
+    other bf16 neighbour where the exact value lies within 2^-34 (relative)
+    of a rounding midpoint, Y elsewhere (both then count as correct)."""
     X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
     M, K = X_bits.shape
     Y = np.empty((M, K), np.uint16)
     H = np.empty((M, K), np.uint16)
+    Ya = np.empty((M, K), np.uint16)
     rp = gp = None
     ldr = K
     if residual_bits is not None:
@@ -380,10 +406,11 @@ def rmsnorm_rows(X_bits, residual_bits=None, g_bits=None, eps: float = 1e-6):
         assert g_bits.shape == (K,)
         gp = _ptr(g_bits, ctypes.c_uint16)
     rc = lib().oracle_rmsnorm_rows(_ptr(X_bits, ctypes.c_uint16), K, rp, ldr, gp, float(eps), M,
-                                   K, _ptr(Y, ctypes.c_uint16), _ptr(H, ctypes.c_uint16))
+                                   K, _ptr(Y, ctypes.c_uint16), _ptr(H, ctypes.c_uint16),
+                                   _ptr(Ya, ctypes.c_uint16))
     if rc != 0:
         raise ValueError(f"oracle_rmsnorm_rows failed ({rc}); K must be a multiple of 256")
-    return Y, H
+    return (Y, H, Ya) if with_alt else (Y, H)
 
 
 def int8_linear_norm(X_bits, Qw, s_w, bias_bits=None, residual_bits=None, g_bits=None,

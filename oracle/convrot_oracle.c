@@ -8,8 +8,11 @@
  * It is deliberately plain and slow: every step is written out in the order of
  * the method's definition, in IEEE single precision with round-to-nearest-even
  * and no operation fused or reordered (compile with -ffp-contract=off and
- * without -ffast-math). Rows are spread over OpenMP threads; that changes no
- * arithmetic, because every output element is computed by one thread alone.
+ * without -ffast-math). Where the definition is the bf16 rounding of an exact
+ * real value (the input activation, the input RMSNorm), that value is
+ * evaluated in double precision and rounded once. Rows are spread over OpenMP
+ * threads; that changes no arithmetic, because every output element is
+ * computed by one thread alone.
  *
  * Sources for what is computed:
  *  - comfy-kitchen 0.2.40 (PyPI page), "Huawei Ascend backend" and "HIP
@@ -73,74 +76,88 @@ uint16_t oracle_f32_to_bf16_rne(float f) {
  * linear(act(proj(x))) never stores act's output. The pages do not list the
  * activations nor their formulas; the readings taken: relu, silu
  * x / (1 + e^-x) and the tanh form of gelu
- * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), computed in fp32 on the
- * widened bf16 input and rounded to bf16 (the precision an unfused bf16
- * activation would store) before the rotation. The gelu is evaluated as
- * x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3), which equals
- * 0.5 x (1 + tanh(u)) and has no cancellation where tanh(u) is near -1.
+ * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))). Each bf16 input x becomes
+ * the bf16 value nearest to the exact act(x) (ties to even), which is what an
+ * unfused activation stored in bf16 would hold at best; that value then goes
+ * through the rotation and the quantiser.
  *
- * e^x: Cody-Waite reduction x = n ln2 + r with ln2 split in a 16-bit head
- * and a tail, each reduction step one fused multiply-add (fmaf: one IEEE
- * rounding), a degree-7 Taylor polynomial of e^r (|r| <= ln2/2, truncation
- * error below 2^-27) in Horner form with fused multiply-adds, then an exact
- * scaling by 2^n (two steps when 2^n is subnormal). */
+ * The exact value is evaluated here in double precision (libm exp), the gelu
+ * as x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3): the same number as
+ * 0.5 x (1 + tanh(u)) without its cancellation where tanh(u) is near -1.
+ * Rounding the double result once to bf16 gives the exact value's bf16
+ * rounding unless that value lies within the double evaluation's error
+ * (about |2u| * 2^-52 relative) of a rounding midpoint. For x != 0 act(x) is
+ * transcendental and never a midpoint itself. One case needs care: for
+ * |x| < 2^-120 the double evaluation returns x/2 exactly (1 + e^-x rounds to
+ * 2), which can be a midpoint between two bf16 subnormals, while the exact
+ * value is strictly above x/2 (act(x) - x/2 = x (sigma(.) - 1/2) > 0, with
+ * sigma(.) - 1/2 of the sign of x) by less than x^2 / 2, far below the
+ * spacing; so there x/2 is rounded with ties going up. */
 #define ACT_NONE 0
 #define ACT_RELU 1
 #define ACT_SILU 2
 #define ACT_GELU_TANH 3
 
-static float pow2i(int k) { /* 2^k for -126 <= k <= 127, exact */
-    uint32_t u = (uint32_t)(k + 127) << 23;
-    float f;
-    memcpy(&f, &u, sizeof f);
-    return f;
+/* float64 -> bf16 by the definition of round-to-nearest-even, from the double
+ * value directly (no intermediate fp32 rounding): bf16 keeps 8 significant
+ * bits, with spacing 2^(e-8) for |v| in [2^(e-1), 2^e) and 2^-133 below
+ * 2^-126 (subnormals); |v| at or above 2^128 - 2^119 overflows to infinity. */
+uint16_t oracle_f64_to_bf16_rne(double v) {
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a != a)
+        return 0x7FC0u;
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+    int qe = e - 8;
+    if (qe < -133)
+        qe = -133;
+    double q = nearbyint(ldexp(a, -qe)); /* exact scaling, then ties to even */
+    double r = ldexp(q, qe);
+    if (r >= 0x1p128)
+        return (uint16_t)(sign | 0x7F80u);
+    float f = (float)r; /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
 }
 
-float oracle_exp(float x) {
-    if (x > 88.8f)
-        return INFINITY;
-    if (x < -104.0f)
-        return 0.0f;
-    const float log2e = 1.442695f;
-    const float ln2_hi = 0.693145751953125f;
-    const float ln2_lo = 1.4286068e-06f;
-    float n = nearbyintf(x * log2e);
-    float r = fmaf(-n, ln2_hi, x);
-    r = fmaf(-n, ln2_lo, r);
-    float p = 1.984127e-04f; /* 1/7!, 1/6!, ... rounded to fp32 */
-    p = fmaf(p, r, 1.3888889e-03f);
-    p = fmaf(p, r, 8.333334e-03f);
-    p = fmaf(p, r, 4.1666668e-02f);
-    p = fmaf(p, r, 1.6666667e-01f);
-    p = fmaf(p, r, 0.5f);
-    p = fmaf(p, r, 1.0f);
-    p = fmaf(p, r, 1.0f);
-    int k = (int)n;
-    if (k > 127)
-        return (p * pow2i(127)) * pow2i(k - 127);
-    if (k < -126)
-        return (p * pow2i(k + 100)) * pow2i(-100);
-    return p * pow2i(k);
-}
-
-float oracle_act(int act, float x) {
+double oracle_act_f64(int act, double x) {
     switch (act) {
     case ACT_RELU:
-        return x > 0.0f ? x : 0.0f;
-    case ACT_SILU: {
-        float e = oracle_exp(-x);
-        return x / (1.0f + e);
-    }
+        return x > 0.0 ? x : 0.0;
+    case ACT_SILU:
+        return x / (1.0 + exp(-x));
     case ACT_GELU_TANH: {
-        float x3 = (x * x) * x;
-        float inner = fmaf(0.044715f, x3, x);
-        float u = 7.978846e-01f * inner; /* sqrt(2/pi) */
-        float e = oracle_exp(-2.0f * u);
-        return x / (1.0f + e);
+        double u = sqrt(2.0 / 3.14159265358979323846) * (x + 0.044715 * (x * x * x));
+        return x / (1.0 + exp(-2.0 * u));
     }
     default:
         return x;
     }
+}
+
+/* The activation of one bf16 input, as bf16 bits. */
+uint16_t oracle_act_bf16(int act, uint16_t xb) {
+    double x = (double)oracle_bf16_to_f32(xb);
+    if (act == ACT_NONE)
+        return xb;
+    if ((act == ACT_SILU || act == ACT_GELU_TANH) && x != 0.0 && fabs(x) < 0x1p-120) {
+        double t = ldexp(x / 2.0, 133); /* x/2 in units of the subnormal spacing */
+        double lo = floor(t);
+        double q = (t - lo == 0.5) ? lo + 1.0 : nearbyint(t);
+        return oracle_f64_to_bf16_rne(copysign(ldexp(q, -133), x)); /* -0 stays -0 */
+    }
+    return oracle_f64_to_bf16_rne(oracle_act_f64(act, x));
+}
+
+void oracle_act_bf16_array(int act, const uint16_t *x, int64_t n, uint16_t *y) {
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = oracle_act_bf16(act, x[i]);
 }
 
 /* ConvRot256 on one block of 256 values, in place. */
@@ -230,10 +247,7 @@ int oracle_quantize_rows_bf16_q(const uint16_t *X, int64_t M, int64_t K, int64_t
             for (int64_t m = 0; m < M; ++m) {
                 const uint16_t *row = X + m * ldx;
                 for (int64_t k = 0; k < K; ++k) {
-                    float v = oracle_bf16_to_f32(row[k]);
-                    if (act != ACT_NONE)
-                        v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));
-                    buf[k] = v;
+                    buf[k] = oracle_bf16_to_f32(oracle_act_bf16(act, row[k]));
                 }
                 if (rotate)
                     for (int64_t b = 0; b < K; b += ROT_N)
@@ -431,23 +445,59 @@ int oracle_num_threads(void) {
  * comfy-kitchen 0.2.40 (PyPI page), "Huawei Ascend backend": int8_linear
  * accepts the input RMSNorm and residual arguments and applies them with the
  * shared device-side helpers, apart from its GEMM. The page prints no
- * formula. The reading here is the usual add-then-normalise form, each step
- * an IEEE fp32 operation:
- *   h   = bf16_rne(float(x) + float(r))      (h = x when there is no residual)
- *   the residual output is h
- *   ss  = the sum of h_k^2 over the row, in this order: 32 partial sums p_l
- *         (l = 0..31), p_l taking, for i = 0, 1, ... and then j = 0..7, the
- *         element k = 256 i + 8 l + j with one fused multiply-add each
- *         (p_l = fma(h_k, h_k, p_l), from +0); then five butterfly levels
- *         p_l = p_l + p_(l xor m) for m = 16, 8, 4, 2, 1 (every l ends with
- *         the same value, the sum)
- *   inv = 1 / sqrt(ss / K + eps)
- *   y   = bf16_rne((h * inv) * float(g_k))   (bf16_rne(h * inv) without g)
- * The order of the sum is part of the reading: the pages give none, and any
- * fixed order defines the same function up to fp32 rounding. */
+ * formula. The reading here is the usual add-then-normalise form:
+ *   h   = bf16_rne(fl32(x + r))   the residual add as a bf16 tensor addition
+ *                                 stores it (h = x when there is no residual);
+ *                                 the residual output is h
+ *   y_k = the bf16 value nearest to h_k g_k / sqrt(mean_k(h_k^2) + eps)
+ *         (ties to even; without g, g_k = 1), the exact real value.
+ * The exact value is evaluated in double precision: every h_k^2 and h_k g_k
+ * is exact in double (8-bit significands), the sum of squares is
+ * compensated (Neumaier's variant of Kahan summation, error about 2^-52
+ * relative), then one division, one square root and two products. Where
+ * that value lies within 2^-34 (relative) of a bf16 rounding midpoint, both
+ * neighbours count as correct: an evaluation in double precision whose sum
+ * of squares runs in any order (relative error below K 2^-53 <= 2^-36 for
+ * K <= 2^17) may land on either side. Yalt receives the other neighbour for
+ * those elements and y itself elsewhere. eps must be > 0 (a zero row then
+ * gives y = 0). */
+static double sum_squares_bf16(const uint16_t *h, int64_t K) {
+    double s = 0.0, c = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double v = (double)oracle_bf16_to_f32(h[k]);
+        double t = v * v; /* exact */
+        double n = s + t;
+        if (fabs(s) >= fabs(t))
+            c += (s - n) + t;
+        else
+            c += (t - n) + s;
+        s = n;
+    }
+    return s + c;
+}
+
+/* Round v to bf16 and report the other neighbour when v lies within
+ * tol * |v| of the midpoint between the two (alt = the rounding otherwise). */
+static uint16_t bf16_round_with_alt(double v, double tol, uint16_t *alt) {
+    uint16_t r = oracle_f64_to_bf16_rne(v);
+    *alt = r;
+    double rv = (double)oracle_bf16_to_f32(r);
+    if (rv == v || isinf(rv))
+        return r;
+    /* the neighbour on v's other side of r */
+    uint16_t o = (uint16_t)((fabs(v) > fabs(rv)) ? r + 1u : r - 1u);
+    if (fabs(rv) == 0.0)
+        o = (uint16_t)((v > 0) ? 0x0001u : 0x8001u);
+    double ov = (double)oracle_bf16_to_f32(o);
+    double mid = 0.5 * (rv + ov); /* exact: both have 8 significant bits */
+    if (fabs(v - mid) <= tol * fabs(v))
+        *alt = o;
+    return r;
+}
+
 int oracle_rmsnorm_rows(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t ldr,
                         const uint16_t *g, float eps, int64_t M, int64_t K, uint16_t *Y,
-                        uint16_t *Rout) {
+                        uint16_t *Rout, uint16_t *Yalt) {
     if (K % ROT_N != 0) return -1;
     int err = 0;
 #pragma omp parallel
@@ -467,25 +517,15 @@ int oracle_rmsnorm_rows(const uint16_t *X, int64_t ldx, const uint16_t *R, int64
             }
             if (Rout)
                 for (int64_t k = 0; k < K; ++k) Rout[m * K + k] = h[k];
-            float p[32], q[32];
-            for (int l = 0; l < 32; ++l) {
-                p[l] = 0.0f;
-                for (int64_t i = 0; i < K / ROT_N; ++i)
-                    for (int j = 0; j < 8; ++j) {
-                        float v = oracle_bf16_to_f32(h[ROT_N * i + 8 * l + j]);
-                        p[l] = fmaf(v, v, p[l]);
-                    }
-            }
-            for (int mm = 16; mm >= 1; mm >>= 1) {
-                for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ mm];
-                for (int l = 0; l < 32; ++l) p[l] = q[l];
-            }
-            float ss = p[0];
-            float inv = 1.0f / sqrtf(ss / (float)K + eps);
+            double ss = sum_squares_bf16(h, K);
+            double inv = 1.0 / sqrt(ss / (double)K + (double)eps);
             for (int64_t k = 0; k < K; ++k) {
-                float v = oracle_bf16_to_f32(h[k]) * inv;
-                if (g) v = v * oracle_bf16_to_f32(g[k]);
-                Y[m * K + k] = oracle_f32_to_bf16_rne(v);
+                double v = (double)oracle_bf16_to_f32(h[k]);
+                if (g) v = v * (double)oracle_bf16_to_f32(g[k]);
+                v = v * inv;
+                uint16_t a;
+                Y[m * K + k] = bf16_round_with_alt(v, 0x1p-34, &a);
+                if (Yalt) Yalt[m * K + k] = a;
             }
         }
         free(h);

@@ -1,10 +1,24 @@
 """Pins for the oracle's input activations (int8_linear(input_act=...),
 comfy-kitchen 0.2.40 "HIP backend": the activation is folded into the fused
 ConvRot quantiser's load). The pages do not list the activations; the ones
-built are relu, silu and the tanh form of gelu, each in fp32 on the widened
-bf16 input and rounded to bf16 before the rotation. The oracle's own e^x is
-checked against float64 exp; the activations against float64 formulas and
-torch's bf16 implementations; the wiring against torch's exact relu."""
+built are relu, silu x / (1 + e^-x) and the tanh form of gelu, each as the
+bf16 value nearest to the exact act(x) of the bf16 input, then rotated.
+
+What pins the oracle here, independently of it:
+  * its float64 -> bf16 rounding against exact rational arithmetic
+    (``fractions``), ties and subnormals included;
+  * its activation of every finite bf16 input (all 65,280 of them) against a
+    90-digit ``decimal`` evaluation of the formulas (pi from Machin's
+    formula), rounded to bf16 with exact rationals; that evaluation also
+    shows every input's exact value lies far from a rounding midpoint, so the
+    bf16 result is unique;
+  * relu against torch's, silu and gelu against torch's fp32-based bf16
+    implementations (within one bf16 ulp), and the quantiser's wiring.
+"""
+from decimal import Decimal, localcontext
+from fractions import Fraction
+import struct
+
 import numpy as np
 import pytest
 import torch
@@ -12,74 +26,168 @@ import torch
 import oracle
 import workloads
 
-
-def ulps32(a, b):
-    a = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
-    b = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
-    a = np.where(a < 0, np.int64(-2 ** 31) - a, a)
-    b = np.where(b < 0, np.int64(-2 ** 31) - b, b)
-    return np.abs(a - b)
+PREC = 90
+GELU_C = Decimal("0.044715")
 
 
-def test_exp_matches_float64_within_4_ulp():
-    x = np.concatenate([np.linspace(-87.0, 88.5, 40001, dtype=np.float32),
-                        np.float32([0.0, -0.0, 1e-30, -1e-30, 0.34657359, -0.34657359])])
-    got = oracle.exp(x)
-    ref = np.exp(x.astype(np.float64)).astype(np.float32)
-    assert ulps32(got, ref).max() <= 4
+def _bits_to_float(b: int) -> float:
+    return struct.unpack("<f", struct.pack("<I", (int(b) & 0xFFFF) << 16))[0]
 
 
-def test_exp_special_values():
-    x = np.float32([-200.0, -104.5, 89.0, 200.0, 0.0, 1.0])
-    got = oracle.exp(x)
-    assert got[0] == 0.0 and got[1] == 0.0
-    assert np.isinf(got[2]) and np.isinf(got[3])
-    assert got[4] == 1.0
-    assert ulps32(got[5], np.float32(np.e)) <= 1
+def _float_to_bits(f: float) -> int:
+    return struct.unpack("<I", struct.pack("<f", f))[0] >> 16
 
 
-def test_exp_subnormal_range_absolute_error():
-    x = np.linspace(-103.9, -87.4, 2001, dtype=np.float32)
-    got = oracle.exp(x).astype(np.float64)
-    ref = np.exp(x.astype(np.float64))
-    assert np.all(np.abs(got - ref) <= 2.0 ** -149 * 2 + ref * 2.0 ** -22)
+def _exact_bf16(v: Fraction) -> tuple[int, Fraction]:
+    """Round an exact rational to bf16 (ties to even). Returns the bits and
+    the distance of v from the nearest rounding midpoint, in units of the
+    local spacing (0.5 means v sits on a representable value)."""
+    neg = v < 0
+    a = -v if neg else v
+    sign = 0x8000 if neg else 0
+    if a == 0:
+        return sign, Fraction(1, 2)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    # 2^(e-1) <= a < 2^e after the adjustment below
+    while Fraction(2) ** e <= a:
+        e += 1
+    while Fraction(2) ** (e - 1) > a:
+        e -= 1
+    qe = max(e - 8, -133)
+    n = a / Fraction(2) ** qe
+    lo = n.numerator // n.denominator
+    rem = n - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    r = Fraction(lo) * Fraction(2) ** qe
+    if r >= Fraction(2) ** 128:
+        return sign | 0x7F80, abs(rem - Fraction(1, 2))
+    return sign | _float_to_bits(float(r)), abs(rem - Fraction(1, 2))
 
 
-def _x():
-    rng = np.random.default_rng(3)
-    return np.concatenate([rng.standard_normal(20000).astype(np.float32) * 3,
-                           np.float32([0.0, -0.0, 50.0, -50.0, 100.0, -100.0, 1e-20, -1e-20])])
+# -------------------------------------------------------- float64 -> bf16
 
 
-def test_relu_exact():
-    x = _x()
-    assert np.array_equal(oracle.act("relu", x), np.maximum(x, np.float32(0)))
+def _some_doubles():
+    rng = np.random.default_rng(17)
+    vals = list(rng.standard_normal(300) * np.exp2(rng.integers(-140, 130, 300)))
+    for b in list(rng.integers(1, 0x7F7F, 200)) + [1, 2, 3, 0x7F, 0x80, 0x81, 0x7F7D, 0x7F7E]:
+        x, y = _bits_to_float(b), _bits_to_float(b + 1)
+        mid = (x + y) / 2  # exact in double
+        ulp = np.spacing(mid)
+        vals += [mid, mid + ulp, mid - ulp, x, -mid, -(mid + ulp)]
+    vals += [0.0, -0.0, 2.0 ** -150, 2.0 ** -134, 3 * 2.0 ** -134, 2.0 ** -134 + 2.0 ** -200,
+             3.3961775292304e38, 3.3961775292305e38, 3.40e38, 1e300, -1e300, 5e-324]
+    return vals
 
 
-def test_silu_matches_float64():
-    x = _x()
-    ref = (x.astype(np.float64) / (1.0 + np.exp(-x.astype(np.float64)))).astype(np.float32)
-    got = oracle.act("silu", x)
-    big = np.abs(ref) > 1e-30
-    assert ulps32(got[big], ref[big]).max() <= 8
-    assert got[-1] == ref[-1] or abs(got[-1]) < 1e-19
+def test_f64_to_bf16_is_exact_rounding():
+    vals = _some_doubles()
+    got = oracle.f64_to_bf16(np.array(vals, np.float64))
+    for v, g in zip(vals, got):
+        want, _ = _exact_bf16(Fraction(v))
+        if v == 0.0 and np.signbit(v):
+            want = 0x8000
+        assert int(g) == want, (v, hex(int(g)), hex(want))
 
 
-def test_gelu_tanh_matches_float64():
-    x = _x()
-    xd = x.astype(np.float64)
-    u = np.sqrt(2.0 / np.pi) * (xd + 0.044715 * xd ** 3)
-    # 0.5 x (1 + tanh(u)) written without the cancellation near tanh(u) = -1
-    with np.errstate(over="ignore"):  # e^(-2u) = inf for very negative x: ref -> -0
-        ref = xd / (1.0 + np.exp(-2.0 * u))
-    got = oracle.act("gelu_tanh", x).astype(np.float64)
-    # fp32 rounding of the argument 2u is amplified by e^(-2u): relative error
-    # grows with |2u| (conditioning, not the method)
-    assert np.all(np.abs(got - ref) <= np.abs(ref) * (2.0 ** -19 + np.abs(2 * u) * 2.0 ** -21) + 1e-37)
-    # and it is the tanh form: 0.5 x (1 + tanh(u)) where that is well conditioned
-    ok = xd > -3.0
-    tanh_form = 0.5 * xd * (1.0 + np.tanh(u))
-    assert np.all(np.abs(got[ok] - tanh_form[ok]) <= np.abs(tanh_form[ok]) * 2.0 ** -18 + 1e-30)
+def test_f64_to_bf16_does_not_round_twice():
+    # 1 + 2^-9 + 2^-30: fp32 would first round it to 1 + 2^-9 (a bf16 tie,
+    # which goes to even: 1.0); the value itself lies above the midpoint
+    v = 1.0 + 2.0 ** -9 + 2.0 ** -30
+    assert int(oracle.f64_to_bf16(np.array([v]))[0]) == _float_to_bits(1.0 + 2.0 ** -8)
+
+
+# -------------------------------------------------------- exact activations
+
+
+def _pi() -> Decimal:
+    """pi from Machin's formula 16 atan(1/5) - 4 atan(1/239)."""
+    def atan_inv(n):
+        x = Decimal(1) / n
+        x2 = x * x
+        term, total, k = x, x, 1
+        while True:
+            term *= -x2
+            t = term / (2 * k + 1)
+            if t == 0 or abs(t) < Decimal(10) ** (-PREC - 5):
+                break
+            total += t
+            k += 1
+        return total
+
+    return 16 * atan_inv(5) - 4 * atan_inv(239)
+
+
+def _exact_act(name: str, x: Decimal, sqrt2pi: Decimal) -> Decimal:
+    if name == "silu":
+        arg = -x
+    else:
+        u = sqrt2pi * (x + GELU_C * x * x * x)
+        arg = -2 * u
+    if arg > 100000:  # e^arg beyond any bf16 ratio: |act| < |x| e^-1e5
+        return Decimal(0) * x.copy_sign(1) if x != 0 else Decimal(0)
+    if arg < -100000:  # e^arg < e^-1e5: act(x) = x (1 - tiny)
+        return x * (1 - Decimal(10) ** -40000)
+    return x / (1 + arg.exp())
+
+
+def _all_finite_bf16():
+    b = np.arange(0x10000, dtype=np.uint32)
+    finite = (b & 0x7F80) != 0x7F80
+    return b[finite].astype(np.uint16)
+
+
+@pytest.mark.parametrize("name", ["silu", "gelu_tanh"])
+def test_every_bf16_input_matches_high_precision_evaluation(name):
+    xs = _all_finite_bf16()
+    got = oracle.act_bf16(name, xs)
+    worst = Fraction(1, 2)
+    with localcontext() as ctx:
+        ctx.prec = PREC
+        ctx.Emax = 10 ** 9
+        ctx.Emin = -10 ** 9
+        sqrt2pi = (Decimal(2) / _pi()).sqrt()
+        for xb, g in zip(xs.tolist(), got.tolist()):
+            x = Decimal(_bits_to_float(xb))
+            v = _exact_act(name, x, sqrt2pi)
+            want, dist = _exact_bf16(Fraction(v))
+            if v == 0:
+                want = 0x8000 if (xb & 0x8000) else 0
+            assert g == want or (g & 0x7FFF) == (want & 0x7FFF) == 0, (hex(xb), hex(g), hex(want))
+            worst = min(worst, dist)
+    # every exact value lies far (relative to the 90-digit evaluation error)
+    # from a rounding midpoint: the bf16 result is unique for every input
+    assert worst > Fraction(1, 10 ** 60), float(worst)
+
+
+def test_relu_every_input_equals_torch():
+    xs = _all_finite_bf16()
+    got = oracle.act_bf16("relu", xs)
+    ref = workloads.bf16_bits(torch.relu(workloads.from_bf16_bits(xs)))
+    same = (got == ref) | (((got & 0x7FFF) == 0) & ((ref & 0x7FFF) == 0))  # -0 vs +0
+    assert same.all()
+
+
+def test_tiny_inputs_round_up_from_half():
+    # act(x) - x/2 > 0 for x != 0 and far below the subnormal spacing, so an
+    # x/2 that is a midpoint rounds up: +min subnormal -> +min subnormal,
+    # -min subnormal -> -0, 3 * min -> 2 * min, -3 * min -> -1 * min
+    xs = np.array([0x0001, 0x8001, 0x0003, 0x8003, 0x0002, 0x8002], np.uint16)
+    want = np.array([0x0001, 0x8000, 0x0002, 0x8001, 0x0001, 0x8001], np.uint16)
+    for name in ("silu", "gelu_tanh"):
+        assert np.array_equal(oracle.act_bf16(name, xs), want), name
+
+
+def test_large_inputs_limits():
+    big = np.array([_float_to_bits(200.0), _float_to_bits(-200.0), 0x7F7F, 0xFF7F], np.uint16)
+    for name in ("silu", "gelu_tanh"):
+        got = oracle.act_bf16(name, big)
+        assert got[0] == big[0] and got[2] == big[2]  # act(x) = x (1 - tiny) -> x
+        assert got[1] in (0x8000,) and got[3] == 0x8000  # |act| far below the smallest subnormal
+    # silu(-90) = -90 e^-90 / (1 + e^-90) is a normal bf16 number, not 0
+    s = oracle.act_bf16("silu", np.array([_float_to_bits(-90.0)], np.uint16))[0]
+    assert abs(_bits_to_float(s) - (-90.0 * np.exp(-90.0))) <= 2.0 ** -8 * 90.0 * np.exp(-90.0)
 
 
 @pytest.mark.parametrize("name,fn", [
@@ -87,15 +195,24 @@ def test_gelu_tanh_matches_float64():
     ("gelu_tanh", lambda t: torch.nn.functional.gelu(t, approximate="tanh")),
 ])
 def test_bf16_activation_close_to_torch(name, fn):
-    # torch's tanh-form gelu underflows to 0 below about x = -5 (1 + tanh(u)
-    # cancels in fp32); compare where both are accurate
-    xs = _x()
+    # torch evaluates in fp32 and rounds; its tanh-form gelu cancels to 0
+    # below about x = -5, so compare where both are accurate
+    rng = np.random.default_rng(3)
+    xs = rng.standard_normal(20000).astype(np.float32) * 3
     x = torch.from_numpy(xs[xs > -4.0]).to(torch.bfloat16)
-    mine = oracle.f32_to_bf16(oracle.act(name, x.float().numpy()))
+    mine = oracle.act_bf16(name, workloads.bf16_bits(x))
     theirs = workloads.bf16_bits(fn(x.float()).to(torch.bfloat16))
     d = np.abs(mine.astype(np.int32) - theirs.astype(np.int32))
     assert (d <= 1).all()
     assert (d != 0).mean() < 0.01
+
+
+def test_act_f64_is_the_tanh_form():
+    x = np.linspace(-3.0, 6.0, 2001)
+    u = np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)
+    assert np.allclose(oracle.act_f64("gelu_tanh", x), 0.5 * x * (1.0 + np.tanh(u)),
+                       rtol=1e-13, atol=1e-300)
+    assert np.allclose(oracle.act_f64("silu", x), x / (1.0 + np.exp(-x)), rtol=1e-15, atol=0)
 
 
 def test_quantize_with_relu_equals_quantize_of_torch_relu():
@@ -110,7 +227,7 @@ def test_quantize_with_relu_equals_quantize_of_torch_relu():
 def test_quantize_with_act_equals_quantize_of_rounded_act(name):
     cfg = workloads.custom(5, 512, 8, seed=10)
     X, _, _ = workloads.make_inputs(cfg)
-    a_bits = oracle.f32_to_bf16(oracle.act(name, X.float().numpy()))
+    a_bits = oracle.act_bf16(name, workloads.bf16_bits(X))
     a = oracle.quantize_rows_bf16(workloads.bf16_bits(X), act=name)
     b = oracle.quantize_rows_bf16(a_bits)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

@@ -29,10 +29,13 @@ MUTATIONS = {
     "epilogue_bias_dropped": ("    f = f + b;\n", "    (void)b;\n"),
     "bf16_truncates": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (rest > 0x8000u || (rest == 0x8000u && (kept & 1u)))", "if (rest >= 0x8000u)"),
-    "gelu_cubic_coefficient": ("float inner = fmaf(0.044715f, x3, x);", "float inner = fmaf(0.04715f, x3, x);"),
-    "silu_wrong_sign": ("float e = oracle_exp(-x);", "float e = oracle_exp(x);"),
-    "exp_drops_a_term": ("p = fmaf(p, r, 1.6666667e-01f);", "p = fmaf(p, r, 0.0f);"),
-    "exp_reduction_head_only": ("r = fmaf(-n, ln2_lo, r);", "r = r - 0.0f;"),
+    "gelu_cubic_coefficient": ("(x + 0.044715 * (x * x * x))", "(x + 0.04715 * (x * x * x))"),
+    "gelu_drops_factor_two": ("return x / (1.0 + exp(-2.0 * u));", "return x / (1.0 + exp(-u));"),
+    "silu_wrong_sign": ("return x / (1.0 + exp(-x));", "return x / (1.0 + exp(x));"),
+    "act_tiny_ties_to_even": ("double q = (t - lo == 0.5) ? lo + 1.0 : nearbyint(t);",
+                              "double q = nearbyint(t);"),
+    "f64_bf16_truncates": ("double q = nearbyint(ldexp(a, -qe));", "double q = floor(ldexp(a, -qe));"),
+    "f64_bf16_no_subnormal_spacing": ("if (qe < -133)\n        qe = -133;", "(void)0;"),
     "int4_qmax_8": ("oracle_quant_row_q(buf, K, 7.0f, q, s_w + n);", "oracle_quant_row_q(buf, K, 8.0f, q, s_w + n);"),
     "int4_nibbles_swapped": ("(uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));",
                              "(uint8_t)(((uint8_t)q[2 * j + 1] & 0xFu) | (((uint8_t)q[2 * j] & 0xFu) << 4));"),
@@ -46,17 +49,18 @@ MUTATIONS = {
     "nvfp4_tensor_scale_constant": ("const float s_t = amax / 2688.0f;", "const float s_t = amax / 2682.0f;"),
     "nvfp4_block_amax_signed": ("                        if (fabsf(y[i]) > ab)\n                            ab = fabsf(y[i]);",
                                 "                        if (y[i] > ab)\n                            ab = y[i];"),
-    "act_not_rounded_to_bf16": ("v = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(oracle_act(act, v)));",
-                                "v = oracle_act(act, v);"),
-    "rmsnorm_eps_outside_sqrt": ("float inv = 1.0f / sqrtf(ss / (float)K + eps);",
-                                 "float inv = 1.0f / (sqrtf(ss / (float)K) + eps);"),
-    "rmsnorm_sum_not_mean": ("float inv = 1.0f / sqrtf(ss / (float)K + eps);",
-                             "float inv = 1.0f / sqrtf(ss + eps);"),
-    "rmsnorm_skips_a_partial": ("for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ mm];",
-                                "for (int l = 0; l < 32; ++l) q[l] = mm == 1 ? p[l] + p[l] : p[l] + p[l ^ mm];"),
-    "rmsnorm_weight_dropped": ("if (g) v = v * oracle_bf16_to_f32(g[k]);", "(void)g;"),
+    "act_not_rounded_to_bf16": ("buf[k] = oracle_bf16_to_f32(oracle_act_bf16(act, row[k]));",
+                                "buf[k] = (float)oracle_act_f64(act, oracle_bf16_to_f32(row[k]));"),
+    "rmsnorm_eps_outside_sqrt": ("double inv = 1.0 / sqrt(ss / (double)K + (double)eps);",
+                                 "double inv = 1.0 / (sqrt(ss / (double)K) + (double)eps);"),
+    "rmsnorm_sum_not_mean": ("double inv = 1.0 / sqrt(ss / (double)K + (double)eps);",
+                             "double inv = 1.0 / sqrt(ss + (double)eps);"),
+    "rmsnorm_drops_a_square": ("    for (int64_t k = 0; k < K; ++k) {\n        double v = (double)oracle_bf16_to_f32(h[k]);\n        double t = v * v;",
+                               "    for (int64_t k = 1; k < K; ++k) {\n        double v = (double)oracle_bf16_to_f32(h[k]);\n        double t = v * v;"),
+    "rmsnorm_weight_dropped": ("if (g) v = v * (double)oracle_bf16_to_f32(g[k]);", "(void)g;"),
     "rmsnorm_residual_subtracted": ("h[k] = R ? oracle_f32_to_bf16_rne(x + oracle_bf16_to_f32(R[m * ldr + k]))",
                                     "h[k] = R ? oracle_f32_to_bf16_rne(x - oracle_bf16_to_f32(R[m * ldr + k]))"),
+    "rmsnorm_no_alt_offered": ("        *alt = o;\n", "        (void)o;\n"),
 }
 
 
@@ -72,7 +76,7 @@ PIN_FILES = {
 
 
 def _pins_for(name: str):
-    if name.startswith(("gelu", "silu", "exp_", "act_")):
+    if name.startswith(("gelu", "silu", "act_", "f64_")):
         return PIN_FILES["act"]
     if name.startswith("int4"):
         return PIN_FILES["int4"]
