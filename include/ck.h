@@ -120,8 +120,8 @@ ck_status ck_quantize_rotate_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int
 ck_status ck_quantize_int8_rowwise(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Qx, float *s_x, ck_stream_t stream);
 
-/* Input activations for the *_act entry points (applied to the bf16 input in
- * fp32, rounded to bf16, then rotated and quantised). */
+/* Input activations for the *_act entry points (each bf16 input becomes the
+ * bf16 value nearest to the exact act(x), then is rotated and quantised). */
 typedef enum ck_act {
     CK_ACT_NONE = 0,
     CK_ACT_RELU = 1,      /* max(x, 0) */
@@ -133,12 +133,16 @@ typedef enum ck_act {
  * quantize_and_rotate_rowwise with an input activation (comfy-kitchen 0.2.40,
  * "HIP backend": int8_linear(input_act=...) folds the activation into the
  * fused ConvRot quantiser's load, so act(x) is never written to memory).
- * Each element becomes bf16_rne(act(float(x))) before ConvRot256; act is a
- * ck_act value (CK_ERR_INVALID_VALUE otherwise). The list of activations and
- * their formulas are a reading: the page names the argument only. e^x is the
- * library's own (Cody-Waite reduction + degree-7 Taylor polynomial, every
- * step one IEEE operation), accurate to a few ulp. Other arguments as for
- * ck_quantize_rotate_rowwise.
+ * Each element x becomes the bf16 value nearest to the exact act(x) (ties to
+ * even; no bf16 input's exact act(x) lies on or near a midpoint, except
+ * |x| < 2^-120, where act(x) is just above x/2 and x/2 rounds with ties
+ * going up) before ConvRot256; act is a ck_act value (CK_ERR_INVALID_VALUE
+ * otherwise). The list of activations and their formulas are a reading: the
+ * page names the argument only. The kernel evaluates act in fp32 (its own
+ * e^x: Cody-Waite reduction and a degree-7 Taylor polynomial) and redoes in
+ * double precision every value whose fp32 result lies near a bf16 rounding
+ * midpoint, so the stored bf16 values are those of the definition. Other
+ * arguments as for ck_quantize_rotate_rowwise.
  */
 ck_status ck_quantize_rotate_rowwise_act(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                          int act, int8_t *Qx, float *s_x, ck_stream_t stream);
@@ -209,15 +213,16 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
  * Input RMSNorm with a residual (comfy-kitchen 0.2.40, "Huawei Ascend backend":
  * int8_linear accepts the input RMSNorm and residual arguments and applies
  * them with shared helpers apart from its GEMM; the page prints no formula).
- * Reading, every step an IEEE fp32 operation:
- *   h   = bf16_rne(x + r), or h = x when residual is NULL;
+ * Reading:
+ *   h   = bf16_rne(fl32(x + r)) (a bf16 tensor addition), or h = x when
+ *         residual is NULL;
  *   residual_out = h (when residual_out is not NULL);
- *   ss  = sum over the row of h^2 in this order: 32 partial sums p_l, p_l
- *         taking, for i = 0, 1, ... and then j = 0..7, element 256 i + 8 l + j
- *         with one fused multiply-add each; then p_l = p_l + p_(l xor m) for
- *         m = 16, 8, 4, 2, 1;
- *   inv = 1 / sqrt(ss / K + eps);
- *   Y   = bf16_rne((h * inv) * g), or bf16_rne(h * inv) when g is NULL.
+ *   Y_k = the bf16 value nearest to h_k g_k / sqrt(mean_k(h_k^2) + eps) (the
+ *         exact real value; g_k = 1 when g is NULL), ties to even.
+ * The kernel sums the squares and forms Y in double precision (each h^2 and
+ * h g exact), so Y is that rounding except where the exact value lies within
+ * about 2^-36 (relative) of a bf16 rounding midpoint, where the summation
+ * order can decide the neighbour.
  *   X            [M, K] bf16, row stride ldx (>= K, % 8 == 0), 16-B aligned.
  *   residual     [M, K] bf16, row stride ldr, or NULL.
  *   residual_out [M, K] bf16, row stride ldo, or NULL (output); it may alias
@@ -390,7 +395,7 @@ ck_status ck_convrot_nvfp4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *
 
 /* Size of the device array that ck_int8_linear_noalloc uses as its
  * workspace: 32 MiB, enough for ck_int8_linear_workspace_bytes(M, K) of e.g.
- * M = 4096, K = 8000 or M = 1024, K = 32512. */
+ * M = 4096, K = 7936 or M = 1024, K = 32512. */
 #define CK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /*
@@ -409,7 +414,11 @@ ck_status ck_convrot_nvfp4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *
  * it reads, so nothing needs clearing), so calls whose work overlaps on the
  * GPU race and give wrong results: order them. The first call on a device
  * looks up the array's device address with that device current; make that
- * first call before any stream capture. Allocates nothing.
+ * first call before any stream capture (the lookup is repeated after the
+ * device's context changes, e.g. after cudaDeviceReset). Argument checks and
+ * their order are ck_int8_linear's (CK_ERR_INVALID_VALUE, then
+ * CK_ERR_UNSUPPORTED_SHAPE, then CK_ERR_MISALIGNED), then the size check,
+ * then CK_ERR_ARCH. Allocates nothing.
  */
 ck_status ck_int8_linear_noalloc(const ck_bf16 *X, int64_t ldx, const int8_t *Qw, const float *s_w,
                                  const ck_bf16 *bias, ck_bf16 *Y, int64_t M, int64_t N, int64_t K,
@@ -442,6 +451,15 @@ ck_status ck_test_int8_gemm_i32(const int8_t *Qx, const int8_t *Qw, int32_t *acc
 /* Same as ck_quantize_int8_rowwise (the quantiser without the rotation). */
 ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                             int8_t *Qx, float *s_x, ck_stream_t stream);
+
+/*
+ * The input activation alone, exactly as the quantiser applies it before the
+ * rotation (same device code), on n bf16 values:
+ *   X [n] bf16 (input), Y [n] bf16 (output), both 16-B aligned; n % 256 == 0;
+ *   act a ck_act value.
+ * Lets the tests compare every possible bf16 input with the definition.
+ */
+ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck_stream_t stream);
 
 /*
  * Fault injection for the bounded waits, host side only: with mode 1 the next

@@ -93,6 +93,7 @@ _SIGS = {
     "ck_test_int8_gemm_i32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_test_quantize_rowwise_norotate": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_test_inject_producer_stall": (_st, [ctypes.c_int, _i64]),
+    "ck_test_input_act": (_st, [_vp, _i64, _st, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -375,6 +376,7 @@ def int8_linear_noalloc(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
     should be passed by such callers (otherwise this wrapper allocates it)."""
     _need(X, "X", torch.bfloat16, 2)
     _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
     _need(s_w, "s_w", torch.float32, 1)
     if bias is not None:
         _need(bias, "bias", torch.bfloat16, 1)
@@ -386,9 +388,14 @@ def int8_linear_noalloc(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     _need(out, "out", torch.bfloat16, 2)
     _rows_contiguous(out, "out")
+    for t, name in ((Qw, "Qw"), (s_w, "s_w"), (bias, "bias"), (out, "out")):
+        if t is not None and t.device != X.device:
+            raise ValueError(f"{name} is on {t.device}, X on {X.device}")
     ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
-    _check(lib.ck_int8_linear_noalloc(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias), _ptr(out),
-                                      M, N, K, _stream(stream)), "ck_int8_linear_noalloc")
+    with torch.cuda.device(X.device):
+        _check(lib.ck_int8_linear_noalloc(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias),
+                                          _ptr(out), M, N, K, _stream(stream)),
+               "ck_int8_linear_noalloc")
     return out
 
 
@@ -536,6 +543,22 @@ def test_int8_gemm_i32(Qx: torch.Tensor, Qw: torch.Tensor, out: torch.Tensor | N
 
 
 test_int8_gemm_i32.__test__ = False
+
+
+def test_input_act(X: torch.Tensor, act: str, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """The input activation alone, as the quantiser applies it (test hook):
+    X contiguous bf16 with numel % 256 == 0."""
+    if X.dtype != torch.bfloat16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA bf16 tensor")
+    if out is None:
+        out = torch.empty_like(X)
+    _check(lib.ck_test_input_act(_ptr(X), X.numel(), ACTS[act], _ptr(out), _stream(stream)),
+           "ck_test_input_act")
+    return out
+
+
+test_input_act.__test__ = False
 
 
 def device_error() -> int:

@@ -27,11 +27,14 @@ struct DeviceState {
     bool arch_ok = false;
     int num_sms = 0;
     unsigned *err = nullptr;
+    CUcontext ctx = nullptr;  // the context the cached addresses belong to
+    unsigned generation = 0;  // bumped whenever the state is rebuilt
 };
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_get = nullptr;
 
 thread_local int t_stall_next = 0;
 thread_local int64_t t_stall_limit_ns = 0;
@@ -45,15 +48,45 @@ ck_status check_k(int64_t K) {
     return CK_OK;
 }
 
-// Returns the state of the current device, initialising it once (arch check,
-// SM count, address of the error word, tensor-map encoder).
+// The context current on this thread, created by the runtime if there is
+// none yet (cudaSetDevice initialises the device's primary context).
+ck_status current_context(int dev, CUcontext *ctx) {
+    if (!g_ctx_get) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return CK_ERR_CUDA;
+        g_ctx_get = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    }
+    *ctx = nullptr;
+    if (g_ctx_get(ctx) != CUDA_SUCCESS) return CK_ERR_CUDA;
+    if (*ctx == nullptr) {
+        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_get(ctx) != CUDA_SUCCESS || !*ctx)
+            return CK_ERR_CUDA;
+    }
+    return CK_OK;
+}
+
+// Returns the state of the current device, initialising it once per context
+// (arch check, SM count, address of the error word, tensor-map encoder). A
+// new context on the device (after cudaDeviceReset, or a different context
+// made current) rebuilds it: the cached addresses belonged to the old one.
 ck_status device_state(DeviceState **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return CK_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mutex);
+    CUcontext ctx = nullptr;
+    if (current_context(dev, &ctx) != CK_OK) return CK_ERR_CUDA;
     DeviceState &st = g_dev[dev];
+    if (st.ready && st.ctx != ctx) {
+        st.ready = false;
+        st.err = nullptr;
+    }
     if (!st.ready) {
+        st.ctx = ctx;
+        ++st.generation;
         int major = 0, minor = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -216,9 +249,12 @@ ck_status weight_common(const float *W, int64_t N, int64_t K, void *Qw, float *s
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
-// Streams and events of ck_int8_linear_host, created once per device.
+// Streams and events of ck_int8_linear_host, created once per device
+// context (a new context, e.g. after cudaDeviceReset, gets new ones; the old
+// handles died with their context).
 struct HostPipe {
     bool ready = false;
+    unsigned generation = 0;
     cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
     cudaEvent_t entry = nullptr, done = nullptr;
     cudaEvent_t in_done[2] = {}, x_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
@@ -226,12 +262,14 @@ struct HostPipe {
 };
 HostPipe g_pipe[kMaxDevices];
 
-ck_status host_pipe(HostPipe **out) {
+ck_status host_pipe(const DeviceState *st, HostPipe **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mutex);
     HostPipe &hp = g_pipe[dev];
+    if (hp.ready && hp.generation != st->generation) hp.ready = false;
     if (!hp.ready) {
+        hp.generation = st->generation;
         const unsigned ef = cudaEventDisableTiming;
         bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
                   cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
@@ -251,6 +289,38 @@ ck_status host_pipe(HostPipe **out) {
 }
 
 }  // namespace
+
+namespace ck {
+
+ck_status check_linear_args(const void *X, int64_t ldx, const void *Qw, const void *s_w,
+                            const void *bias, const void *Y, int64_t M, int64_t N, int64_t K,
+                            const void *workspace, bool with_workspace) {
+    if (M < 0 || N < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (ldx < K) return CK_ERR_INVALID_VALUE;
+    if (M > 0 && N > 0 && (!X || !Qw || !s_w || !Y || (with_workspace && !workspace)))
+        return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return CK_OK;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Qw) || !aligned16(s_w) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) ||
+        (with_workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return CK_ERR_MISALIGNED;
+    return CK_OK;
+}
+
+ck_status check_current_device(unsigned *generation) {
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    *generation = st->generation;
+    return CK_OK;
+}
+
+}  // namespace ck
 
 extern "C" {
 
@@ -351,18 +421,9 @@ ck_status ck_int8_linear_act(const ck_bf16 *X, int64_t ldx, int act, const int8_
                              const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
                              int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                              ck_stream_t stream) {
-    if (M < 0 || N < 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
-    ck_status s = check_k(K);
-    if (s == CK_ERR_INVALID_VALUE) return s;
-    if (ldx < K) return CK_ERR_INVALID_VALUE;
-    if (M > 0 && N > 0 && (!X || !Qw || !s_w || !Y || !workspace)) return CK_ERR_INVALID_VALUE;
-    if (s != CK_OK) return s;
-    if (N % 8 != 0 || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
-        return CK_ERR_UNSUPPORTED_SHAPE;
-    if (M == 0 || N == 0) return CK_OK;
-    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(Qw) || !aligned16(s_w) || !aligned16(Y) ||
-        (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return CK_ERR_MISALIGNED;
+    if (act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
+    ck_status s = ck::check_linear_args(X, ldx, Qw, s_w, bias, Y, M, N, K, workspace, true);
+    if (s != CK_OK || M == 0 || N == 0) return s;
     if (workspace_bytes < ck_int8_linear_workspace_bytes(M, K)) return CK_ERR_WORKSPACE;
     DeviceState *st = nullptr;
     s = device_state(&st);
@@ -490,7 +551,7 @@ ck_status ck_int8_linear_host(const ck_bf16 *X_host, int64_t ldx, int act, const
     s = device_state(&st);
     if (s != CK_OK) return s;
     HostPipe *hp = nullptr;
-    s = host_pipe(&hp);
+    s = host_pipe(st, &hp);
     if (s != CK_OK) return s;
     std::lock_guard<std::mutex> lock(hp->m);
 
@@ -793,6 +854,19 @@ ck_status ck_test_int8_gemm_i32(const int8_t *Qx, const int8_t *Qw, int32_t *acc
     if (s != CK_OK) return s;
     return run_gemm(Qx, nullptr, Qw, nullptr, nullptr, nullptr, acc, M, N, K, st,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck_stream_t stream) {
+    if (n < 0 || act < CK_ACT_NONE || act > CK_ACT_GELU_TANH) return CK_ERR_INVALID_VALUE;
+    if (n > 0 && (!X || !Y)) return CK_ERR_INVALID_VALUE;
+    if (n % 256 != 0) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (n == 0) return CK_OK;
+    if (!aligned16(X) || !aligned16(Y)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_test_input_act(X, n, act, Y, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
 const char *ck_status_string(ck_status status) {

@@ -5,7 +5,22 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "ck.h"
+
 namespace ck {
+
+// ---- host-side checks shared by the entry points (api.cu)
+
+// ck_int8_linear's argument checks before its workspace size check, in its
+// order (CK_ERR_INVALID_VALUE, CK_ERR_UNSUPPORTED_SHAPE, CK_ERR_MISALIGNED);
+// with_workspace = false leaves the workspace pointer out.
+ck_status check_linear_args(const void *X, int64_t ldx, const void *Qw, const void *s_w,
+                            const void *bias, const void *Y, int64_t M, int64_t N, int64_t K,
+                            const void *workspace, bool with_workspace);
+// CK_OK on a B200 (compute capability 10.0) current device, else CK_ERR_ARCH or
+// CK_ERR_CUDA; *generation changes whenever the device's context changed
+// (e.g. after cudaDeviceReset), so per-context caches know to refresh.
+ck_status check_current_device(unsigned *generation);
 
 // ---- fused ConvRot256 + per-row INT8 quantiser (quant_rotate.cu)
 
@@ -17,6 +32,11 @@ namespace ck {
 cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                    bool rotate, int act, int qmax, int8_t *Q, float *S,
                                    unsigned *err, int num_sms, cudaStream_t stream);
+
+// Test hook: the input activation of n bf16 values (n % 256 == 0) as the
+// staged quantiser applies it (0 none, 1 relu, 2 silu, 3 tanh-form gelu).
+cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,
+                                  cudaStream_t stream);
 
 // Rows of fp32 with row stride K (offline weight preparation), always rotated;
 // int4_packed: signed INT4 codes packed two per byte into Q [N, K/2].

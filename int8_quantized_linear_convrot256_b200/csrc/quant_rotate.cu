@@ -101,14 +101,28 @@ __device__ __forceinline__ float2 widen_bf16x2(uint32_t w) {
 }
 
 // ------------------------------------------------------------------ input_act
-// int8_linear(input_act=...) (comfy-kitchen 0.2.40, "HIP backend"): the
-// activation is applied to the widened bf16 input, in fp32, and rounded to
-// bf16 before the rotation. relu; silu x / (1 + e^-x); gelu (tanh form)
+// int8_linear(input_act=...) (comfy-kitchen 0.2.40, "HIP backend"): each bf16
+// input x becomes the bf16 value nearest to the exact act(x) (ties to even)
+// before the rotation. relu; silu x / (1 + e^-x); gelu (tanh form)
 // 0.5 x (1 + tanh(u)) = x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3).
-// e^x: Cody-Waite reduction x = n ln2 + r (ln2 = 16-bit head + tail),
-// degree-7 Taylor polynomial of e^r in Horner form, exact scaling by 2^n;
-// every step is one IEEE operation (fused multiply-adds where the definition
-// has them), so CPU and GPU agree bit for bit.
+//
+// Fast path, fp32: e^v by Cody-Waite reduction v = n ln2 + r (ln2 = 16-bit
+// head + tail) and a degree-7 Taylor polynomial of e^r (truncation below
+// 2^-27), a reciprocal approximation of the denominator and one product. Its
+// result q is within E fp32 ulps of the exact value, E = 4 for silu (its
+// exponent argument -x is exact) and E = 4 + 3.5 |v| for gelu (the fp32
+// rounding of v = -2u, a few ulps, is amplified by e^v when e^v is not
+// negligible against 1). The bf16 rounding of q is the exact value's unless
+// q lies within E ulps of a bf16 rounding midpoint (its low 16 bits near
+// 0x8000); those values (a window of W = 8 + 4 |v| ulps is flagged, |v| taken
+// as 0 where e^v < 2^-20), and denominators above 1e36, are redone in double
+// precision and rounded to bf16 from the double value directly. The double
+// result differs from the exact value by a few 2^-52 relative, far less than
+// its distance from any midpoint for every bf16 input (the whole input set,
+// 65,280 finite values, is checked against the CPU oracle).
+// For |x| < 2^-120 the double evaluation gives x/2 exactly, which can sit on
+// a midpoint between bf16 subnormals while the exact value lies just above
+// x/2; there x/2 is rounded with ties going up.
 constexpr int kActNone = 0;
 constexpr int kActRelu = 1;
 constexpr int kActSilu = 2;
@@ -119,10 +133,8 @@ constexpr int kActGeluTanh = 3;
 // the sum's bits; r = x - n ln2 (two fused steps, 16-bit head + tail);
 // degree-7 Taylor polynomial of e^r by fused Horner steps (packed
 // fma.f32x2); then p * 2^k as (p * 2^a) * 2^b with a = floor(k/2),
-// b = ceil(k/2): p * 2^a is exact and normal (p >= 0.7, a >= -75), so the
-// result is p * 2^k rounded once, as the definition's scaling gives for every
-// k in range. Outside [-104, 88.8] the definition's limits (0, +inf) are
-// selected.
+// b = ceil(k/2): p * 2^a is exact and normal (p >= 0.7, a >= -75). Outside
+// [-104, 88.8] the limits 0 and +inf are selected.
 __device__ __forceinline__ float2 act_exp2(float2 x) {
     const float kRound = 12582912.0f;  // 1.5 * 2^23
     const float2 m = __fadd2_rn(__fmul2_rn(x, make_float2(1.442695f, 1.442695f)),
@@ -154,24 +166,23 @@ __device__ __forceinline__ float2 act_exp2(float2 x) {
     return e;
 }
 
-// x / d where only bf16_rne of the quotient is used: a reciprocal
-// approximation (error <= 1 ulp) times x is within 2 fp32 ulps of the
-// correctly rounded quotient, so its bf16 rounding is the same unless it
-// lies within a few ulps of a bf16 rounding midpoint (the low 16 bits near
-// 0x8000) or d is huge; `exact` is set for those, and the caller then redoes
-// the value with the IEEE division.
-__device__ __forceinline__ float div_for_bf16(float x, float d, bool &exact) {
+// x / d where only the bf16 rounding of the quotient is used: a reciprocal
+// approximation times x. `redo` is raised when the result lies within w fp32
+// ulps of a bf16 rounding midpoint, or d is huge (the reciprocal would leave
+// the normal range).
+__device__ __forceinline__ float div_for_bf16(float x, float d, uint32_t w, bool &redo) {
     float r;
     asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(d));
     const float q = __fmul_rn(x, r);
     const uint32_t lo = __float_as_uint(q) & 0xFFFFu;
-    exact = exact || (lo - 0x7FF8u <= 16u) || (d > 1.0e36f);
+    redo = redo || (lo - (0x8000u - w) <= 2u * w) || (d > 1.0e36f);
     return q;
 }
 
-// Denominator 1 + e^v of silu (v = -x) and of the tanh-form gelu (v = -2u).
+// Denominators 1 + e^v of silu (v = -x) and of the tanh-form gelu (v = -2u),
+// and the flag window of each value in fp32 ulps.
 template <int kAct>
-__device__ __forceinline__ float2 act_denominator(float2 x) {
+__device__ __forceinline__ float2 act_denominator(float2 x, uint32_t &wx, uint32_t &wy) {
     float2 v;
     if (kAct == kActSilu) {
         v = make_float2(-x.x, -x.y);
@@ -181,40 +192,70 @@ __device__ __forceinline__ float2 act_denominator(float2 x) {
         const float2 u = __fmul2_rn(make_float2(7.978846e-01f, 7.978846e-01f), inner);
         v = __fmul2_rn(make_float2(-2.0f, -2.0f), u);
     }
-    return __fadd2_rn(make_float2(1.0f, 1.0f), act_exp2(v));
+    const float2 e = act_exp2(v);
+    if (kAct == kActSilu) {
+        wx = wy = 8u;
+    } else {
+        // |v| <= 83 wherever e^v is in [2^-20, 1e36]; outside that the value
+        // is flagged anyway (d > 1e36) or the amplified error is negligible
+        const float kTiny = 9.5367431640625e-07f;  // 2^-20
+        wx = 8u + (e.x >= kTiny && e.x <= 1.0e36f ? uint32_t(4.0f * fabsf(v.x)) : 0u);
+        wy = 8u + (e.y >= kTiny && e.y <= 1.0e36f ? uint32_t(4.0f * fabsf(v.y)) : 0u);
+    }
+    return __fadd2_rn(make_float2(1.0f, 1.0f), e);
 }
 
 // bf16x2 word -> activation of both values -> bf16x2 word (round to nearest
-// even). `exact` is raised when a quotient needs the IEEE division; then
+// even). `redo` is raised when a value needs the double-precision path; then
 // act_bf16x2_exact gives the word.
 template <int kAct>
-__device__ __forceinline__ uint32_t act_bf16x2(uint32_t w, bool &exact) {
+__device__ __forceinline__ uint32_t act_bf16x2(uint32_t w, bool &redo) {
     if (kAct == kActNone) return w;
     const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
     float2 a;
     if (kAct == kActRelu) {
         a = make_float2(x.x > 0.0f ? x.x : 0.0f, x.y > 0.0f ? x.y : 0.0f);
     } else {
-        const float2 d = act_denominator<kAct>(x);
-        a = make_float2(div_for_bf16(x.x, d.x, exact), div_for_bf16(x.y, d.y, exact));
+        uint32_t wx, wy;
+        const float2 d = act_denominator<kAct>(x, wx, wy);
+        a = make_float2(div_for_bf16(x.x, d.x, wx, redo), div_for_bf16(x.y, d.y, wy, redo));
     }
     const __nv_bfloat162 h = __floats2bfloat162_rn(a.x, a.y);
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// One value in double precision, rounded once to bf16 (the bits).
+template <int kAct>
+__device__ __forceinline__ uint32_t act_bf16_double(float xf) {
+    const double x = xf;
+    double v;
+    if (x != 0.0 && fabs(x) < 7.52316384526264e-37) {  // |x| < 2^-120
+        // x/2 in units of the bf16 subnormal spacing 2^-133; a tie goes up
+        const double t = x * 5.444517870735016e+39;  // 2^132
+        const double lo = floor(t);
+        const double q = (t - lo == 0.5) ? lo + 1.0 : rint(t);
+        v = copysign(q * 9.183549615799121e-41, x);  // q * 2^-133
+    } else if (kAct == kActSilu) {
+        v = x / (1.0 + exp(-x));
+    } else {
+        const double u = 0.7978845608028654 * (x + 0.044715 * (x * x * x));  // sqrt(2/pi)
+        v = x / (1.0 + exp(-2.0 * u));
+    }
+    const __nv_bfloat16 h = __double2bfloat16(v);
+    return *reinterpret_cast<const uint16_t *>(&h);
+}
+
 template <int kAct>
 __device__ __noinline__ uint32_t act_bf16x2_exact(uint32_t w) {
-    const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-    const float2 d = act_denominator<kAct>(x);
-    const __nv_bfloat162 h = __floats2bfloat162_rn(__fdiv_rn(x.x, d.x), __fdiv_rn(x.y, d.y));
-    return *reinterpret_cast<const uint32_t *>(&h);
+    return act_bf16_double<kAct>(__uint_as_float(w << 16)) |
+           (act_bf16_double<kAct>(__uint_as_float(w & 0xFFFF0000u)) << 16);
 }
 
 template <int kAct>
 __device__ __forceinline__ uint32_t act_bf16x2(uint32_t w) {
-    bool exact = false;
-    const uint32_t r = act_bf16x2<kAct>(w, exact);
-    return exact ? act_bf16x2_exact<kAct>(w) : r;
+    bool redo = false;
+    const uint32_t r = act_bf16x2<kAct>(w, redo);
+    return redo ? act_bf16x2_exact<kAct>(w) : r;
 }
 
 // Lane t's 64 values of one block; base points at element 8t of the block.
@@ -282,6 +323,25 @@ __device__ __forceinline__ void act_in_smem(uint32_t saddr) {
                      "r"(ay), "r"(az), "r"(aw)
                      : "memory");
     }
+}
+
+// Test hook: the input activation exactly as the staged quantiser applies it
+// (act_in_smem on each quad's 512-byte block of 256 values), on whole 16-byte
+// chunks; 8192 values per CTA of 128 threads.
+template <int kAct>
+__global__ void __launch_bounds__(128)
+input_act_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Y, int64_t n16) {
+    __shared__ __align__(16) uint4 buf[1024];
+    const int t = threadIdx.x;
+    const int64_t base = int64_t(blockIdx.x) * 1024;
+    for (int i = t; i < 1024; i += 128)
+        buf[i] = base + i < n16 ? X[base + i] : make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    // lane l of quad q: chunks 32 q + l + 4 i (i = 0..7), 64 bytes apart
+    act_in_smem<kAct>(smem_u32(&buf[32 * (t >> 2) + (t & 3)]));
+    __syncthreads();
+    for (int i = t; i < 1024; i += 128)
+        if (base + i < n16) Y[base + i] = buf[i];
 }
 
 // Shared-memory loads of lane t's 64 staged values (the block's bf16 at
@@ -1252,6 +1312,24 @@ cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int6
             return launch_bf16<true, kActGeluTanh>(X, M, K, ldx, Q, S, err, num_sms, stream);
         default: return launch_bf16<true, kActNone>(X, M, K, ldx, Q, S, err, num_sms, stream);
     }
+}
+
+cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,
+                                  cudaStream_t stream) {
+    const int64_t n16 = n / 8;  // n % 256 == 0: whole 16-byte chunks
+    if (n16 <= 0) return cudaSuccess;
+    const unsigned grid = unsigned((n16 + 1023) / 1024);
+    const uint4 *x = reinterpret_cast<const uint4 *>(X);
+    uint4 *y = reinterpret_cast<uint4 *>(Y);
+    switch (act) {
+        case kActRelu: input_act_kernel<kActRelu><<<grid, 128, 0, stream>>>(x, y, n16); break;
+        case kActSilu: input_act_kernel<kActSilu><<<grid, 128, 0, stream>>>(x, y, n16); break;
+        case kActGeluTanh:
+            input_act_kernel<kActGeluTanh><<<grid, 128, 0, stream>>>(x, y, n16);
+            break;
+        default: input_act_kernel<kActNone><<<grid, 128, 0, stream>>>(x, y, n16); break;
+    }
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_rows_f32(const float *W, int64_t N, int64_t K, bool int4_packed,

@@ -1,14 +1,16 @@
 // Input RMSNorm with a residual, before the ConvRot quantiser
 // (comfy-kitchen 0.2.40, "Huawei Ascend backend": int8_linear accepts the input
 // RMSNorm and residual arguments and applies them with shared helpers, apart
-// from its GEMM; no formula is printed). Reading, every step an IEEE fp32
-// operation:
-//   h   = bf16_rne(x + r)          (h = x without a residual); Rout = h
-//   ss  = sum of h^2 in a fixed order: lane l of the row's warp takes, for
-//         i = 0, 1, ... and j = 0..7, element 256 i + 8 l + j with one fused
-//         multiply-add each; then five butterfly levels xor 16, 8, 4, 2, 1
-//   inv = 1 / sqrt(ss / K + eps)
-//   y   = bf16_rne((h * inv) * g)  (bf16_rne(h * inv) without g)
+// from its GEMM; no formula is printed). Reading:
+//   h   = bf16_rne(fl32(x + r))  (h = x without a residual); Rout = h
+//   y_k = the bf16 value nearest to h_k g_k / sqrt(mean(h^2) + eps), the
+//         exact real value (g_k = 1 without g)
+// Evaluated in double precision: every h^2 and h g is exact in double; the
+// sum of squares (each lane's share in index order, then a five-level xor
+// butterfly), one division, one square root and one product per value carry
+// a relative error below K 2^-53 + 2^-51, and cvt.rn.bf16.f64 rounds the
+// double result once. So y is the exact value's rounding except within about
+// 2^-36 (relative) of a bf16 rounding midpoint.
 // Memory-bound: one warp per row, 16-byte loads and stores, two passes over
 // the row (the second re-reads it from L2, or reads back Rout).
 #include <cstdint>
@@ -28,6 +30,13 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Two doubles rounded once each to bf16 (cvt.rn.bf16.f64), packed low first.
+__device__ __forceinline__ uint32_t pack_bf16x2_d(double lo, double hi) {
+    const __nv_bfloat16 a = __double2bfloat16(lo), b = __double2bfloat16(hi);
+    return uint32_t(*reinterpret_cast<const uint16_t *>(&a)) |
+           (uint32_t(*reinterpret_cast<const uint16_t *>(&b)) << 16);
 }
 
 __device__ __forceinline__ uint4 ld16_nc(const uint16_t *p) {
@@ -71,7 +80,7 @@ rmsnorm_rows_kernel(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t l
     uint16_t *y = Y + row * int64_t(K);
 
     // pass 1: h (stored to Rout), the lane's partial sum of squares
-    float p = 0.0f;
+    double p = 0.0;
     for (int i = 0; i < nb; ++i) {
         const int c = 256 * i + 8 * lane;
         uint32_t h[4];
@@ -79,15 +88,14 @@ rmsnorm_rows_kernel(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t l
         if (ro) *reinterpret_cast<uint4 *>(ro + c) = make_uint4(h[0], h[1], h[2], h[3]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float lo = bf16_lo(h[q]), hi = bf16_hi(h[q]);
-            p = __fmaf_rn(lo, lo, p);
-            p = __fmaf_rn(hi, hi, p);
+            const double lo = bf16_lo(h[q]), hi = bf16_hi(h[q]);
+            p = __fma_rn(lo, lo, p);
+            p = __fma_rn(hi, hi, p);
         }
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xFFFFFFFFu, p, m));
-    const float inv =
-        __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(p, static_cast<float>(K)), eps)));
+    for (int m = 16; m >= 1; m >>= 1) p = __dadd_rn(p, __shfl_xor_sync(0xFFFFFFFFu, p, m));
+    const double inv = 1.0 / sqrt(p / double(K) + double(eps));
 
     // pass 2: y
     for (int i = 0; i < nb; ++i) {
@@ -102,13 +110,10 @@ rmsnorm_rows_kernel(const uint16_t *X, int64_t ldx, const uint16_t *R, int64_t l
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            float lo = __fmul_rn(bf16_lo(h[q]), inv);
-            float hi = __fmul_rn(bf16_hi(h[q]), inv);
-            if (g) {
-                lo = __fmul_rn(lo, bf16_lo(gw[q]));
-                hi = __fmul_rn(hi, bf16_hi(gw[q]));
-            }
-            o[q] = pack_bf16x2(lo, hi);
+            // h g is exact in double; one rounding for the product with inv
+            const double lo = __dmul_rn(double(bf16_lo(h[q])) * double(bf16_lo(gw[q])), inv);
+            const double hi = __dmul_rn(double(bf16_hi(h[q])) * double(bf16_hi(gw[q])), inv);
+            o[q] = pack_bf16x2_d(lo, hi);
         }
         *reinterpret_cast<uint4 *>(y + c) = make_uint4(o[0], o[1], o[2], o[3]);
     }

@@ -1,7 +1,11 @@
 """Input RMSNorm with a residual on the GPU against the CPU oracle (through the C ABI).
 
-The normalised rows, the residual output, the codes and the row scales are
-compared bit for bit; linear outputs within 1 bf16 ulp (0 expected).
+Bar: the residual output bit for bit; each normalised value equal to the
+oracle's bf16 rounding of the exact value, or, where that value lies within
+2^-34 (relative) of a rounding midpoint, to either neighbour (the oracle's
+Yalt); the codes and row scales of the normalised rows equal the oracle's
+for some admissible choice there (the rest: bit for bit); linear outputs
+within 1 bf16 ulp.
 Source: comfy-kitchen 0.2.40, "Huawei Ascend backend" (int8_linear's input
 RMSNorm and residual arguments); the reading is stated in include/ck.h.
 """
@@ -11,6 +15,7 @@ import torch
 
 import oracle
 import workloads
+from parity_helpers import assert_bf16_close, assert_codes_admissible, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -39,39 +44,39 @@ def _inputs(M, K, seed, scale=1.0):
     return X, R, w
 
 
-def _ordered(bits):
-    b = bits.astype(np.int32)
-    return np.where(b & 0x8000, 0x8000 - b, b)
+def _assert_y(got, Yr, Ya):
+    ok = (got == Yr) | (got == Ya)
+    assert ok.all(), f"{(~ok).sum()} normalised values differ from both admissible roundings"
 
 
 @pytest.mark.parametrize("M,K", [(1, 256), (37, 768), (130, 5376), (9, 28672), (2, 132864)])
 @pytest.mark.parametrize("with_residual,with_g", [(True, True), (False, True), (True, False),
                                                   (False, False)])
-def test_rmsnorm_bit_exact(ck, M, K, with_residual, with_g):
+def test_rmsnorm_matches_oracle(ck, M, K, with_residual, with_g):
     X, R, w = _inputs(M, K, M + K)
     eps = 1e-5
     R = R if with_residual else None
     w = w if with_g else None
-    Yr, Hr = oracle.rmsnorm_rows(_bits(X), None if R is None else _bits(R),
-                                 None if w is None else _bits(w), eps)
+    Yr, Hr, Ya = oracle.rmsnorm_rows(_bits(X), None if R is None else _bits(R),
+                                     None if w is None else _bits(w), eps, with_alt=True)
     Ro = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     Y = ck.rmsnorm_residual(X.cuda(), None if R is None else R.cuda(),
                             None if w is None else w.cuda(), eps, residual_out=Ro)
-    assert np.array_equal(_bits(Y), Yr)
+    _assert_y(_bits(Y), Yr, Ya)
     assert np.array_equal(_bits(Ro), Hr)
 
 
 def test_rmsnorm_in_place_residual_and_strides(ck):
     M, K = 45, 1024
     X, R, w = _inputs(M, K, 5)
-    Yr, Hr = oracle.rmsnorm_rows(_bits(X), _bits(R), _bits(w), 1e-6)
+    Yr, Hr, Ya = oracle.rmsnorm_rows(_bits(X), _bits(R), _bits(w), 1e-6, with_alt=True)
     wideX = torch.zeros((M, K + 256), dtype=torch.bfloat16, device="cuda")
     wideX[:, :K] = X.cuda()
     wideR = torch.zeros((M, K + 512), dtype=torch.bfloat16, device="cuda")
     wideR[:, :K] = R.cuda()
     r = wideR[:, :K]
     Y = ck.rmsnorm_residual(wideX[:, :K], r, w.cuda(), 1e-6, residual_out=r)  # in place
-    assert np.array_equal(_bits(Y), Yr)
+    _assert_y(_bits(Y), Yr, Ya)
     assert np.array_equal(_bits(r), Hr)
     assert not wideR[:, K:].any()
 
@@ -87,9 +92,37 @@ def test_rmsnorm_extreme_rows(ck):
     x[3] = 1e-3
     X = x.to(torch.bfloat16)
     for eps in (1e-6, 1.0):
-        Yr, _ = oracle.rmsnorm_rows(_bits(X), None, _bits(w), eps)
+        Yr, _, Ya = oracle.rmsnorm_rows(_bits(X), None, _bits(w), eps, with_alt=True)
         Y = ck.rmsnorm_residual(X.cuda(), None, w.cuda(), eps)
-        assert np.array_equal(_bits(Y), Yr)
+        _assert_y(_bits(Y), Yr, Ya)
+
+
+def _norm_linear_check(ck, X, R, w, W, bias, eps, rows=None):
+    """ck_int8_linear_norm against the oracle: residual output bit for bit,
+    the normalised rows in the workspace admissible, codes and row scales
+    admissible, output rows (those whose normalised values are unambiguous)
+    within 1 bf16 ulp."""
+    M, K = X.shape
+    Qw, s_w = ck.rotate_quant_weight(W.cuda())
+    Qw_r, s_w_r = oracle.rotate_quant_weight(W.numpy())
+    Yn, Hr, Ya = oracle.rmsnorm_rows(_bits(X), _bits(R), _bits(w), eps, with_alt=True)
+    ws = torch.empty((ck.norm_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
+    Ro = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    Y = ck.int8_linear_norm(X.cuda(), Qw, s_w, bias.cuda(), R.cuda(), w.cuda(), eps,
+                            residual_out=Ro, workspace=ws)
+    torch.cuda.synchronize()
+    off_q = (M * K * 2 + 255) // 256 * 256
+    Qx = ws[off_q: off_q + M * K].view(M, K).view(torch.int8).cpu().numpy()
+    off_s = off_q + (M * K + 255) // 256 * 256
+    s_x = ws[off_s: off_s + 4 * M].view(torch.float32).cpu().numpy()
+    assert np.array_equal(_bits(Ro), Hr)
+    _assert_y(_bits(ws[: M * K * 2].view(torch.bfloat16).view(M, K)), Yn, Ya)
+    assert_codes_admissible(Qx, s_x, Yn, Ya)
+    Qx_r, s_x_r = oracle.quantize_rows_bf16(Yn, rotate=True)
+    rows = np.arange(M) if rows is None else rows
+    rows = rows[~(Yn[rows] != Ya[rows]).any(axis=1)]
+    Yr = oracle.linear_rows(Qx_r, s_x_r, Qw_r, s_w_r, _bits(bias), rows)
+    assert_bf16_close(_bits(Y[torch.from_numpy(rows).cuda()]), Yr)
 
 
 @pytest.mark.parametrize("M,K,N", [(1, 256, 8), (130, 5376, 264), (300, 1024, 520)])
@@ -97,37 +130,33 @@ def test_int8_linear_norm_matches_oracle(ck, M, K, N):
     X, R, w = _inputs(M, K, 3 * M + K)
     cfg = workloads.custom(M, K, N, seed=M + N)
     _, W, bias = workloads.make_inputs(cfg)
-    Qw, s_w = ck.rotate_quant_weight(W.cuda())
-    Qw_r, s_w_r = oracle.rotate_quant_weight(W.numpy())
-    Yr, Hr, Qx_r, s_x_r = oracle.int8_linear_norm(_bits(X), Qw_r, s_w_r, _bits(bias), _bits(R),
-                                                  _bits(w), 1e-6)
-    ws = torch.empty((ck.norm_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
-    Ro = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
-    Y = ck.int8_linear_norm(X.cuda(), Qw, s_w, bias.cuda(), R.cuda(), w.cuda(), 1e-6,
-                            residual_out=Ro, workspace=ws)
-    torch.cuda.synchronize()
-    off_q = (M * K * 2 + 255) // 256 * 256
-    Qx = ws[off_q: off_q + M * K].view(M, K).view(torch.int8)
-    off_s = off_q + (M * K + 255) // 256 * 256
-    s_x = ws[off_s: off_s + 4 * M].view(torch.float32)
-    assert np.array_equal(_bits(Ro), Hr)
-    assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_x_r.view(np.uint32))
-    assert np.array_equal(Qx.cpu().numpy(), Qx_r)
-    d = np.abs(_ordered(_bits(Y)) - _ordered(Yr))
-    assert d.max(initial=0) <= 1
+    _norm_linear_check(ck, X, R, w, W, bias, 1e-6)
+
+
+@pytest.mark.slow
+def test_int8_linear_norm_full_size_ragged(ck):
+    """The ragged M8193/K5376/N16128 workload with a residual and a weight:
+    every code and row scale, every residual and normalised value, and all
+    outputs of one row per 256-row M-tile."""
+    cfg = workloads.CONFIGS[1]
+    X, W, bias = workloads.make_inputs(cfg)
+    g = torch.Generator().manual_seed(321)
+    R = torch.randn(cfg.M, cfg.K, generator=g).to(torch.bfloat16)
+    w = (1.0 + 0.25 * torch.randn(cfg.K, generator=g)).to(torch.bfloat16)
+    _norm_linear_check(ck, X, R, w, W, bias, 1e-6, rows=tile_rows(cfg.M))
 
 
 @pytest.mark.slow
 def test_rmsnorm_full_size_headline(ck):
     """M32700/K5376 (the benchmarked activation shape) with a residual and a
-    weight: every normalised value and residual output bit-exact."""
+    weight: every normalised value admissible, every residual output exact."""
     cfg = workloads.HEADLINE
     X, _, _ = workloads.make_inputs(cfg)
     g = torch.Generator().manual_seed(123)
     R = torch.randn(cfg.M, cfg.K, generator=g).to(torch.bfloat16)
     w = (1.0 + 0.25 * torch.randn(cfg.K, generator=g)).to(torch.bfloat16)
-    Yr, Hr = oracle.rmsnorm_rows(_bits(X), _bits(R), _bits(w), 1e-6)
+    Yr, Hr, Ya = oracle.rmsnorm_rows(_bits(X), _bits(R), _bits(w), 1e-6, with_alt=True)
     Ro = torch.empty((cfg.M, cfg.K), dtype=torch.bfloat16, device="cuda")
     Y = ck.rmsnorm_residual(X.cuda(), R.cuda(), w.cuda(), 1e-6, residual_out=Ro)
-    assert np.array_equal(_bits(Y), Yr)
+    _assert_y(_bits(Y), Yr, Ya)
     assert np.array_equal(_bits(Ro), Hr)

@@ -14,10 +14,9 @@ import torch
 
 import oracle
 import workloads
+from parity_helpers import assert_bf16_close, tile_rows
 
 pytestmark = pytest.mark.gpu
-
-BF16_ULP_TOL = 1
 
 
 @pytest.fixture(scope="module")
@@ -29,17 +28,6 @@ def ck():
     m.clear_device_error()
     yield m
     assert m.device_error() == m.CK_OK
-
-
-def bf16_ordered(bits: np.ndarray) -> np.ndarray:
-    """Map bf16 bit patterns to integers whose differences count ulps."""
-    b = bits.astype(np.int32)
-    return np.where(b & 0x8000, 0x8000 - b, b)
-
-
-def assert_bf16_close(got_bits: np.ndarray, ref_bits: np.ndarray, tol: int = BF16_ULP_TOL):
-    d = np.abs(bf16_ordered(got_bits) - bf16_ordered(ref_bits))
-    assert d.max(initial=0) <= tol, f"max bf16 ulp distance {d.max()} at {np.unravel_index(d.argmax(), d.shape)}"
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -253,16 +241,23 @@ def _sample_rows(M):
     rows = {0, 1, 126, 127, 128, 129, M // 2, M - 129, M - 128, M - 2, M - 1}
     rng = np.random.default_rng(M)
     rows |= set(rng.integers(0, M, 24).tolist())
+    rows |= set(tile_rows(M).tolist())
     return np.array(sorted(r for r in rows if 0 <= r < M), np.int64)
+
+
+GUARD = 0x5A
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("cfg", workloads.CONFIGS, ids=[c.name for c in workloads.CONFIGS])
 def test_full_size_config(ck, cfg):
     """At the full sizes, in the launch configuration the benchmark times:
-    every code and row scale of activations and weights bit-exact; INT32
-    accumulators and BF16 outputs of sampled rows (tile edges and the ragged
-    last row included) against the oracle computed row by row."""
+    every code and row scale of activations and weights bit-exact; all N
+    outputs of one row in every 256-row M-tile (its position in the tile
+    varying), tile edges and the ragged last row against the oracle computed
+    row by row; the 2-SM GEMM's INT32 accumulators of a 300-row slice at the
+    full K and N; and guard bands after the codes, the row scales and Y
+    left untouched."""
     X, W, bias = workloads.make_inputs(cfg)
     Xd, Wd, bd = dev(X), dev(W), dev(bias)
     Qw, s_w = ck.rotate_quant_weight(Wd)
@@ -272,12 +267,22 @@ def test_full_size_config(ck, cfg):
     assert np.array_equal(to_np(Qw), rqw)
     del W
 
-    ws = torch.empty((ck.workspace_bytes(cfg.M, cfg.K),), dtype=torch.uint8, device="cuda")
-    Y = ck.int8_linear(Xd, Qw, s_w, bd, workspace=ws)
+    need = ck.workspace_bytes(cfg.M, cfg.K)
+    ws = torch.full((need + 4096,), GUARD, dtype=torch.uint8, device="cuda")
+    Ybuf = torch.full((cfg.M + 2, cfg.N), 0.0, dtype=torch.bfloat16, device="cuda")
+    Ybuf.view(torch.uint8).fill_(GUARD)
+    Y = ck.int8_linear(Xd, Qw, s_w, bd, out=Ybuf[: cfg.M], workspace=ws)
     torch.cuda.synchronize()
-    Qx = ws[: cfg.M * cfg.K].view(cfg.M, cfg.K).view(torch.int8)
+    assert Y.data_ptr() == Ybuf.data_ptr()
     off = (cfg.M * cfg.K + 255) // 256 * 256
+    Qx = ws[: cfg.M * cfg.K].view(cfg.M, cfg.K).view(torch.int8)
     s_x = ws[off: off + 4 * cfg.M].view(torch.float32)
+    # guard bands: the padding after the codes, everything after the scales,
+    # the two rows after Y
+    assert bool((ws[cfg.M * cfg.K: off] == GUARD).all())
+    assert bool((ws[off + 4 * cfg.M:] == GUARD).all())
+    assert bool((Ybuf[cfg.M:].view(torch.uint8) == GUARD).all())
+
     rqx, rsx = oracle.quantize_rows_bf16(workloads.bf16_bits(X))
     assert np.array_equal(to_np(s_x).view(np.uint32), rsx.view(np.uint32))
     assert np.array_equal(to_np(Qx), rqx)
@@ -287,8 +292,9 @@ def test_full_size_config(ck, cfg):
     Ys = to_np(Y[torch.from_numpy(rows).cuda()])
     assert_bf16_close(Ys, Yr)
 
-    acc_rows = ck.test_int8_gemm_i32(Qx[torch.from_numpy(rows[:8]).cuda()].contiguous(), Qw)
-    assert np.array_equal(to_np(acc_rows), oracle.gemm_i32(rqx[rows[:8]], rqw))
+    lo = cfg.M // 2 - 150
+    acc = ck.test_int8_gemm_i32(Qx[lo: lo + 300].contiguous(), Qw)  # M > 128: 2-SM kernel
+    assert np.array_equal(to_np(acc), oracle.gemm_i32(rqx[lo: lo + 300], rqw))
 
 
 # ------------------------------------------------------------------ input activation
@@ -303,6 +309,19 @@ def _act_inputs(M, K, seed):
     x[1::7, 9] = 3.0e4
     x[::3] *= 3.0
     return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("act", ["none", "relu", "silu", "gelu_tanh"])
+def test_input_act_every_bf16_input(ck, act):
+    """The activation as the quantiser applies it, on every finite bf16
+    input, equals the oracle's bf16 rounding of the exact act(x) bit for bit."""
+    bits = np.arange(0x10000, dtype=np.uint32).astype(np.uint16)
+    X = workloads.from_bf16_bits(bits)
+    got = to_np(ck.test_input_act(dev(X), act))
+    finite = (bits & 0x7F80) != 0x7F80
+    want = oracle.act_bf16(act, bits)
+    bad = np.nonzero((got != want) & finite)[0]
+    assert bad.size == 0, [(hex(int(bits[i])), hex(int(got[i])), hex(int(want[i]))) for i in bad[:8]]
 
 
 @pytest.mark.parametrize("act", ["relu", "silu", "gelu_tanh"])
@@ -326,6 +345,30 @@ def test_int8_linear_act_matches_oracle(ck, act):
     Y = ck.int8_linear(dev(X), Qw, s_w, dev(bias), input_act=act)
     Yr = oracle.int8_linear(workloads.bf16_bits(X), rqw, rsw, workloads.bf16_bits(bias), act=act)[0]
     assert_bf16_close(to_np(Y), Yr)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh"])
+def test_int8_linear_act_full_size(ck, act):
+    """int8_linear(input_act) on the ragged M8193/K5376/N16128 workload:
+    every code and row scale, and all outputs of one row per 256-row M-tile."""
+    cfg = workloads.CONFIGS[1]
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw, s_w = ck.rotate_quant_weight(dev(W))
+    rqw, rsw = oracle.rotate_quant_weight(W.numpy())
+    del W
+    ws = torch.empty((ck.workspace_bytes(cfg.M, cfg.K),), dtype=torch.uint8, device="cuda")
+    Y = ck.int8_linear(dev(X), Qw, s_w, dev(bias), workspace=ws, input_act=act)
+    torch.cuda.synchronize()
+    off = (cfg.M * cfg.K + 255) // 256 * 256
+    Qx = to_np(ws[: cfg.M * cfg.K].view(cfg.M, cfg.K).view(torch.int8))
+    s_x = to_np(ws[off: off + 4 * cfg.M].view(torch.float32))
+    rqx, rsx = oracle.quantize_rows_bf16(workloads.bf16_bits(X), act=act)
+    assert np.array_equal(s_x.view(np.uint32), rsx.view(np.uint32))
+    assert np.array_equal(Qx, rqx)
+    rows = tile_rows(cfg.M)
+    Yr = oracle.linear_rows(rqx, rsx, rqw, rsw, workloads.bf16_bits(bias), rows)
+    assert_bf16_close(to_np(Y[torch.from_numpy(rows).cuda()]), Yr)
 
 
 # ------------------------------------------------------------------ convrot_w4a4_linear
