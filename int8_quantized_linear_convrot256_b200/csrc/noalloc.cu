@@ -21,7 +21,9 @@
 //    them, e.g. on one stream.
 //  * The first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress) with that device current and caches it; make that
-//    first call before any stream capture on the device.
+//    first call before any stream capture on the device. The lookup is done
+//    again when the device's context changes (after cudaDeviceReset, or when
+//    another context is made current), since the address belongs to a context.
 //  * Problems whose codes and scales need more than the array holds
 //    (ck_int8_linear_workspace_bytes(M, K) > CK_NOALLOC_SCRATCH_BYTES) are
 //    rejected with CK_ERR_WORKSPACE before anything is launched.
@@ -32,6 +34,7 @@
 #include <mutex>
 
 #include "ck.h"
+#include "internal.h"
 
 namespace {
 
@@ -42,21 +45,29 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[CK_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+    void *ptr = nullptr;
+    unsigned generation = 0;  // device-state generation the address was taken in
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of the array on the current device, looked up once per
-// device with that device current.
-ck_status scratch_address(void **out) {
+// Device address of the array on the current device (a B200: the caller has
+// checked), looked up once per device context with that device current.
+ck_status scratch_address(unsigned generation, void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr &a = g_scratch[dev];
+    if (a.ptr == nullptr || a.generation != generation) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();  // leave no sticky-looking error for the caller's next check
             return CK_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        }
+        a.ptr = p;
+        a.generation = generation;
     }
-    *out = g_scratch_addr[dev];
+    *out = a.ptr;
     return CK_OK;
 }
 
@@ -65,14 +76,16 @@ ck_status scratch_address(void **out) {
 extern "C" ck_status ck_int8_linear_noalloc(const ck_bf16 *X, int64_t ldx, const int8_t *Qw,
                                             const float *s_w, const ck_bf16 *bias, ck_bf16 *Y,
                                             int64_t M, int64_t N, int64_t K, ck_stream_t stream) {
-    if (M < 0 || N < 0 || K <= 0) return CK_ERR_INVALID_VALUE;
-    if (K % 256 != 0 || K > CK_MAX_K || N % 8 != 0) return CK_ERR_UNSUPPORTED_SHAPE;
+    // the checks of ck_int8_linear, in its order, then the array's size
+    ck_status s = ck::check_linear_args(X, ldx, Qw, s_w, bias, Y, M, N, K, nullptr, false);
+    if (s != CK_OK || M == 0 || N == 0) return s;
     if (ck_int8_linear_workspace_bytes(M, K) > CK_NOALLOC_SCRATCH_BYTES) return CK_ERR_WORKSPACE;
+    unsigned generation = 0;
+    s = ck::check_current_device(&generation);  // CK_ERR_ARCH before any symbol lookup
+    if (s != CK_OK) return s;
     void *scratch = nullptr;
-    if (M > 0 && N > 0) {
-        const ck_status s = scratch_address(&scratch);
-        if (s != CK_OK) return s;
-    }
+    s = scratch_address(generation, &scratch);
+    if (s != CK_OK) return s;
     return ck_int8_linear(X, ldx, Qw, s_w, bias, Y, M, N, K, scratch, CK_NOALLOC_SCRATCH_BYTES,
                           stream);
 }
