@@ -558,9 +558,55 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
     return line
 
 
+def launch_ranks(args, argv) -> int:
+    """Runs this script once per GPU under torch.distributed.run (one process
+    per rank, rendezvous on 127.0.0.1) and returns the launcher's status."""
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_dry(args, cfg, rank, world):
+    """The rank plumbing without a GPU (gloo): every rank times a small host
+    loop for each step, the times are reduced as the max over ranks, and rank
+    0 prints a JSON line with the same keys as a real run."""
+    import torch.distributed as dist
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        if world > 1:
+            dist.barrier()
+        t = time.perf_counter()
+        float(np.sum(np.arange(10000, dtype=np.float64)))
+        if i >= args.warmup:
+            times.append(1e3 * (time.perf_counter() - t))
+    ms = max_over_ranks([sum(times) / len(times)])[0]
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                          "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None,
+                          "dtype": "int8", "data": "synthetic", "impl": args.impl,
+                          "dry_run": "gloo ranks on the host, no GPU work",
+                          "config": config_dict(cfg, world, args.scaling, args.act, args.path)}),
+              flush=True)
+    return 0
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of this node; above 1 the script starts one rank per GPU itself "
+                         "(torch.distributed.run) unless it already runs as a rank")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="exercise the rank launch and the max-over-ranks timing on the host "
+                         "(gloo), with no GPU work")
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -583,10 +629,29 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args, argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but {world} ranks were started")
     cfg = workloads.BY_NAME[args.workload]
+
+    if args.dry_run:
+        import datetime
+
+        import torch.distributed as dist
+
+        if world > 1:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        try:
+            return run_dry(args, cfg, rank, world)
+        finally:
+            if world > 1:
+                dist.destroy_process_group()
 
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)

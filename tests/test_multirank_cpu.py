@@ -74,3 +74,26 @@ def test_two_gloo_ranks_split_rows_and_reduce_timings(tmp_path):
     mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
     assert (tmp_path / "ok").exists(), os.listdir(tmp_path)
+
+
+def test_bench_starts_its_own_ranks():
+    """`bench.py --gpus 2` launches two ranks itself (torch.distributed.run on
+    127.0.0.1); the dry run does the rank plumbing on gloo with no GPU work and
+    rank 0 alone prints one JSON line reporting both GPUs."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "3", "--warmup", "3"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=240)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["dry_run"] and line["ms_per_step"] > 0
+    assert line["config"]["parallelism"].startswith("replicas x2")
