@@ -394,6 +394,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     if status != ck.CK_OK:
         raise RuntimeError(f"device error during the timed region: {ck.status_string(status)}")
 
+    probe_tops = None
+    if args.path in ("int8", "norm") and not args.no_probe:
+        probe_tops = max_over_ranks([i8_probe_tops(ck, stream)], dev)[0]
+
     q_ms = [e[0].elapsed_time(e[1]) for e in ev]
     g_ms = [e[1].elapsed_time(e[2]) for e in ev]
     s_ms = [e[0].elapsed_time(e[2]) for e in ev]
@@ -410,7 +414,29 @@ def run_ours(args, cfg, rank, world, local_rank):
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
     return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
-                  clocks, t_wall0, t_wall1, spread)
+                  clocks, t_wall0, t_wall1, spread, probe_tops)
+
+
+PROBE_MMAS = 200_000
+
+
+def i8_probe_tops(ck, stream):
+    """The device's INT8 tensor-core ceiling (ck_test_i8_mma_peak: back-to-back
+    pair MMAs of the GEMM's shape, no memory traffic), best of three ~15 ms
+    launches after one warm-up, timed with events on the launching stream."""
+    import torch
+
+    ck.test_i8_mma_peak(PROBE_MMAS // 10, stream=stream)
+    best = 0.0
+    for _ in range(3):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ops = ck.test_i8_mma_peak(PROBE_MMAS, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        best = max(best, ops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    return best
 
 
 E2E_CHUNK_ROWS = 2048
@@ -451,7 +477,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
 
 
 def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
-           t_wall0, t_wall1, spread=None):
+           t_wall0, t_wall1, spread=None, probe_tops=None):
     # per-rank work: the full batch (weak, replicas) or this rank's row shard
     # (strong); the job's total is world x per-rank (weak) or the whole batch
     M, N, K = X.shape[0], cfg.N, cfg.K
@@ -536,6 +562,8 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                          ("frac_of_spec_9000" if args.path == "nvfp4" else "frac_of_spec_4500"):
                              gemm_tops / (9000.0 if args.path == "nvfp4" else 4500.0),
                          "frac_of_measured_sustained": gemm_tops / sustained_peak,
+                         **({"i8_probe_tops": probe_tops, "frac_of_i8_probe": gemm_tops / probe_tops}
+                            if probe_tops else {}),
                          "ms_per_launch": ms_g},
             "quantizer": {"kernel": ("nvfp4_bulk_kernel<1> + <2> (ConvRot256 + NVFP4, two "
                                      "staged passes over X)" if args.path == "nvfp4" else
@@ -623,6 +651,8 @@ def main(argv=None):
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-probe", action="store_true",
+                    help="skip the INT8 tensor-core peak probe run after the timed region")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
     args = ap.parse_args(argv)

@@ -462,6 +462,17 @@ ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t
 ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck_stream_t stream);
 
 /*
+ * The INT8 tensor-core ceiling, measured: on every pair of SMs the GEMM uses
+ * (*pairs receives their number), mmas_per_pair back-to-back
+ * tcgen05.mma.cta_group::2.kind::i8 of the GEMM's shape (M 256, N 256, K 32:
+ * 2 * 256 * 256 * 32 operations each) on shared-memory operands, with no
+ * global-memory traffic. Time it with events on `stream`; the operation count
+ * is 4194304 * mmas_per_pair * *pairs. No counterpart in the pages: it gives
+ * the INT8 GEMM's roofline a measured denominator.
+ */
+ck_status ck_test_i8_mma_peak(int64_t mmas_per_pair, int *pairs, ck_stream_t stream);
+
+/*
  * Fault injection for the bounded waits, host side only: with mode 1 the next
  * GEMM launch (INT8 or NVFP4) on this thread's current device runs with its TMA producer
  * issuing nothing, so the MMA warp's wait for the first stage can never be

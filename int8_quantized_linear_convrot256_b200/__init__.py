@@ -94,6 +94,7 @@ _SIGS = {
     "ck_test_quantize_rowwise_norotate": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_test_inject_producer_stall": (_st, [ctypes.c_int, _i64]),
     "ck_test_input_act": (_st, [_vp, _i64, _st, _vp, _vp]),
+    "ck_test_i8_mma_peak": (_st, [_i64, ctypes.POINTER(ctypes.c_int), _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -559,6 +560,18 @@ def test_input_act(X: torch.Tensor, act: str, out: torch.Tensor | None = None,
 
 
 test_input_act.__test__ = False
+
+
+def test_i8_mma_peak(mmas_per_pair: int, stream=None) -> int:
+    """Launches the INT8 tensor-core peak probe; returns the operations it
+    performs (4194304 per pair MMA) for the caller's event timing."""
+    pairs = ctypes.c_int(0)
+    _check(lib.ck_test_i8_mma_peak(mmas_per_pair, ctypes.byref(pairs), _stream(stream)),
+           "ck_test_i8_mma_peak")
+    return 2 * 256 * 256 * 32 * mmas_per_pair * pairs.value
+
+
+test_i8_mma_peak.__test__ = False
 
 
 def device_error() -> int:

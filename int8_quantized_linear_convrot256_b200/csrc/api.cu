@@ -869,6 +869,16 @@ ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
+ck_status ck_test_i8_mma_peak(int64_t mmas_per_pair, int *pairs, ck_stream_t stream) {
+    if (mmas_per_pair <= 0 || !pairs) return CK_ERR_INVALID_VALUE;
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_i8_mma_peak(mmas_per_pair, st->err, ck::kDefaultWaitLimitNs, pairs,
+                                           reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
 const char *ck_status_string(ck_status status) {
     switch (status) {
         case CK_OK: return "CK_OK";

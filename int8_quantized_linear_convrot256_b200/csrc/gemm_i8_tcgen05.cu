@@ -662,6 +662,64 @@ __device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t
     }
 }
 
+// ---------------------------------------------------------------- peak probe
+//
+// The INT8 tensor-core ceiling of this device, measured: every CTA pair
+// issues `mmas` back-to-back tcgen05.mma.cta_group::2.kind::i8 of the GEMM's
+// shape (M 256, N 256, K 32, int32 accumulators in TMEM) on operands that sit
+// in shared memory (their values do not matter), with no global-memory
+// traffic and no epilogue. 2 * 256 * 256 * 32 operations per instruction.
+constexpr int kProbeThreads = 128;
+constexpr size_t kProbeSmemBytes = 1024 + 2 * size_t(kPairABytes) + 64;
+
+__global__ void __launch_bounds__(kProbeThreads, 1)
+i8_mma_peak_kernel(int64_t mmas, unsigned *err, uint64_t limit_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *done = reinterpret_cast<uint64_t *>(smem + 2 * kPairABytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    const int warp = threadIdx.x >> 5;
+    const bool leader = cluster_ctarank() == 0;
+
+    for (int i = threadIdx.x; i < 2 * kPairABytes / 16; i += kProbeThreads)
+        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(done), 1);
+        fence_mbar_init();
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros visible to the MMA
+    if (warp == 0) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kPairBN);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (leader && threadIdx.x == 32) {
+        const uint32_t a = smem_u32(smem);
+        const uint64_t adesc = smem_desc_sw128(a);
+        const uint64_t bdesc = smem_desc_sw128(a + kPairABytes);
+        for (int64_t i = 0; i < mmas; ++i) {
+            const uint64_t k = uint64_t(2 * (i & 3));  // the four K steps of a 128-byte K-block
+            umma_i8_pair(tmem, adesc + k, bdesc + k, kPairIdesc, i != 0 ? 1u : 0u);
+        }
+        umma_commit_pair_mc(smem_u32(done), 0x3);
+    }
+    if (threadIdx.x == 0 && !mbar_wait_bounded(smem_u32(done), 0u, limit_ns, nullptr))
+        atomicMax(err, kDevErrTimeout);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kPairBN);
+    }
+}
+
 }  // namespace
 
 namespace {
@@ -718,6 +776,34 @@ cudaError_t max_active_pairs(int dev, int *out) {
 }
 
 }  // namespace
+
+cudaError_t launch_i8_mma_peak(int64_t mmas, unsigned *err, uint64_t limit_ns, int *pairs_out,
+                               cudaStream_t stream) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int pairs = 0;
+    e = max_active_pairs(dev, &pairs);  // one probe pair per pair of SMs the GEMM uses
+    if (e != cudaSuccess) return e;
+    if (pairs <= 0) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(i8_mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kProbeSmemBytes));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kProbeThreads, 1, 1);
+    cfg.dynamicSmemBytes = kProbeSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    *pairs_out = pairs;
+    return cudaLaunchKernelEx(&cfg, i8_mma_peak_kernel, mmas, err, limit_ns);
+}
 
 cudaError_t plan_gemm(int M, int N, int num_sms, GemmPlan *plan) {
     int dev = 0;

@@ -114,6 +114,12 @@ cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const
                            const GemmParams &p, bool raw_i32, const GemmPlan &plan,
                            cudaStream_t stream);
 
+// INT8 tensor-core peak probe: `mmas` back-to-back pair MMAs of the GEMM's
+// shape (2 * 256 * 256 * 32 ops each) per CTA pair, on every pair of SMs the
+// GEMM would use; *pairs_out receives the number of pairs launched.
+cudaError_t launch_i8_mma_peak(int64_t mmas, unsigned *err, uint64_t limit_ns, int *pairs_out,
+                               cudaStream_t stream);
+
 // ---- block-scaled NVFP4 GEMM with fused epilogue (gemm_nvfp4_tcgen05.cu)
 
 struct Nvfp4GemmParams {

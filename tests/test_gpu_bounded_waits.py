@@ -66,3 +66,4 @@ def test_stalled_producer_times_out_in_the_nvfp4_gemm(ck, M):
     r = workloads.from_bf16_bits(Yr).double().numpy()
     assert np.all(np.abs(y - r) <= np.abs(r) * 2.0 ** -7 + K * 2.0 ** -24 * mag + 1e-30)
     assert ck.device_error() == ck.CK_OK
+
