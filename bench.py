@@ -332,7 +332,6 @@ def run_ours(args, cfg, rank, world, local_rank):
             R = R[lo:hi].contiguous()
         Rd, gd = R.to(dev), w_norm.to(dev)
         Ro = torch.empty_like(Rd)  # the residual output (a separate buffer: steps stay equal)
-        Xn = torch.empty_like(Xd)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
@@ -347,9 +346,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         elif args.path == "nvfp4":
             ck.quantize_rotate_nvfp4(Xd, Qx, Sx, s_x)
         elif args.path == "norm":
-            # int8_linear's input RMSNorm and residual, then the quantiser
-            ck.rmsnorm_residual(Xd, Rd, gd, NORM_EPS, residual_out=Ro, out=Xn)
-            ck.quantize_rotate_rowwise(Xn, Qx, s_x)
+            # int8_linear's input RMSNorm and residual inside the quantiser
+            ck.quantize_rotate_rowwise_norm(Xd, Rd, gd, NORM_EPS, residual_out=Ro, Qx=Qx, s_x=s_x)
         elif args.act == "none":
             ck.quantize_rotate_rowwise(Xd, Qx, s_x)
         else:
@@ -389,14 +387,18 @@ def run_ours(args, cfg, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     t_wall1 = time.time()
-    clocks.stop()
     status = ck.device_error()
     if status != ck.CK_OK:
+        clocks.stop()
         raise RuntimeError(f"device error during the timed region: {ck.status_string(status)}")
 
     probe_tops = None
+    probe_clocks = None
     if args.path in ("int8", "norm") and not args.no_probe:
+        t_p0 = time.time()
         probe_tops = max_over_ranks([i8_probe_tops(ck, stream)], dev)[0]
+        probe_clocks = clocks.summary(t_p0, time.time())
+    clocks.stop()
 
     q_ms = [e[0].elapsed_time(e[1]) for e in ev]
     g_ms = [e[1].elapsed_time(e[2]) for e in ev]
@@ -414,7 +416,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
     return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
-                  clocks, t_wall0, t_wall1, spread, probe_tops)
+                  clocks, t_wall0, t_wall1, spread, probe_tops, probe_clocks)
 
 
 PROBE_MMAS = 200_000
@@ -477,7 +479,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
 
 
 def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
-           t_wall0, t_wall1, spread=None, probe_tops=None):
+           t_wall0, t_wall1, spread=None, probe_tops=None, probe_clocks=None):
     # per-rank work: the full batch (weak, replicas) or this rank's row shard
     # (strong); the job's total is world x per-rank (weak) or the whole batch
     M, N, K = X.shape[0], cfg.N, cfg.K
@@ -492,10 +494,10 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
         q_bytes = 2.0 * M * K + 0.5 * M * K + M * K / 16.0 + 4.0
         int8_peak = P["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
     elif args.path == "norm":
-        # the input RMSNorm (X and the residual read, residual output and the
-        # normalised rows written) and the quantiser (those rows read, codes
-        # and row scales written)
-        q_bytes = 8.0 * M * K + 3.0 * M * K + 4.0 * M
+        # the input RMSNorm inside the quantiser: X and the residual read, the
+        # residual output, the codes and the row scales written (the
+        # normalised rows never reach memory)
+        q_bytes = 7.0 * M * K + 4.0 * M
         int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     else:
         q_bytes = 3.0 * M * K + 4.0 * M
@@ -562,13 +564,14 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                          ("frac_of_spec_9000" if args.path == "nvfp4" else "frac_of_spec_4500"):
                              gemm_tops / (9000.0 if args.path == "nvfp4" else 4500.0),
                          "frac_of_measured_sustained": gemm_tops / sustained_peak,
-                         **({"i8_probe_tops": probe_tops, "frac_of_i8_probe": gemm_tops / probe_tops}
+                         **({"i8_probe_tops": probe_tops, "frac_of_i8_probe": gemm_tops / probe_tops,
+                             "i8_probe_clocks": probe_clocks}
                             if probe_tops else {}),
                          "ms_per_launch": ms_g},
             "quantizer": {"kernel": ("nvfp4_bulk_kernel<1> + <2> (ConvRot256 + NVFP4, two "
                                      "staged passes over X)" if args.path == "nvfp4" else
-                                     "rmsnorm_rows_kernel + quant_rows_bulk_kernel (input "
-                                     "RMSNorm with residual, then ConvRot256 + per-row INT8)"
+                                     "quant_norm_bulk_kernel (input RMSNorm with residual "
+                                     "fused into ConvRot256 + per-row INT8)"
                                      if args.path == "norm" else
                                      ("quant_rows_bulk_kernel" if K <= 28672 else
                                       "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)"),
@@ -580,7 +583,7 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
                     "call": f"ck_int8_linear_host: X from and Y to pinned host memory, chunks of "
                             f"{min(E2E_CHUNK_ROWS, M)} rows with copies overlapped with the kernels"},
-            "gpu_launches": {"w4a4": 3, "nvfp4": 4, "norm": 3}.get(args.path, 2) * args.steps,
+            "gpu_launches": {"w4a4": 3, "nvfp4": 4}.get(args.path, 2) * args.steps,
             "clocks": clocks.summary(t_wall0, t_wall1),
         }
     return line
@@ -646,7 +649,7 @@ def main(argv=None):
                     help="int8: int8_linear; w4a4: convrot_w4a4_linear (INT4 codes, packed "
                          "INT4 weights unpacked per step); nvfp4: ConvRot NVFP4 (two-pass "
                          "FP4 quantiser + block-scaled FP4 GEMM); norm: int8_linear with its "
-                         "input RMSNorm and a residual (ck_rmsnorm_residual first)")
+                         "input RMSNorm and a residual (normalised inside the quantiser)")
     ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

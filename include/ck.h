@@ -237,13 +237,37 @@ ck_status ck_rmsnorm_residual(const ck_bf16 *X, int64_t ldx, const ck_bf16 *resi
                               ck_bf16 *residual_out, int64_t ldo, const ck_bf16 *g, float eps,
                               int64_t M, int64_t K, ck_bf16 *Y, ck_stream_t stream);
 
+/* Largest K for which ck_int8_linear_norm normalises inside the quantiser. */
+#define CK_NORM_FUSED_MAX_K 14336
+
+/*
+ * quantize_and_rotate_rowwise on the input RMSNorm of X (comfy-kitchen
+ * 0.2.40, "Huawei Ascend backend": int8_linear's input RMSNorm and residual
+ * arguments), in one kernel: the normalised values (defined as in
+ * ck_rmsnorm_residual) are formed in the quantiser's staged load, rotated and
+ * quantised; only residual_out (when given), Qx and s_x are written.
+ * Arguments as in ck_rmsnorm_residual for X, residual, residual_out, g, eps,
+ * and as in ck_quantize_rotate_rowwise for Qx [M, K] and s_x [M].
+ * K <= CK_NORM_FUSED_MAX_K (CK_ERR_UNSUPPORTED_SHAPE otherwise).
+ */
+ck_status ck_quantize_rotate_rowwise_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual,
+                                          int64_t ldr, ck_bf16 *residual_out, int64_t ldo,
+                                          const ck_bf16 *g, float eps, int64_t M, int64_t K,
+                                          int8_t *Qx, float *s_x, ck_stream_t stream);
+
 /*
  * ck_int8_linear on the input RMSNorm of X (with an optional residual), as
- * the page's int8_linear takes them: ck_rmsnorm_residual into the workspace,
- * then the ConvRot quantiser and the INT8 GEMM on the normalised rows.
- * Arguments as in ck_rmsnorm_residual and ck_int8_linear. Workspace:
- * ck_int8_linear_norm_workspace_bytes(M, K) bytes, 256-B aligned (the
- * normalised rows, then the codes and row scales).
+ * the page's int8_linear takes them. For K <= CK_NORM_FUSED_MAX_K the
+ * normalisation runs inside the ConvRot quantiser's staged load (x and the
+ * residual staged together, the residual output written from there, the sum
+ * of squares in double, each normalised value rounded to bf16 as
+ * ck_rmsnorm_residual defines it and then rotated and quantised), so the
+ * normalised rows never reach memory; larger K runs ck_rmsnorm_residual into
+ * the workspace first. Then the INT8 GEMM. Arguments as in
+ * ck_rmsnorm_residual and ck_int8_linear. Workspace:
+ * ck_int8_linear_norm_workspace_bytes(M, K) bytes, 256-B aligned (the codes
+ * and row scales, as ck_int8_linear's; for K > CK_NORM_FUSED_MAX_K the
+ * normalised rows come first).
  */
 size_t ck_int8_linear_norm_workspace_bytes(int64_t M, int64_t K);
 ck_status ck_int8_linear_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual,

@@ -65,6 +65,8 @@ _SIGS = {
     "ck_rmsnorm_residual": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, ctypes.c_float, _i64,
                                   _i64, _vp, _vp]),
     "ck_int8_linear_norm_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "ck_quantize_rotate_rowwise_norm": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp,
+                                              ctypes.c_float, _i64, _i64, _vp, _vp, _vp]),
     "ck_int8_linear_norm": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, ctypes.c_float, _vp, _vp,
                                   _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "ck_rotate_quant_weight_int4": (_st, [_vp, _i64, _i64, _vp, _vp, _vp]),
@@ -285,6 +287,31 @@ def rmsnorm_residual(X: torch.Tensor, residual: torch.Tensor | None = None,
                                    _ptr(residual_out), ldo, _ptr(g), float(eps), M, K, _ptr(out),
                                    _stream(stream)), "ck_rmsnorm_residual")
     return out
+
+
+NORM_FUSED_MAX_K = 14336
+
+
+def quantize_rotate_rowwise_norm(X: torch.Tensor, residual: torch.Tensor | None = None,
+                                 g: torch.Tensor | None = None, eps: float = 1e-6,
+                                 residual_out: torch.Tensor | None = None, Qx=None, s_x=None,
+                                 stream=None):
+    """quantize_and_rotate_rowwise of the input RMSNorm of X in one kernel
+    (ck_quantize_rotate_rowwise_norm): the normalised rows are never stored.
+    Returns (Qx int8 [M, K], s_x fp32 [M]); K <= NORM_FUSED_MAX_K."""
+    M, K, ldr, ldo = _norm_args(X, residual, residual_out, g)
+    if Qx is None:
+        Qx = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if s_x is None:
+        s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _need(Qx, "Qx", torch.int8, 2)
+    _rows_contiguous(Qx, "Qx")
+    _need(s_x, "s_x", torch.float32, 1)
+    _check(lib.ck_quantize_rotate_rowwise_norm(_ptr(X), _row_stride(X, K), _ptr(residual), ldr,
+                                               _ptr(residual_out), ldo, _ptr(g), float(eps), M, K,
+                                               _ptr(Qx), _ptr(s_x), _stream(stream)),
+           "ck_quantize_rotate_rowwise_norm")
+    return Qx, s_x
 
 
 def norm_workspace_bytes(M: int, K: int) -> int:

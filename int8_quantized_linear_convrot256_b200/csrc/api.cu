@@ -477,8 +477,33 @@ ck_status ck_rmsnorm_residual(const ck_bf16 *X, int64_t ldx, const ck_bf16 *resi
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
+ck_status ck_quantize_rotate_rowwise_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *residual,
+                                          int64_t ldr, ck_bf16 *residual_out, int64_t ldo,
+                                          const ck_bf16 *g, float eps, int64_t M, int64_t K,
+                                          int8_t *Qx, float *s_x, ck_stream_t stream) {
+    if (M < 0) return CK_ERR_INVALID_VALUE;
+    ck_status s = check_k(K);
+    if (s == CK_ERR_INVALID_VALUE) return s;
+    if (M > 0 && (!X || !Qx || !s_x)) return CK_ERR_INVALID_VALUE;
+    if (s != CK_OK) return s;
+    if (K > CK_NORM_FUSED_MAX_K || M >= (int64_t(1) << 31)) return CK_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return CK_OK;
+    s = check_norm(X, ldx, residual, ldr, residual_out, ldo, g, eps, K);
+    if (s != CK_OK) return s;
+    if (!aligned16(Qx) || !aligned4(s_x)) return CK_ERR_MISALIGNED;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    bool launched = false;
+    cudaError_t e = ck::launch_quant_norm_bf16(X, M, K, ldx, residual, ldr, residual_out, ldo, g,
+                                               eps, Qx, s_x, st->err, st->num_sms,
+                                               reinterpret_cast<cudaStream_t>(stream), &launched);
+    return (e == cudaSuccess && launched) ? CK_OK : CK_ERR_CUDA;
+}
+
 size_t ck_int8_linear_norm_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
+    if (K <= CK_NORM_FUSED_MAX_K) return ck_int8_linear_workspace_bytes(M, K);
     return round256(size_t(M) * size_t(K) * 2) + ck_int8_linear_workspace_bytes(M, K);
 }
 
@@ -505,11 +530,22 @@ ck_status ck_int8_linear_norm(const ck_bf16 *X, int64_t ldx, const ck_bf16 *resi
     s = device_state(&st);
     if (s != CK_OK) return s;
     uint8_t *base = static_cast<uint8_t *>(workspace);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (K <= CK_NORM_FUSED_MAX_K) {
+        // the normalisation inside the quantiser's staged load
+        int8_t *Qx = reinterpret_cast<int8_t *>(base);
+        float *s_x = reinterpret_cast<float *>(base + round256(size_t(M) * size_t(K)));
+        bool launched = false;
+        cudaError_t e = ck::launch_quant_norm_bf16(X, M, K, ldx, residual, ldr, residual_out, ldo,
+                                                   g, eps, Qx, s_x, st->err, st->num_sms, cs,
+                                                   &launched);
+        if (e != cudaSuccess || !launched) return CK_ERR_CUDA;
+        return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
+    }
     ck_bf16 *Xn = reinterpret_cast<ck_bf16 *>(base);
     int8_t *Qx = reinterpret_cast<int8_t *>(base + round256(size_t(M) * size_t(K) * 2));
     float *s_x = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Qx) +
                                            round256(size_t(M) * size_t(K)));
-    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = ck::launch_rmsnorm_rows(X, ldx, residual, ldr, residual_out, ldo, g, eps, M, K,
                                             Xn, cs);
     if (e != cudaSuccess) return CK_ERR_CUDA;

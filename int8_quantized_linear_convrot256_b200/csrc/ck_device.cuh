@@ -98,6 +98,16 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, int32_t x, int32_
         : "memory");
 }
 
+// As tma_store_2d, with an L2 eviction policy for the written lines.
+__device__ __forceinline__ void tma_store_2d_hint(const void *tmap, int32_t x, int32_t y,
+                                                  uint32_t smem_src, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint"
+        " [%0, {%1, %2}], [%3], %4;" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(x), "r"(y), "r"(smem_src), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -226,6 +236,32 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t smem_dst, const void *
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster_addr)
         : "memory");
+}
+
+// As tma_load_2d_pair, with an L2 eviction policy (createpolicy) for the
+// loaded lines.
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t smem_dst, const void *tmap,
+                                                      int32_t x, int32_t y,
+                                                      uint32_t bar_cluster_addr, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster_addr), "l"(policy)
+        : "memory");
+}
+
+// L2 policies: keep lines (operands reused by later tiles) or let them go
+// first (results written once).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t smem_slot, uint32_t ncols) {

@@ -376,6 +376,9 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             const uint32_t leader_full0 = mapa_shared(smem_u32(&ctl->full[0]), 0);
+            // Qw is re-read by every group of M-tiles: keep it in L2 while
+            // A (reused within a group only) and Y (written once) pass through
+            const uint64_t keep = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_parity = 0;
             bool ok = true;
@@ -396,7 +399,7 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         const uint32_t dst = smem_u32(smem + size_t(stage) * kPairStageBytes);
                         const uint32_t bar = leader_full0 + uint32_t(8 * stage);
                         tma_load_2d_pair(dst, &tmA, kb * BK, a_row, bar);
-                        tma_load_2d_pair(dst + kPairABytes, &tmB, kb * BK, b_row, bar);
+                        tma_load_2d_pair_hint(dst + kPairABytes, &tmB, kb * BK, b_row, bar, keep);
                         issued |= 1u << stage;
                         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                         if (++stage == kPairStages) {
@@ -592,7 +595,7 @@ __device__ __forceinline__ void store_accumulators_tma(const GemmParams &p,
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(tmY, n0, row0, buf);
+            tma_store_2d_hint(tmY, n0, row0, buf, l2_policy_evict_first());
             bulk_commit_group();
         }
         ++chunk_count;

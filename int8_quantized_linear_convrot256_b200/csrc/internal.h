@@ -33,6 +33,17 @@ cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int6
                                    bool rotate, int act, int qmax, int8_t *Q, float *S,
                                    unsigned *err, int num_sms, cudaStream_t stream);
 
+// The input RMSNorm (h = bf16(x + r) written to Rout when given, y = the
+// bf16 rounding of h g / sqrt(mean(h^2) + eps)) fused into the ConvRot256
+// INT8 quantiser's staged load: codes Q [M, K] and row scales S of y, which
+// never reaches memory. *launched is false when the rows do not fit the
+// staging buffers (then nothing ran); Rout may alias X or R.
+cudaError_t launch_quant_norm_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                   const uint16_t *R, int64_t ldr, uint16_t *Rout, int64_t ldo,
+                                   const uint16_t *g, float eps, int8_t *Q, float *S,
+                                   unsigned *err, int num_sms, cudaStream_t stream,
+                                   bool *launched);
+
 // Test hook: the input activation of n bf16 values (n % 256 == 0) as the
 // staged quantiser applies it (0 none, 1 relu, 2 silu, 3 tanh-form gelu).
 cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,

@@ -759,6 +759,301 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     }
 }
 
+// ------------------------------------------------- input RMSNorm, fused
+// int8_linear with its input RMSNorm and residual (comfy-kitchen 0.2.40,
+// "Huawei Ascend backend"), the normalisation done inside the quantiser's
+// staged load so the normalised rows never reach HBM:
+//   h   = bf16_rne(x + r)  (h = x without a residual), written to Rout
+//   y_k = the bf16 value nearest to h_k g_k / sqrt(mean(h^2) + eps)
+//   then ConvRot256 and the per-row INT8 quantiser on y, as above.
+// The residual add is one bf16x2 add: for two bf16 values the rounding of the
+// exact sum equals the rounding of the fp32 sum (when the fp32 sum is inexact
+// the smaller operand is below 2^-16 of the larger, far under half a bf16
+// spacing, so both give the larger operand's neighbourhood the same way).
+// The sum of squares runs in double (each h^2 exact): a lane's 64 values in
+// order, the quad's four lanes by shuffles, then the row's quads in block
+// order through shared memory, so one row gives one result. inv = 1 /
+// sqrt(ss / K + eps) in double, inv32 its fp32 rounding. Fast path per value:
+// hg = h g in fp32 (exact while the product is a normal fp32 number: 8-bit
+// significands), then a = fl(hg fl(inv32 (1 - 2^-21))) and
+// b = fl(hg fl(inv32 (1 + 2^-21))): four roundings of 2^-24 each and inv's
+// own error (2^-24 + 2^-36) keep the exact value strictly between a and b.
+// Rounding is monotonic, so when a and b round to the same bf16 word, that
+// word is the exact value's rounding. A chunk of 8 values is redone in double
+// precision (h g exact in double, one product with inv, one rounding to bf16)
+// when some value's two words differ (it lies near a bf16 rounding midpoint)
+// or its smallest |a| is below T = 2^-125 max(1, inv32): a subnormal h g or a
+// shows up there (zeros included, which the double path gives exactly).
+// |h inv| <= sqrt(K), so with G = max |g| < 2^16 (the weight vector is staged
+// in shared memory when the CTA starts) no product overflows; weights of 2^16
+// or more send every value through the double path.
+constexpr float kNormLo = 0.99999952316284180f;  // 1 - 2^-21
+constexpr float kNormHi = 1.00000047683715820f;  // 1 + 2^-21
+
+struct NormArgs {
+    const uint16_t *R;   // residual rows or nullptr
+    int64_t ldr;
+    uint16_t *Rout;      // residual output or nullptr (may alias X or R)
+    int64_t ldo;
+    const uint16_t *g;   // weight [K] or nullptr
+    float eps;
+};
+
+// y of two values (h, g as bf16x2 words) in double precision.
+__device__ __forceinline__ uint32_t norm_bf16x2_exact(uint32_t hw, uint32_t gw, double inv) {
+    const double lo = double(__uint_as_float(hw << 16)) * double(__uint_as_float(gw << 16));
+    const double hi =
+        double(__uint_as_float(hw & 0xFFFF0000u)) * double(__uint_as_float(gw & 0xFFFF0000u));
+    const __nv_bfloat16 a = __double2bfloat16(lo * inv), b = __double2bfloat16(hi * inv);
+    return uint32_t(*reinterpret_cast<const uint16_t *>(&a)) |
+           (uint32_t(*reinterpret_cast<const uint16_t *>(&b)) << 16);
+}
+
+// The two bf16 halves of a word as doubles (exact).
+__device__ __forceinline__ void bf16x2_to_f64(uint32_t w, double &lo, double &hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f64.bf16 %0, l;\n\t"
+        "cvt.f64.bf16 %1, h;\n\t}"
+        : "=d"(lo), "=d"(hi)
+        : "r"(w));
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Persistent, staged like quant_rows_bulk_kernel: x rows in two buffers
+// (two groups ahead), the residual rows in one buffer refilled for the CTA's
+// next group as soon as the current group's rows are in registers, then the
+// weight vector. Two CTA barriers per group: one before the row's sum of
+// squares is read (after it the staging buffers may be refilled), one before
+// the row's absmax is read.
+template <bool kResidual>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
+                       int rows_per_cta, const NormArgs na, int8_t *__restrict__ Q,
+                       float *__restrict__ S, unsigned *err, uint64_t limit_ns) {
+    extern __shared__ __align__(128) uint8_t stage_raw[];
+    __shared__ unsigned s_amax[3][kMaxRowsPerCta];
+    __shared__ double s_ss[kMaxThreads / 4];
+    __shared__ __align__(8) uint64_t full[3];  // x buffers 0 and 1, the residual buffer
+    const int tid = threadIdx.x;
+    const int t = tid & 3;
+    const int quad = tid >> 2;
+    const int nb = K >> 8;
+    const int R = rows_per_cta;
+    const int row_local = quad / nb;
+    const int blk = quad - row_local * nb;
+    const int col0 = blk * kBlock + 8 * t;
+    const int sw5 = quad & 1;
+    const int64_t ngroups = (M + R - 1) / R;
+    const uint32_t row_bytes = uint32_t(K) * 2u;
+    const uint32_t buf0 = smem_u32(stage_raw);
+    const uint32_t buf_bytes = uint32_t(R) * row_bytes;
+    const uint32_t rbuf = buf0 + 2u * buf_bytes;  // residual rows (single buffer)
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        mbar_init(smem_u32(&full[2]), 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 3 * kMaxRowsPerCta; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
+    // the weight vector (1 without one) staged once after the two staging
+    // buffers, and G = max |g| (bf16 magnitude bits order like the values)
+    __shared__ unsigned s_gmax;
+    uint16_t *s_g = reinterpret_cast<uint16_t *>(stage_raw + (kResidual ? 3 : 2) * size_t(buf_bytes));
+    const uint32_t sg0 = smem_u32(s_g);
+    if (tid == 0) s_gmax = 0u;
+    __syncthreads();
+    {
+        unsigned gm = 0u;
+        for (int k = 8 * tid; k < K; k += 8 * blockDim.x) {
+            uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+            if (na.g) v = __ldg(reinterpret_cast<const uint4 *>(na.g + k));
+            *reinterpret_cast<uint4 *>(s_g + k) = v;
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                gm = max(gm, max(w[q] & 0x7FFFu, (w[q] >> 16) & 0x7FFFu));
+        }
+        if (gm) atomicMax(&s_gmax, gm);
+    }
+    __syncthreads();
+
+    // Thread 0: stage the rows of group g (x, or the residual when res) into
+    // the buffer at dst, completing on barrier `bar`.
+    auto issue = [&](int64_t g, bool res, uint32_t dst, uint32_t bar) {
+        const int64_t r0 = g * R;
+        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
+        const uint16_t *src = res ? na.R : X;
+        const int64_t ld = res ? na.ldr : ldx;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
+        for (int r = 0; r < n; ++r)
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(dst + uint32_t(r) * row_bytes),
+                "l"(reinterpret_cast<uint64_t>(src + (r0 + r) * ld)), "r"(row_bytes), "r"(bar)
+                : "memory");
+    };
+
+    const int64_t g0 = blockIdx.x;
+    const int64_t step = gridDim.x;
+    if (tid == 0) {
+        if (g0 < ngroups) {
+            issue(g0, false, buf0, smem_u32(&full[0]));
+            if (kResidual) issue(g0, true, rbuf, smem_u32(&full[2]));
+        }
+        if (g0 + step < ngroups) issue(g0 + step, false, buf0 + buf_bytes, smem_u32(&full[1]));
+    }
+    int slot = 0;
+    for (int i = 0; g0 + i * step < ngroups; ++i) {
+        const int64_t g = g0 + i * step;
+        const int b = i & 1;
+        bool ok = mbar_wait_bounded(smem_u32(&full[b]), uint32_t(i >> 1) & 1u, limit_ns, nullptr);
+        if (kResidual)
+            ok = ok && mbar_wait_bounded(smem_u32(&full[2]), uint32_t(i) & 1u, limit_ns, nullptr);
+        const int64_t row = g * R + row_local;
+        const bool active = ok && row_local < R && row < M;
+        const uint32_t rowoff = uint32_t(row_local) * row_bytes + uint32_t(col0) * 2u;
+        const uint32_t sx = buf0 + uint32_t(b) * buf_bytes + rowoff;
+        // h of this lane's 64 values (register group i = chunk i ^ sw5),
+        // stored as the residual output, and its sum of squares (one
+        // accumulator per chunk, combined in chunk order)
+        uint32_t hw[kPairs];
+        double acc[8];
+        if (active) {
+#pragma unroll
+            for (int i8 = 0; i8 < 8; ++i8)
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(hw[4 * i8]), "=r"(hw[4 * i8 + 1]), "=r"(hw[4 * i8 + 2]),
+                               "=r"(hw[4 * i8 + 3])
+                             : "r"(sx + 64u * uint32_t(i8 ^ sw5)));
+#pragma unroll
+            for (int i8 = 0; i8 < 8; ++i8) {
+                const int c = i8 ^ sw5;
+                if (kResidual) {
+                    uint32_t rw[4];
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(rw[0]), "=r"(rw[1]), "=r"(rw[2]), "=r"(rw[3])
+                                 : "r"(rbuf + rowoff + 64u * uint32_t(c)));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const __nv_bfloat162 s2 =
+                            __hadd2(*reinterpret_cast<const __nv_bfloat162 *>(&hw[4 * i8 + q]),
+                                    *reinterpret_cast<const __nv_bfloat162 *>(&rw[q]));
+                        hw[4 * i8 + q] = *reinterpret_cast<const uint32_t *>(&s2);
+                    }
+                }
+                if (na.Rout)
+                    *reinterpret_cast<uint4 *>(na.Rout + row * na.ldo + col0 + 32 * c) =
+                        make_uint4(hw[4 * i8], hw[4 * i8 + 1], hw[4 * i8 + 2], hw[4 * i8 + 3]);
+                double a = 0.0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    double lo, hi;
+                    bf16x2_to_f64(hw[4 * i8 + q], lo, hi);
+                    a = __fma_rn(lo, lo, a);
+                    a = __fma_rn(hi, hi, a);
+                }
+                acc[i8] = a;
+            }
+        } else {
+#pragma unroll
+            for (int i8 = 0; i8 < 8; ++i8) acc[i8] = 0.0;
+        }
+        const double ss0 = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
+        const double ss1 = __dadd_rn(__dadd_rn(acc[4], acc[5]), __dadd_rn(acc[6], acc[7]));
+        double ss = __dadd_rn(ss0, ss1);
+        ss = __dadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, 1));
+        ss = __dadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, 2));
+        if (active && t == 0) s_ss[quad] = ss;
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicMax(err, kDevErrTimeout);
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000ull) {
+            }
+            break;
+        }
+        // every thread has its values in registers: refill x buffer b two
+        // groups ahead and the residual buffer for the next group
+        if (tid == 0) {
+            if (g + 2 * step < ngroups) issue(g + 2 * step, false, buf0 + uint32_t(b) * buf_bytes,
+                                              smem_u32(&full[b]));
+            if (kResidual && g + step < ngroups) issue(g + step, true, rbuf, smem_u32(&full[2]));
+        }
+        const int clear = slot == 0 ? 2 : slot - 1;
+        if (tid < R) s_amax[clear][tid] = 0u;
+
+        float2 P[kPairs];
+        if (active) {
+            // the row's sum in block order, four chains
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+            const double *part = &s_ss[row_local * nb];
+            int q = 0;
+            for (; q + 4 <= nb; q += 4) {
+                s0 = __dadd_rn(s0, part[q]);
+                s1 = __dadd_rn(s1, part[q + 1]);
+                s2 = __dadd_rn(s2, part[q + 2]);
+                s3 = __dadd_rn(s3, part[q + 3]);
+            }
+            for (; q < nb; ++q) s0 = __dadd_rn(s0, part[q]);
+            const double ssr = __dadd_rn(__dadd_rn(s0, s1), __dadd_rn(s2, s3));
+            const double inv = rsqrt(ssr / double(K) + double(na.eps));
+            const float inv32 = __double2float_rn(inv);
+            const float ilo = __fmul_rn(inv32, kNormLo), ihi = __fmul_rn(inv32, kNormHi);
+            const float2 lo2 = make_float2(ilo, ilo), hi2 = make_float2(ihi, ihi);
+            // T, or +inf (every chunk redone) when G >= 2^16 or not finite
+            const float tiny = s_gmax < 0x4780u
+                                   ? fmaxf(1.0f, inv32) * 2.3509887016445750e-38f
+                                   : __uint_as_float(0x7F800000u);
+            // per chunk: the fast path for its 4 words, the chunk again in
+            // double when flagged, then the widening fused with h = 1
+#pragma unroll
+            for (int i8 = 0; i8 < 8; ++i8) {
+                uint32_t gw[4];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(gw[0]), "=r"(gw[1]), "=r"(gw[2]), "=r"(gw[3])
+                             : "r"(sg0 + 2u * uint32_t(col0 + 32 * (i8 ^ sw5))));
+                uint32_t yw[4];
+                uint32_t diff = 0u;
+                float amin = __uint_as_float(0x7F800000u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 hg = __fmul2_rn(widen_bf16x2(hw[4 * i8 + q]), widen_bf16x2(gw[q]));
+                    const float2 a = __fmul2_rn(hg, lo2), b = __fmul2_rn(hg, hi2);
+                    const __nv_bfloat162 ra = __floats2bfloat162_rn(a.x, a.y);
+                    const __nv_bfloat162 rb = __floats2bfloat162_rn(b.x, b.y);
+                    const uint32_t wa = *reinterpret_cast<const uint32_t *>(&ra);
+                    yw[q] = wa;
+                    diff |= wa ^ *reinterpret_cast<const uint32_t *>(&rb);
+                    amin = min3(amin, fabsf(a.x), fabsf(a.y));
+                }
+                if (diff != 0u || amin < tiny) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yw[q] = norm_bf16x2_exact(hw[4 * i8 + q], gw[q], inv);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) P[4 * i8 + q] = widen_stage1(yw[q]);
+            }
+        } else {
+            zero_block(P);
+        }
+        butterflies<true>(P, t, sw5);
+        const float m = block_absmax(P);
+        if (active && t == 0) atomicMax(&s_amax[slot][row_local], __float_as_uint(m));
+        __syncthreads();
+        if (active) {
+            const RowQuant rq = row_quant<true, 127>(__uint_as_float(s_amax[slot][row_local]));
+            if (blk == 0 && t == 0) S[row] = rq.s;
+            quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0, sw5);
+        }
+        slot = slot == 2 ? 0 : slot + 1;
+    }
+}
+
 // Two passes for long rows (K > 32768): one CTA per row, 128 quads; pass 1
 // rotates every block and reduces the absmax, pass 2 reloads (from L2),
 // rotates again and quantises.
@@ -1312,6 +1607,65 @@ cudaError_t launch_quant_rows_bf16(const uint16_t *X, int64_t M, int64_t K, int6
             return launch_bf16<true, kActGeluTanh>(X, M, K, ldx, Q, S, err, num_sms, stream);
         default: return launch_bf16<true, kActNone>(X, M, K, ldx, Q, S, err, num_sms, stream);
     }
+}
+
+template <bool kResidual>
+cudaError_t launch_norm_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                             const NormArgs &na, int8_t *Q, float *S, unsigned *err, int num_sms,
+                             cudaStream_t stream, bool *launched) {
+    *launched = false;
+    const int nb = static_cast<int>(K / kBlock);
+    // per row: two x buffers (+ one residual buffer); then the weight vector
+    const size_t per_row = 2 * size_t(K) * (kResidual ? 3 : 2);
+    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / per_row), kMaxRowsPerCta);
+    if (max_rows < 1 || 4 * nb > kMaxThreads) return cudaSuccess;
+    int threads = 0;
+    const int rows = pick_rows_per_cta(nb, 4, max_rows, kMaxThreads, 256, &threads);
+    const size_t smem = size_t(rows) * per_row + 2 * size_t(K);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_occ_mutex);
+        const auto key = std::make_tuple(dev, 1000 + (kResidual ? 1 : 0), threads, smem);
+        auto it = g_bulk_occupancy.find(key);
+        if (it != g_bulk_occupancy.end()) {
+            per_sm = it->second;
+        } else {
+            e = cudaFuncSetAttribute(quant_norm_bulk_kernel<kResidual>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(kBulkSmemBudget + 2 * 14336));
+            if (e != cudaSuccess) return e;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, quant_norm_bulk_kernel<kResidual>, threads, smem);
+            if (e != cudaSuccess) return e;
+            g_bulk_occupancy[key] = per_sm;
+        }
+    }
+    if (per_sm < 1) return cudaSuccess;
+    const int64_t groups = (M + rows - 1) / rows;
+    const int64_t cap = int64_t(per_sm) * num_sms;
+    const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
+    quant_norm_bulk_kernel<kResidual><<<grid, threads, smem, stream>>>(
+        X, M, static_cast<int>(K), ldx, rows, na, Q, S, err, kDefaultWaitLimitNs);
+    *launched = true;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_norm_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                   const uint16_t *R, int64_t ldr, uint16_t *Rout, int64_t ldo,
+                                   const uint16_t *g, float eps, int8_t *Q, float *S,
+                                   unsigned *err, int num_sms, cudaStream_t stream,
+                                   bool *launched) {
+    *launched = false;
+    if (M <= 0) {
+        *launched = true;
+        return cudaSuccess;
+    }
+    const NormArgs na{R, ldr, Rout, ldo, g, eps};
+    if (R) return launch_norm_bulk<true>(X, M, K, ldx, na, Q, S, err, num_sms, stream, launched);
+    return launch_norm_bulk<false>(X, M, K, ldx, na, Q, S, err, num_sms, stream, launched);
 }
 
 cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,

@@ -231,10 +231,16 @@ def lin_norm(X=FAKE, ldx=512, R=None, ldr=512, Ro=None, ldo=512, g=None, eps=1e-
 
 
 def test_norm_workspace_bytes():
+    # K <= CK_NORM_FUSED_MAX_K: the normalisation runs inside the quantiser,
+    # so only the codes and row scales need room; above it the normalised
+    # rows come first
+    assert ck.NORM_FUSED_MAX_K == 14336
     assert ck.norm_workspace_bytes(0, 256) == 0
-    assert ck.norm_workspace_bytes(3, 256) == 3 * 256 * 2 + 768 + 256
+    assert ck.norm_workspace_bytes(3, 256) == ck.workspace_bytes(3, 256) == 768 + 256
     M, K = 32700, 5376
-    assert ck.norm_workspace_bytes(M, K) == M * K * 2 + ck.workspace_bytes(M, K)
+    assert ck.norm_workspace_bytes(M, K) == ck.workspace_bytes(M, K)
+    assert ck.norm_workspace_bytes(5, 14336) == ck.workspace_bytes(5, 14336)
+    assert ck.norm_workspace_bytes(5, 14592) == 5 * 14592 * 2 + ck.workspace_bytes(5, 14592)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -248,9 +254,32 @@ def test_norm_workspace_bytes():
     (dict(g=MIS), ck.CK_ERR_MISALIGNED),
     (dict(Qw=MIS), ck.CK_ERR_MISALIGNED),
     (dict(ws=FAKE + 16), ck.CK_ERR_MISALIGNED),
-    (dict(ws_bytes=4096), ck.CK_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), ck.CK_ERR_WORKSPACE),
+    (dict(K=14592, ldx=14592, ldr=14592, ldo=14592, ws_bytes=4 * 14592 * 2), ck.CK_ERR_WORKSPACE),
     (dict(M=0), ck.CK_OK),
     (dict(N=0), ck.CK_OK),
 ])
 def test_int8_linear_norm_validation(kw, status):
     assert lin_norm(**kw) == status
+
+
+def quant_norm(X=FAKE, ldx=512, R=None, ldr=512, Ro=None, ldo=512, g=None, eps=1e-6, M=4, K=512,
+               Qx=FAKE, s_x=FAKE):
+    return ck.lib.ck_quantize_rotate_rowwise_norm(X, ldx, R, ldr, Ro, ldo, g, eps, M, K, Qx, s_x,
+                                                  None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(X=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(Qx=None), ck.CK_ERR_INVALID_VALUE),
+    (dict(eps=0.0), ck.CK_ERR_INVALID_VALUE),
+    (dict(M=-1), ck.CK_ERR_INVALID_VALUE),
+    (dict(K=300), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(K=14592, ldx=14592), ck.CK_ERR_UNSUPPORTED_SHAPE),
+    (dict(X=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(R=FAKE, ldr=516), ck.CK_ERR_MISALIGNED),
+    (dict(Qx=MIS), ck.CK_ERR_MISALIGNED),
+    (dict(M=0), ck.CK_OK),
+])
+def test_quantize_rotate_rowwise_norm_validation(kw, status):
+    assert quant_norm(**kw) == status
