@@ -311,53 +311,17 @@ def run_ours(args, cfg, rank, world, local_rank):
         X = X[lo:hi].contiguous()
     Xd = X.to(dev)
     bd = bias.to(dev)
-    if args.path == "w4a4":
-        Qw4, s_w = ck.rotate_quant_weight_int4(W.to(dev))
-        Qw = torch.empty((cfg.N, cfg.K), dtype=torch.int8, device=dev)
-    elif args.path == "nvfp4":
-        Qw, Sw, s_w = ck.rotate_quant_weight_nvfp4(W.to(dev))
-    else:
-        Qw, s_w = ck.rotate_quant_weight(W.to(dev))
     Wcpu = W
     M, N, K = X.shape[0], cfg.N, cfg.K
-    Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
-    s_x = torch.empty((M,), dtype=torch.float32, device=dev)
-    if args.path == "nvfp4":
-        Qx = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-        Sx = torch.empty((ck.nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
-        s_x = torch.empty((1,), dtype=torch.float32, device=dev)
-    if args.path == "norm":
-        R, w_norm = norm_inputs(cfg, cfg.M)
-        if args.scaling == "strong":
-            R = R[lo:hi].contiguous()
-        Rd, gd = R.to(dev), w_norm.to(dev)
-        Ro = torch.empty_like(Rd)  # the residual output (a separate buffer: steps stay equal)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     ck.clear_device_error()
-
-    def quantize():
-        # convrot_w4a4_linear: INT4 codes of X, then the packed weights unpacked
-        if args.path == "w4a4":
-            ck.quantize_rotate_rowwise_int4(Xd, Qx, s_x)
-            ck.unpack_int4(Qw4, out=Qw)
-        elif args.path == "nvfp4":
-            ck.quantize_rotate_nvfp4(Xd, Qx, Sx, s_x)
-        elif args.path == "norm":
-            # int8_linear's input RMSNorm and residual inside the quantiser
-            ck.quantize_rotate_rowwise_norm(Xd, Rd, gd, NORM_EPS, residual_out=Ro, Qx=Qx, s_x=s_x)
-        elif args.act == "none":
-            ck.quantize_rotate_rowwise(Xd, Qx, s_x)
-        else:
-            ck.quantize_rotate_rowwise_act(Xd, args.act, Qx, s_x)
-
-    def gemm():
-        if args.path == "nvfp4":
-            ck.nvfp4_gemm(Qx, Sx, s_x, Qw, Sw, s_w, bd, out=Y)
-        else:
-            ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+    rows = (lo, hi) if args.scaling == "strong" else None
+    pth = make_path(ck, args.path, args.act, cfg, Xd, W, bd, Y, dev, rows)
+    quantize, gemm = pth["quantize"], pth["gemm"]
+    Qw, s_w = pth["Qw"], pth["s_w"]
+    ws = torch.empty((ck.workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
 
     def step():
         quantize()
@@ -415,22 +379,146 @@ def run_ours(args, cfg, rank, world, local_rank):
         ms_e2e = float("nan")
     else:
         ms_e2e = run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev)
+    del pth, quantize, gemm, ws
+
+    # ---- the other paths of the same workload, briefly (one GPU, default path)
+    subpaths = None
+    if world == 1 and args.path == "int8" and args.act == "none" and not args.no_subpaths:
+        del Qw, s_w
+        subpaths = {}
+        for sp in ("norm", "w4a4", "nvfp4"):
+            sub = make_path(ck, sp, "none", cfg, Xd, W, bd, Y, dev, None)
+            for _ in range(3):
+                flush.zero_()
+                sub["quantize"]()
+                sub["gemm"]()
+            sq, sg, ss_ = time_steps(sub["quantize"], sub["gemm"], flush, SUBPATH_STEPS, stream)
+            del sub
+            torch.cuda.synchronize()
+            subpaths[sp] = path_record(sp, cfg, M, P, sq, sg, ss_)
+        if ck.device_error() != ck.CK_OK:
+            raise RuntimeError("device error while timing the other paths")
     return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
-                  clocks, t_wall0, t_wall1, spread, probe_tops, probe_clocks)
+                  clocks, t_wall0, t_wall1, spread, probe_tops, probe_clocks, subpaths)
 
 
-PROBE_MMAS = 200_000
+SUBPATH_STEPS = 10
+
+
+def make_path(ck, path, act, cfg, Xd, W, bd, Y, dev, rows):
+    """Device inputs and the two launches (quantiser, GEMM) of one path's step
+    on the workload: weights prepared offline first (rotated and quantised;
+    for w4a4 also unpacked once); `rows` = (lo, hi) keeps that row shard."""
+    import torch
+
+    M, N, K = Xd.shape[0], cfg.N, cfg.K
+    d = {}
+    if path == "w4a4":
+        # packed INT4 weights, unpacked to int8 codes once (offline, like the
+        # rotation and quantisation of the weights)
+        Qw4, s_w = ck.rotate_quant_weight_int4(W.to(dev))
+        Qw = ck.unpack_int4(Qw4)
+        del Qw4
+    elif path == "nvfp4":
+        Qw, Sw, s_w = ck.rotate_quant_weight_nvfp4(W.to(dev))
+    else:
+        Qw, s_w = ck.rotate_quant_weight(W.to(dev))
+    if path == "nvfp4":
+        Qx = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        Sx = torch.empty((ck.nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+        s_x = torch.empty((1,), dtype=torch.float32, device=dev)
+    else:
+        Qx = torch.empty((M, K), dtype=torch.int8, device=dev)
+        s_x = torch.empty((M,), dtype=torch.float32, device=dev)
+    if path == "norm":
+        R, w_norm = norm_inputs(cfg, cfg.M)
+        if rows is not None:
+            R = R[rows[0]:rows[1]].contiguous()
+        Rd, gd = R.to(dev), w_norm.to(dev)
+        Ro = torch.empty_like(Rd)  # the residual output (a separate buffer: steps stay equal)
+
+    def quantize():
+        if path == "w4a4":
+            # convrot_w4a4_linear on the unpacked weights: INT4 codes of X
+            ck.quantize_rotate_rowwise_int4(Xd, Qx, s_x)
+        elif path == "nvfp4":
+            ck.quantize_rotate_nvfp4(Xd, Qx, Sx, s_x)
+        elif path == "norm":
+            # int8_linear's input RMSNorm and residual inside the quantiser
+            ck.quantize_rotate_rowwise_norm(Xd, Rd, gd, NORM_EPS, residual_out=Ro, Qx=Qx, s_x=s_x)
+        elif act == "none":
+            ck.quantize_rotate_rowwise(Xd, Qx, s_x)
+        else:
+            ck.quantize_rotate_rowwise_act(Xd, act, Qx, s_x)
+
+    def gemm():
+        if path == "nvfp4":
+            ck.nvfp4_gemm(Qx, Sx, s_x, Qw, Sw, s_w, bd, out=Y)
+        else:
+            ck.int8_gemm_rowscale(Qx, s_x, Qw, s_w, bd, out=Y)
+
+    d.update(quantize=quantize, gemm=gemm, Qw=Qw, s_w=s_w)
+    return d
+
+
+def time_steps(quantize, gemm, flush, steps, stream):
+    """Per-step CUDA-event times (quantiser, GEMM, step) in ms, L2 flushed
+    between steps."""
+    import torch
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        quantize()
+        ev[i][1].record(stream)
+        gemm()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    return ([e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev],
+            [e[0].elapsed_time(e[2]) for e in ev])
+
+
+def path_bytes_and_peak(path, M, K, P):
+    """Algorithmic bytes of a path's quantiser launch, and its GEMM's peak."""
+    if path == "nvfp4":
+        # bf16 X read once (the absmax pass's re-read is not algorithmic),
+        # packed FP4 codes and one E4M3 scale per 16 values written
+        return 2.0 * M * K + 0.5 * M * K + M * K / 16.0 + 4.0, P["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    if path == "norm":
+        # X and the residual read, the residual output, codes and row scales
+        # written (the normalised rows never reach memory)
+        return 7.0 * M * K + 4.0 * M, P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    return 3.0 * M * K + 4.0 * M, P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+
+
+def path_record(path, cfg, M, P, q_ms, g_ms, s_ms):
+    n = len(s_ms)
+    ms_q, ms_g, ms_s = sum(q_ms) / n, sum(g_ms) / n, sum(s_ms) / n
+    ops = 2.0 * M * cfg.N * cfg.K
+    q_bytes, gpeak = path_bytes_and_peak(path, M, cfg.K, P)
+    return {"steps": n, "ms_per_step": ms_s, "tops": ops / (ms_s / 1e3) / 1e12,
+            "gemm": {"ms_per_launch": ms_g, "tops": ops / (ms_g / 1e3) / 1e12,
+                     "frac": ops / (ms_g / 1e3) / 1e12 / gpeak, "peak": gpeak},
+            "quantizer": {"ms_per_launch": ms_q, "bytes_per_launch": q_bytes,
+                          "gbs": q_bytes / (ms_q / 1e3) / 1e9,
+                          "frac": q_bytes / (ms_q / 1e3) / 1e9 / P["hbm_gbs"]},
+            "launches_per_step": 2}
+
+
+PROBE_MMAS = 50_000
 
 
 def i8_probe_tops(ck, stream):
     """The device's INT8 tensor-core ceiling (ck_test_i8_mma_peak: back-to-back
-    pair MMAs of the GEMM's shape, no memory traffic), best of three ~15 ms
-    launches after one warm-up, timed with events on the launching stream."""
+    pair MMAs of the GEMM's shape, no memory traffic), best of five ~4 ms
+    launches after one warm-up, timed with events on the launching stream
+    (short bursts: MMA-only load reaches the power cap within milliseconds)."""
     import torch
 
     ck.test_i8_mma_peak(PROBE_MMAS // 10, stream=stream)
     best = 0.0
-    for _ in range(3):
+    for _ in range(5):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -479,7 +567,7 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
 
 
 def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
-           t_wall0, t_wall1, spread=None, probe_tops=None, probe_clocks=None):
+           t_wall0, t_wall1, spread=None, probe_tops=None, probe_clocks=None, subpaths=None):
     # per-rank work: the full batch (weak, replicas) or this rank's row shard
     # (strong); the job's total is world x per-rank (weak) or the whole batch
     M, N, K = X.shape[0], cfg.N, cfg.K
@@ -488,20 +576,7 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
     value = job_ops / (ms_step / 1e3) / 1e12
     e2e_value = job_ops / (ms_e2e / 1e3) / 1e12
     gemm_tops = ops / (ms_g / 1e3) / 1e12
-    if args.path == "nvfp4":
-        # bf16 X read once (the second, absmax pass is not algorithmic), packed
-        # FP4 codes and one E4M3 scale per 16 values written
-        q_bytes = 2.0 * M * K + 0.5 * M * K + M * K / 16.0 + 4.0
-        int8_peak = P["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
-    elif args.path == "norm":
-        # the input RMSNorm inside the quantiser: X and the residual read, the
-        # residual output, the codes and the row scales written (the
-        # normalised rows never reach memory)
-        q_bytes = 7.0 * M * K + 4.0 * M
-        int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
-    else:
-        q_bytes = 3.0 * M * K + 4.0 * M
-        int8_peak = P["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    q_bytes, int8_peak = path_bytes_and_peak(args.path, M, K, P)
     q_gbs = q_bytes / (ms_q / 1e3) / 1e9
     ratio = NOMINAL_FP4_OVER_BF16 if args.path == "nvfp4" else NOMINAL_INT8_OVER_BF16
     sustained_peak = P["bf16_tflops_sustained"] * ratio
@@ -583,9 +658,18 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
                     "call": f"ck_int8_linear_host: X from and Y to pinned host memory, chunks of "
                             f"{min(E2E_CHUNK_ROWS, M)} rows with copies overlapped with the kernels"},
-            "gpu_launches": {"w4a4": 3, "nvfp4": 4}.get(args.path, 2) * args.steps,
+            "gpu_launches": {"nvfp4": 4}.get(args.path, 2) * args.steps,
             "clocks": clocks.summary(t_wall0, t_wall1),
         }
+        if subpaths:
+            line["other_paths"] = {
+                "note": f"the same workload's other paths, {SUBPATH_STEPS} steps each after 3 "
+                        "warm-up steps, timed with CUDA events after the main measurement: norm = "
+                        "int8_linear with its input RMSNorm and a residual fused into the "
+                        "quantiser; w4a4 = convrot_w4a4_linear (INT4 codes, weights unpacked "
+                        "once offline); nvfp4 = ConvRot NVFP4 (two-pass FP4 quantiser, "
+                        "block-scaled FP4 GEMM, GEMM peak = 4 x bf16)",
+                **subpaths}
     return line
 
 
@@ -647,13 +731,16 @@ def main(argv=None):
                          "batch's rows are split over the ranks")
     ap.add_argument("--path", default="int8", choices=["int8", "w4a4", "nvfp4", "norm"],
                     help="int8: int8_linear; w4a4: convrot_w4a4_linear (INT4 codes, packed "
-                         "INT4 weights unpacked per step); nvfp4: ConvRot NVFP4 (two-pass "
+                         "INT4 weights unpacked once, offline); nvfp4: ConvRot NVFP4 (two-pass "
                          "FP4 quantiser + block-scaled FP4 GEMM); norm: int8_linear with its "
                          "input RMSNorm and a residual (normalised inside the quantiser)")
     ap.add_argument("--act", default="none", choices=["none", "relu", "silu", "gelu_tanh"],
                     help="input activation folded into the quantiser (int8_linear(input_act=...))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-subpaths", action="store_true",
+                    help="skip the brief timing of the norm, w4a4 and nvfp4 paths that the "
+                         "default (int8) run adds to its line")
     ap.add_argument("--no-probe", action="store_true",
                     help="skip the INT8 tensor-core peak probe run after the timed region")
     ap.add_argument("--no-e2e", action="store_true",

@@ -352,6 +352,18 @@ ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Q
                                  int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                                  ck_stream_t stream);
 
+/* convrot_w4a4_linear on weights unpacked once, offline (ck_unpack_int4 of
+ * the packed codes: Qw [N, K] int8 in [-7, 7], 16-B aligned): the INT4
+ * quantiser into the workspace (ck_int8_linear_workspace_bytes(M, K) bytes,
+ * 256-B aligned: codes, then row scales) and the INT8 GEMM, with no unpack
+ * per call; results equal ck_convrot_w4a4_linear's. Static weights trade
+ * N * K / 2 more bytes of weight memory for the per-call unpack (1.5 N K
+ * bytes of traffic and a kernel). Other arguments as for ck_int8_linear. */
+ck_status ck_convrot_w4a4_linear_unpacked(const ck_bf16 *X, int64_t ldx, const int8_t *Qw,
+                                          const float *s_w, const ck_bf16 *bias, ck_bf16 *Y,
+                                          int64_t M, int64_t N, int64_t K, void *workspace,
+                                          size_t workspace_bytes, ck_stream_t stream);
+
 /*
  * The GEMM and fused epilogue alone, on activations already quantised (by
  * ck_quantize_rotate_rowwise):

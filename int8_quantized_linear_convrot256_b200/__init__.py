@@ -75,6 +75,8 @@ _SIGS = {
     "ck_convrot_w4a4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "ck_convrot_w4a4_linear": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                      ctypes.c_size_t, _vp]),
+    "ck_convrot_w4a4_linear_unpacked": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                              _vp, ctypes.c_size_t, _vp]),
     "ck_dequantize_int8": (_st, [_vp, _vp, _i64, _i64, _st, _st, _vp, _vp]),
     "ck_quantize_int8_tensorwise": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_int8_linear_noalloc": (_st, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
@@ -494,6 +496,38 @@ def convrot_w4a4_linear(X: torch.Tensor, Qw4: torch.Tensor, s_w: torch.Tensor,
                                       M, N, K, _ptr(workspace),
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "ck_convrot_w4a4_linear")
+    return out
+
+
+def convrot_w4a4_linear_unpacked(X: torch.Tensor, Qw: torch.Tensor, s_w: torch.Tensor,
+                                 bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                                 workspace: torch.Tensor | None = None,
+                                 stream=None) -> torch.Tensor:
+    """convrot_w4a4_linear on weights unpacked once offline (``unpack_int4``:
+    int8 codes in [-7, 7], [N, K]); no unpack per call."""
+    _need(X, "X", torch.bfloat16, 2)
+    _need(Qw, "Qw", torch.int8, 2)
+    _rows_contiguous(Qw, "Qw")
+    _need(s_w, "s_w", torch.float32, 1)
+    M, K = X.shape
+    N = Qw.shape[0]
+    if Qw.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch between X, Qw and s_w")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, 2)
+    _rows_contiguous(out, "out")
+    need = workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    ldx = X.stride(0) if M > 1 else max(K, X.stride(0))
+    _check(lib.ck_convrot_w4a4_linear_unpacked(_ptr(X), ldx, _ptr(Qw), _ptr(s_w), _ptr(bias),
+                                               _ptr(out), M, N, K, _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(),
+                                               _stream(stream)),
+           "ck_convrot_w4a4_linear_unpacked")
     return out
 
 

@@ -862,6 +862,26 @@ ck_status ck_convrot_w4a4_linear(const ck_bf16 *X, int64_t ldx, const uint8_t *Q
     return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
 }
 
+ck_status ck_convrot_w4a4_linear_unpacked(const ck_bf16 *X, int64_t ldx, const int8_t *Qw,
+                                          const float *s_w, const ck_bf16 *bias, ck_bf16 *Y,
+                                          int64_t M, int64_t N, int64_t K, void *workspace,
+                                          size_t workspace_bytes, ck_stream_t stream) {
+    ck_status s = ck::check_linear_args(X, ldx, Qw, s_w, bias, Y, M, N, K, workspace, true);
+    if (s != CK_OK || M == 0 || N == 0) return s;
+    if (workspace_bytes < ck_int8_linear_workspace_bytes(M, K)) return CK_ERR_WORKSPACE;
+    DeviceState *st = nullptr;
+    s = device_state(&st);
+    if (s != CK_OK) return s;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    int8_t *Qx = reinterpret_cast<int8_t *>(base);
+    float *s_x = reinterpret_cast<float *>(base + round256(size_t(M) * size_t(K)));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e =
+        ck::launch_quant_rows_bf16(X, M, K, ldx, true, CK_ACT_NONE, 7, Qx, s_x, st->err, st->num_sms, cs);
+    if (e != cudaSuccess) return CK_ERR_CUDA;
+    return run_gemm(Qx, s_x, Qw, s_w, bias, Y, nullptr, M, N, K, st, cs);
+}
+
 ck_status ck_int8_gemm_rowscale(const int8_t *Qx, const float *s_x, const int8_t *Qw,
                                 const float *s_w, const ck_bf16 *bias, ck_bf16 *Y, int64_t M,
                                 int64_t N, int64_t K, ck_stream_t stream) {

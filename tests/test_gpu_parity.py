@@ -413,6 +413,21 @@ def test_convrot_w4a4_linear_matches_oracle(ck, M, K, N):
     assert_bf16_close(to_np(Y), Yr)
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 256, 8), (300, 1024, 264), (129, 5376, 520)])
+def test_convrot_w4a4_linear_unpacked_weights(ck, M, K, N):
+    """The same linear on weights unpacked once: identical to the packed
+    entry point and to the oracle."""
+    cfg = workloads.custom(M, K, N, seed=M + 3 * K + N)
+    X, W, bias = workloads.make_inputs(cfg)
+    Qw4, s_w = ck.rotate_quant_weight_int4(dev(W))
+    Qw = ck.unpack_int4(Qw4)
+    r4, rs = oracle.rotate_quant_weight_int4(W.numpy())
+    Y = to_np(ck.convrot_w4a4_linear_unpacked(dev(X), Qw, s_w, dev(bias)))
+    assert np.array_equal(Y, to_np(ck.convrot_w4a4_linear(dev(X), Qw4, s_w, dev(bias))))
+    Yr = oracle.convrot_w4a4_linear(workloads.bf16_bits(X), r4, rs, workloads.bf16_bits(bias))[0]
+    assert_bf16_close(Y, Yr)
+
+
 @pytest.mark.slow
 def test_convrot_w4a4_linear_full_size_sampled_rows(ck):
     cfg = workloads.CONFIGS[1]  # ragged M8193/K5376/N16128
