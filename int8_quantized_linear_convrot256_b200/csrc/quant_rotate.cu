@@ -82,7 +82,8 @@ constexpr float kNearQuarter = 1.52587890625e-05f;   // 2^-16
 constexpr float kNearHalf = 0.4999847412109375f;     // 0.5 - 2^-16
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
 constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
-constexpr size_t kBulkSmemBudget = 112 * 1024;       // per-CTA staging budget (2 buffers)
+constexpr size_t kBulkSmemBudget = 112 * 1024;       // per-CTA staging budget (all buffers)
+constexpr int kBulkBufs = 2;                         // row groups staged per CTA of the INT8 quantiser (3 timed no faster)
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 // a - b with one rounding: b * (-1) is exact, then the sum is rounded once.
@@ -661,9 +662,9 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
 }
 
 // Persistent single pass for BF16 rows: row groups are staged into shared
-// memory with cp.async.bulk two groups ahead (2 buffers). One CTA barrier per
-// group: after it, every thread has read its values out of the buffer (so the
-// buffer can be refilled) and the row absmax is complete. The absmax slots are
+// memory with cp.async.bulk kBulkBufs groups ahead (one buffer each). One CTA
+// barrier per group: after it, every thread has read its values out of the
+// buffer (so the buffer can be refilled) and the row absmax is complete. The absmax slots are
 // triple-buffered so a slot is cleared one full barrier before its next use.
 template <bool kRotate, int kAct, int kQ>
 __global__ void __launch_bounds__(kMaxThreads, 1)
@@ -672,7 +673,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
                        unsigned *err, uint64_t limit_ns) {
     extern __shared__ __align__(128) uint8_t stage_raw[];
     __shared__ unsigned s_amax[3][kMaxRowsPerCta];
-    __shared__ __align__(8) uint64_t full[2];
+    __shared__ __align__(8) uint64_t full[kBulkBufs];
     const int tid = threadIdx.x;
     const int t = tid & 3;
     const int quad = tid >> 2;
@@ -688,8 +689,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     const uint32_t buf_bytes = uint32_t(R) * row_bytes;
 
     if (tid == 0) {
-        mbar_init(smem_u32(&full[0]), 1);
-        mbar_init(smem_u32(&full[1]), 1);
+        for (int j = 0; j < kBulkBufs; ++j) mbar_init(smem_u32(&full[j]), 1);
         fence_mbar_init();
     }
     for (int i = tid; i < 3 * kMaxRowsPerCta; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
@@ -714,16 +714,15 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
 
     const int64_t g0 = blockIdx.x;
     const int64_t step = gridDim.x;
-    if (tid == 0) {
-        if (g0 < ngroups) issue(g0, 0);
-        if (g0 + step < ngroups) issue(g0 + step, 1);
-    }
+    if (tid == 0)
+        for (int j = 0; j < kBulkBufs; ++j)
+            if (g0 + j * step < ngroups) issue(g0 + j * step, j);
     int slot = 0;  // i % 3
+    int b = 0;     // i % kBulkBufs
+    uint32_t par = 0;  // (i / kBulkBufs) & 1
     for (int i = 0; g0 + i * step < ngroups; ++i) {
         const int64_t g = g0 + i * step;
-        const int b = i & 1;
-        const bool ok = mbar_wait_bounded(smem_u32(&full[b]), uint32_t(i >> 1) & 1u, limit_ns,
-                                          nullptr);
+        const bool ok = mbar_wait_bounded(smem_u32(&full[b]), par, limit_ns, nullptr);
         const int64_t row = g * R + row_local;
         const bool active = ok && row_local < R && row < M;
         float2 P[kPairs];
@@ -746,8 +745,8 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
             }
             break;
         }
-        // Buffer b has been read by every thread: refill it two groups ahead.
-        if (tid == 0 && g + 2 * step < ngroups) issue(g + 2 * step, b);
+        // Buffer b has been read by every thread: refill it kBulkBufs groups ahead.
+        if (tid == 0 && g + kBulkBufs * step < ngroups) issue(g + kBulkBufs * step, b);
         const int clear = slot == 0 ? 2 : slot - 1;  // (i + 2) % 3
         if (tid < R) s_amax[clear][tid] = 0u;
         if (active) {
@@ -756,6 +755,10 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
             quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0, sw5);
         }
         slot = slot == 2 ? 0 : slot + 1;
+        if (++b == kBulkBufs) {
+            b = 0;
+            par ^= 1u;
+        }
     }
 }
 
@@ -1159,12 +1162,12 @@ cudaError_t launch_bulk(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, in
                         unsigned *err, int num_sms, cudaStream_t stream, bool *launched) {
     *launched = false;
     const int nb = static_cast<int>(K / kBlock);
-    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2)),
+    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / (kBulkBufs * size_t(K) * 2)),
                                   kMaxRowsPerCta);
     if (max_rows < 1 || 4 * nb > kMaxThreads) return cudaSuccess;
     int threads = 0;
     const int rows = pick_rows_per_cta(nb, 4, max_rows, kMaxThreads, 256, &threads);
-    const size_t smem = 2 * size_t(rows) * size_t(K) * 2;
+    const size_t smem = kBulkBufs * size_t(rows) * size_t(K) * 2;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
