@@ -107,20 +107,25 @@ __device__ __forceinline__ float2 widen_bf16x2(uint32_t w) {
 // before the rotation. relu; silu x / (1 + e^-x); gelu (tanh form)
 // 0.5 x (1 + tanh(u)) = x / (1 + e^(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3).
 //
-// Fast path, fp32: e^v by Cody-Waite reduction v = n ln2 + r (ln2 = 16-bit
-// head + tail) and a degree-7 Taylor polynomial of e^r (truncation below
-// 2^-27), a reciprocal approximation of the denominator and one product. Its
-// result q is within E fp32 ulps of the exact value, E = 4 for silu (its
-// exponent argument -x is exact) and E = 4 + 3.5 |v| for gelu (the fp32
-// rounding of v = -2u, a few ulps, is amplified by e^v when e^v is not
-// negligible against 1). The bf16 rounding of q is the exact value's unless
-// q lies within E ulps of a bf16 rounding midpoint (its low 16 bits near
-// 0x8000); those values (a window of W = 8 + 4 |v| ulps is flagged, |v| taken
-// as 0 where e^v < 2^-20), and denominators above 1e36, are redone in double
-// precision and rounded to bf16 from the double value directly. The double
+// Fast path, fp32: with v the exponent (-x, or -2u), e^v by Cody-Waite
+// reduction v = n ln2 + r (ln2 = 16-bit head + tail) and a degree-7 Taylor
+// polynomial of e^r (truncation below 2^-27), d = 1 + e, and the quotient
+// x rcp.approx(d): within 4 fp32 ulps of the exact value for silu (whose v is
+// exact) and within 4 + 3.5 |v| for gelu (the fp32 rounding of v, a few ulps,
+// amplified by e^v when it is not negligible against 1). The bf16 rounding of
+// the result is the exact value's unless it lies near a bf16 rounding
+// midpoint: values within W = 8 (silu) or 8 + 4 |v| (gelu) fp32 ulps of one,
+// and denominators above 1e36, are redone in double precision and rounded to
+// bf16 from the double value directly. (The hardware's ex2.approx timed
+// slower here: its error grows with |v|, and the wider windows it needs send
+// more values to the double path.) The double
 // result differs from the exact value by a few 2^-52 relative, far less than
 // its distance from any midpoint for every bf16 input (the whole input set,
 // 65,280 finite values, is checked against the CPU oracle).
+// Where v > 182 the exact value's magnitude is below |x| e^-182 < 2^-134,
+// half the smallest bf16 subnormal, for every bf16 x: the result is a zero
+// with the sign of x, taken without a redo (gelu; for silu that needs
+// x < -182, which goes to the double path).
 // For |x| < 2^-120 the double evaluation gives x/2 exactly, which can sit on
 // a midpoint between bf16 subnormals while the exact value lies just above
 // x/2; there x/2 is rounded with ties going up.
@@ -170,40 +175,24 @@ __device__ __forceinline__ float2 act_exp2(float2 x) {
 // x / d where only the bf16 rounding of the quotient is used: a reciprocal
 // approximation times x. `redo` is raised when the result lies within w fp32
 // ulps of a bf16 rounding midpoint, or d is huge (the reciprocal would leave
-// the normal range).
-__device__ __forceinline__ float div_for_bf16(float x, float d, uint32_t w, bool &redo) {
+// the normal range); `zero` gives x's signed zero instead (no redo).
+__device__ __forceinline__ float div_for_bf16(float x, float d, uint32_t w, bool zero, bool &redo) {
     float r;
     asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(d));
     const float q = __fmul_rn(x, r);
     const uint32_t lo = __float_as_uint(q) & 0xFFFFu;
+    if (zero) return __fmul_rn(x, 0.0f);
     redo = redo || (lo - (0x8000u - w) <= 2u * w) || (d > 1.0e36f);
     return q;
 }
 
-// Denominators 1 + e^v of silu (v = -x) and of the tanh-form gelu (v = -2u),
-// and the flag window of each value in fp32 ulps.
+// The flag window of one value in fp32 ulps: 8 for silu (its exponent -x is
+// exact); for gelu 8 + 4 |v|, the fp32 rounding of v = -2u amplified by e^v,
+// counted where e^v is not negligible against 1 (|v| <= 83 there).
 template <int kAct>
-__device__ __forceinline__ float2 act_denominator(float2 x, uint32_t &wx, uint32_t &wy) {
-    float2 v;
-    if (kAct == kActSilu) {
-        v = make_float2(-x.x, -x.y);
-    } else {
-        const float2 x3 = __fmul2_rn(__fmul2_rn(x, x), x);
-        const float2 inner = __ffma2_rn(make_float2(0.044715f, 0.044715f), x3, x);
-        const float2 u = __fmul2_rn(make_float2(7.978846e-01f, 7.978846e-01f), inner);
-        v = __fmul2_rn(make_float2(-2.0f, -2.0f), u);
-    }
-    const float2 e = act_exp2(v);
-    if (kAct == kActSilu) {
-        wx = wy = 8u;
-    } else {
-        // |v| <= 83 wherever e^v is in [2^-20, 1e36]; outside that the value
-        // is flagged anyway (d > 1e36) or the amplified error is negligible
-        const float kTiny = 9.5367431640625e-07f;  // 2^-20
-        wx = 8u + (e.x >= kTiny && e.x <= 1.0e36f ? uint32_t(4.0f * fabsf(v.x)) : 0u);
-        wy = 8u + (e.y >= kTiny && e.y <= 1.0e36f ? uint32_t(4.0f * fabsf(v.y)) : 0u);
-    }
-    return __fadd2_rn(make_float2(1.0f, 1.0f), e);
+__device__ __forceinline__ uint32_t act_window(float e, float v) {
+    if (kAct == kActSilu) return 8u;
+    return 8u + (e >= 9.5367431640625e-07f && e <= 1.0e36f ? uint32_t(4.0f * fabsf(v)) : 0u);
 }
 
 // bf16x2 word -> activation of both values -> bf16x2 word (round to nearest
@@ -217,9 +206,22 @@ __device__ __forceinline__ uint32_t act_bf16x2(uint32_t w, bool &redo) {
     if (kAct == kActRelu) {
         a = make_float2(x.x > 0.0f ? x.x : 0.0f, x.y > 0.0f ? x.y : 0.0f);
     } else {
-        uint32_t wx, wy;
-        const float2 d = act_denominator<kAct>(x, wx, wy);
-        a = make_float2(div_for_bf16(x.x, d.x, wx, redo), div_for_bf16(x.y, d.y, wy, redo));
+        float2 v;
+        if (kAct == kActSilu) {
+            v = make_float2(-x.x, -x.y);
+        } else {
+            const float2 x3 = __fmul2_rn(__fmul2_rn(x, x), x);
+            const float2 inner = __ffma2_rn(make_float2(0.044715f, 0.044715f), x3, x);
+            const float2 u = __fmul2_rn(make_float2(7.978846e-01f, 7.978846e-01f), inner);
+            v = __fmul2_rn(make_float2(-2.0f, -2.0f), u);
+        }
+        const float2 e = act_exp2(v);
+        const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), e);
+        // the signed-zero rule matters for gelu only (its v passes 182 below
+        // x = -13.1; silu's only below x = -182, left to the double path)
+        const bool gelu = kAct == kActGeluTanh;
+        a = make_float2(div_for_bf16(x.x, d.x, act_window<kAct>(e.x, v.x), gelu && v.x > 182.0f, redo),
+                        div_for_bf16(x.y, d.y, act_window<kAct>(e.y, v.y), gelu && v.y > 182.0f, redo));
     }
     const __nv_bfloat162 h = __floats2bfloat162_rn(a.x, a.y);
     return *reinterpret_cast<const uint32_t *>(&h);
