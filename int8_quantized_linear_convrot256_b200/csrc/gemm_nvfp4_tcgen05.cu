@@ -367,7 +367,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 // rows (its tensor core needs all of them). All loads are TMA loads whose
 // completion bytes go to the even CTA's barrier. The even CTA copies the
 // scale tiles into TMEM (tcgen05.cp.cta_group::2: each CTA's shared memory
-// into its own TMEM) and issues the MMAs. TMEM holds one 256-column fp32
+// into its own TMEM) from a warp of its own, as soon as a stage's loads have
+// landed, and signals each stage's copies on a barrier the MMA thread waits
+// for; the copies for the next stages are thereby already queued while a
+// stage's MMAs run. TMEM holds one 256-column fp32
 // accumulator plus the scale columns of the 5 stages, so there is no room
 // for a second accumulator. Instead 8 epilogue warps per CTA move the
 // accumulator into registers (128 columns each) and release it before doing
@@ -381,7 +384,8 @@ constexpr int kPairStageBytesN = 2 * kPairRowsN * BKB + kPairSfaBytes + kPairSfb
 constexpr int kPairStagesN = 5;
 constexpr uint32_t kPairSfCol0 = 256;
 constexpr uint32_t kPairSfColsPerStage = 48;  // 16 for A, 32 for B
-constexpr int kPairThreadsN = 320;            // producer, MMA, 8 epilogue warps
+constexpr int kPairThreadsN = 352;            // producer, MMA, 8 epilogue warps, scale copies
+constexpr int kPairCopyWarpN = 10;
 constexpr uint32_t kPairEpiWarpsN = 16;       // both CTAs
 constexpr int kPairGroupMN = 8;
 
@@ -391,6 +395,7 @@ static_assert(kPairStageBytesN % 1024 == 0, "stages keep the 1024-byte swizzle a
 struct PairControlN {
     uint64_t full[kPairStagesN];
     uint64_t empty[kPairStagesN];
+    uint64_t sf_ready[kPairStagesN];  // the stage's scale copies have completed (even CTA)
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
@@ -466,6 +471,7 @@ gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int s = 0; s < kPairStagesN; ++s) {
             mbar_init(smem_u32(&ctl->full[s]), 1);
             mbar_init(smem_u32(&ctl->empty[s]), 1);
+            mbar_init(smem_u32(&ctl->sf_ready[s]), 1);
         }
         mbar_init(smem_u32(&ctl->tmem_full), 1);
         mbar_init(smem_u32(&ctl->tmem_empty), kPairEpiWarpsN);
@@ -556,20 +562,15 @@ gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait_bounded(smem_u32(&ctl->sf_ready[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_src = smem_u32(smem + size_t(stage) * kPairStageBytesN);
-                    const uint32_t sfa_src = a_src + 2 * kPairRowsN * BKB;
-                    const uint32_t sfb_src = sfa_src + kPairSfaBytes;
                     const uint32_t tsfa =
                         tmem_base + kPairSfCol0 + uint32_t(stage) * kPairSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tmem_cp_sf_pair(tsfa + 4u * j, desc_sf(sfa_src + kSfTileBytes * j));
-                        tmem_cp_sf_pair(tsfb + 8u * j, desc_sf(sfb_src + kSfTileBytes * j));
-                        tmem_cp_sf_pair(tsfb + 8u * j + 4u,
-                                        desc_sf(sfb_src + 4 * kSfTileBytes + kSfTileBytes * j));
-                    }
                     const uint64_t adesc = desc_sw128(a_src);
                     const uint64_t bdesc = desc_sw128(a_src + kPairRowsN * BKB);
 #pragma unroll
@@ -591,6 +592,51 @@ gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             umma_commit_pair_mc(smem_u32(&ctl->drain), 0x1);
             if (!mbar_wait_bounded(smem_u32(&ctl->drain), 0u, limit, nullptr))
                 raise_timeout(abort, p.err);
+        }
+    } else if (warp == kPairCopyWarpN) {
+        // ------------------------------------------------ scale tiles to TMEM (leader)
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_parity = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+                for (int kb = 0; kb < nk; ++kb) {
+                    // the stage's loads have landed; the MMAs that last read its
+                    // scale columns completed before the stage was refilled
+                    if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_src =
+                        smem_u32(smem + size_t(stage) * kPairStageBytesN) + 2 * kPairRowsN * BKB;
+                    const uint32_t sfb_src = sfa_src + kPairSfaBytes;
+                    const uint32_t tsfa =
+                        tmem_base + kPairSfCol0 + uint32_t(stage) * kPairSfColsPerStage;
+                    const uint32_t tsfb = tsfa + 16u;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tmem_cp_sf_pair(tsfa + 4u * j, desc_sf(sfa_src + kSfTileBytes * j));
+                        tmem_cp_sf_pair(tsfb + 8u * j, desc_sf(sfb_src + kSfTileBytes * j));
+                        tmem_cp_sf_pair(tsfb + 8u * j + 4u,
+                                        desc_sf(sfb_src + 4 * kSfTileBytes + kSfTileBytes * j));
+                    }
+                    umma_commit_pair_mc(smem_u32(&ctl->sf_ready[stage]), 0x1);
+                    issued |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kPairStagesN) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            // every copy this thread issued completes before TMEM is freed
+            for (int s = 0; s < kPairStagesN; ++s)
+                if (issued & (1u << s))
+                    if (!mbar_wait_bounded(smem_u32(&ctl->sf_ready[s]), (last_parity >> s) & 1u,
+                                           limit, nullptr))
+                        raise_timeout(abort, p.err);
         }
     } else {
         // ------------------------------------------------ epilogue (warps 2-9, both CTAs)
