@@ -13,14 +13,16 @@
 // Design:
 //  * Persistent CTAs, one per SM, over 128 x 128 output tiles grouped by 16
 //    M-tiles. Warp 0 loads (one lane), warp 1 issues the MMAs and owns TMEM,
-//    warps 2-5 run the epilogue.
+//    warps 2-5 run the epilogue, warp 6 copies the scale tiles into TMEM.
 //  * 5-stage ring. A stage holds one K-block of 256 values: A and B as
 //    128 rows x 128 packed bytes (2-D TMA, 128-byte swizzle, zero fill past M
 //    and N), plus the four 512-byte scale tiles of A and of B that cover the
 //    block. The blocked layout keeps those tiles contiguous, so each is one
 //    2 KB bulk copy.
-//  * Before the block's MMAs, the MMA lane copies the scale tiles into TMEM
-//    (tcgen05.cp 32x128b.warpx4). A tile's 32 lines of 16 bytes land in TMEM
+//  * As soon as a stage's loads land, the copy warp's lane copies its scale
+//    tiles into TMEM (tcgen05.cp 32x128b.warpx4) and commits them to the
+//    stage's sf_ready barrier, which the MMA lane waits for; copies of later
+//    stages are thereby queued while a stage's MMAs run. A tile's 32 lines of 16 bytes land in TMEM
 //    lanes 0-31 and again in 32-63, 64-95 and 96-127, four columns wide.
 //    Row r then finds its four scales in lane r, column r / 32, which is
 //    where the MMA reads them.
@@ -56,7 +58,8 @@ constexpr int kAccBufs = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = uint32_t(kAccBufs * BN);
 constexpr uint32_t kSfColsPerStage = 32;  // 16 for A, then 16 for B
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // producer, MMA, 4 epilogue warps, scale copies
+constexpr int kCopyWarp = 6;
 constexpr int kEpilogueThreads = 128;
 constexpr int kGroupM = 16;
 constexpr int kMmaKBytes = 32;  // 64 FP4 values per tcgen05.mma
@@ -67,6 +70,7 @@ static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignm
 struct Control {
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t sf_ready[kStages];  // the stage's scale copies have completed
     uint64_t tmem_full[kAccBufs];
     uint64_t tmem_empty[kAccBufs];
     uint64_t drain;
@@ -160,6 +164,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&ctl->full[s]), 1);
             mbar_init(smem_u32(&ctl->empty[s]), 1);
+            mbar_init(smem_u32(&ctl->sf_ready[s]), 1);
         }
         for (int a = 0; a < kAccBufs; ++a) {
             mbar_init(smem_u32(&ctl->tmem_full[a]), 1);
@@ -245,17 +250,14 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait_bounded(smem_u32(&ctl->sf_ready[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_src = smem_u32(smem + size_t(stage) * kStageBytes);
-                    const uint32_t sfa_src = a_src + kABytes + kBBytes;
-                    const uint32_t sfb_src = sfa_src + kSfBytes;
                     const uint32_t tsfa = tmem_base + kSfCol0 + uint32_t(stage) * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tmem_cp_sf(tsfa + 4u * j, desc_sf(sfa_src + kSfTileBytes * j));
-                        tmem_cp_sf(tsfb + 4u * j, desc_sf(sfb_src + kSfTileBytes * j));
-                    }
                     const uint64_t adesc = desc_sw128(a_src);
                     const uint64_t bdesc = desc_sw128(a_src + kABytes);
 #pragma unroll
@@ -279,6 +281,48 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             umma_commit(smem_u32(&ctl->drain));
             if (!mbar_wait_bounded(smem_u32(&ctl->drain), 0u, limit, nullptr))
                 raise_timeout(abort, p.err);
+        }
+    } else if (warp == kCopyWarp) {
+        // ------------------------------------------------ scale tiles to TMEM
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_parity = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                for (int kb = 0; kb < nk; ++kb) {
+                    // the stage's loads have landed; the MMAs that last read its
+                    // scale columns completed before the stage was refilled
+                    if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), phase, limit, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_src =
+                        smem_u32(smem + size_t(stage) * kStageBytes) + kABytes + kBBytes;
+                    const uint32_t sfb_src = sfa_src + kSfBytes;
+                    const uint32_t tsfa = tmem_base + kSfCol0 + uint32_t(stage) * kSfColsPerStage;
+                    const uint32_t tsfb = tsfa + 16u;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tmem_cp_sf(tsfa + 4u * j, desc_sf(sfa_src + kSfTileBytes * j));
+                        tmem_cp_sf(tsfb + 4u * j, desc_sf(sfb_src + kSfTileBytes * j));
+                    }
+                    umma_commit(smem_u32(&ctl->sf_ready[stage]));
+                    issued |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) raise_timeout(abort, p.err);
+            // every copy this thread issued completes before TMEM is freed
+            for (int s = 0; s < kStages; ++s)
+                if (issued & (1u << s))
+                    if (!mbar_wait_bounded(smem_u32(&ctl->sf_ready[s]), (last_parity >> s) & 1u,
+                                           limit, nullptr))
+                        raise_timeout(abort, p.err);
         }
     } else {
         // ------------------------------------------------ epilogue (warps 2-5)
