@@ -643,8 +643,8 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                              "i8_probe_clocks": probe_clocks}
                             if probe_tops else {}),
                          "ms_per_launch": ms_g},
-            "quantizer": {"kernel": ("nvfp4_bulk_kernel<1> + <2> (ConvRot256 + NVFP4, two "
-                                     "staged passes over X)" if args.path == "nvfp4" else
+            "quantizer": {"kernel": ("nvfp4_warp_kernel<1> + <2> (ConvRot256 + NVFP4, two "
+                                     "passes over X, staging private to each warp)" if args.path == "nvfp4" else
                                      "quant_norm_bulk_kernel (input RMSNorm with residual "
                                      "fused into ConvRot256 + per-row INT8)"
                                      if args.path == "norm" else

@@ -1451,95 +1451,140 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
     }
 }
 
-// Staged, persistent variant of the two NVFP4 passes for bf16 rows (as
-// quant_rows_bulk_kernel: row groups arrive by cp.async.bulk into two
-// buffers, the next group landing while the current one is computed). No
-// row-wide reduction is needed, so the CTA barrier of a group comes right
-// after its values are in registers and the buffer is refilled at once.
-// kPass 1: absmax of the rotated tensor into *amax_bits; kPass 2: codes and
-// block scales (as nvfp4_quant_kernel).
+// Staged, persistent variant of the two NVFP4 passes for bf16 rows, with
+// staging private to each warp and no CTA barrier in the loop (the passes
+// need no reduction over a row, so warps never wait for one another; a CTA
+// barrier per row group, as the INT8 quantiser has, cost pass 2 more than
+// two stalled warps per issued instruction). The row-major sequence of
+// 256-blocks (block b = row nb + blk) is cut into units of 8 consecutive
+// blocks; warp gw of the grid takes units gw, gw + W, gw + 2W, ... (W warps
+// in the grid), and quad q of the warp takes block q of the unit. Each warp
+// stages its units in kNvWarpBufs 4 KB buffers of its own (one
+// cp.async.bulk per run of blocks within one row, completing on the
+// buffer's mbarrier) and refills a buffer as soon as its own lanes have read
+// it (__syncwarp). kPass 1: absmax of the rotated tensor into *amax_bits;
+// kPass 2: codes and block scales (as nvfp4_quant_kernel).
+constexpr int kNvWarpBufs = 3;
+constexpr int kNvUnitBlocks = 8;
+constexpr uint32_t kNvUnitBytes = kNvUnitBlocks * 512;
+constexpr int kNvWarpThreads = 256;
+constexpr int kNvWarpsPerCta = kNvWarpThreads / 32;
+
 template <int kPass>
-__global__ void __launch_bounds__(kMaxThreads, 1)
-nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx, int rows_per_cta,
+__global__ void __launch_bounds__(kNvWarpThreads, 2)
+nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
                   unsigned *amax_bits, uint8_t *__restrict__ Q, uint8_t *__restrict__ S,
                   unsigned *err, uint64_t limit_ns) {
     extern __shared__ __align__(128) uint8_t stage_raw[];
-    __shared__ unsigned s_max;
-    __shared__ __align__(8) uint64_t full[2];
-    const int tid = threadIdx.x;
-    const int t = tid & 3;
-    const int quad = tid >> 2;
+    __shared__ __align__(8) uint64_t full[kNvWarpsPerCta][kNvWarpBufs];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t = lane & 3;
+    const int qw = lane >> 2;
     const int nb = K >> 8;
-    const int R = rows_per_cta;
-    const int row_local = quad / nb;
-    const int blk = quad - row_local * nb;
-    const int col0 = blk * kBlock + 8 * t;
-    const int64_t ngroups = (M + R - 1) / R;
-    const uint32_t row_bytes = uint32_t(K) * 2u;
-    const uint32_t buf0 = smem_u32(stage_raw);
-    const uint32_t buf_bytes = uint32_t(R) * row_bytes;
     const int C = K >> 4;
+    const int64_t nblocks = M * nb;
+    const int64_t nunits = (nblocks + kNvUnitBlocks - 1) / kNvUnitBlocks;
+    const int64_t gw = int64_t(blockIdx.x) * kNvWarpsPerCta + warp;
+    const int64_t wstep = int64_t(gridDim.x) * kNvWarpsPerCta;
+    const uint32_t wbuf = smem_u32(stage_raw) + uint32_t(warp) * kNvWarpBufs * kNvUnitBytes;
 
-    if (tid == 0) {
-        mbar_init(smem_u32(&full[0]), 1);
-        mbar_init(smem_u32(&full[1]), 1);
+    if (lane == 0) {
+        for (int j = 0; j < kNvWarpBufs; ++j) mbar_init(smem_u32(&full[warp][j]), 1);
         fence_mbar_init();
-        s_max = 0u;
     }
     __syncthreads();
 
-    auto issue = [&](int64_t g, int b) {
-        const int64_t r0 = g * R;
-        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
-        const uint32_t bar = smem_u32(&full[b]);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
-        for (int r = 0; r < n; ++r) {
-            const uint16_t *src = X + (r0 + r) * ldx;
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                ::"r"(buf0 + uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes),
-                "l"(reinterpret_cast<uint64_t>(src)), "r"(row_bytes), "r"(bar)
-                : "memory");
+    // Blocks advance by 8 wstep per unit of this warp: (row, blk) of a
+    // unit's first block are kept incrementally (one division up front).
+    const int64_t ustep = int64_t(kNvUnitBlocks) * wstep;
+    const int64_t drow = ustep / nb;
+    const int dblk = int(ustep - drow * nb);
+    auto advance = [&](int64_t &row, int &blk) {
+        row += drow;
+        blk += dblk;
+        if (blk >= nb) {
+            blk -= nb;
+            ++row;
         }
     };
 
-    const int64_t g0 = blockIdx.x;
-    const int64_t step = gridDim.x;
-    if (tid == 0) {
-        if (g0 < ngroups) issue(g0, 0);
-        if (g0 + step < ngroups) issue(g0 + step, 1);
+    // Lane 0: stage unit u (first block at row, blk) into buffer b.
+    auto issue = [&](int64_t u, int64_t row, int blk, int b) {
+        const int64_t left = nblocks - u * kNvUnitBlocks;
+        const int n = int(left < kNvUnitBlocks ? left : kNvUnitBlocks);
+        const uint32_t bar = smem_u32(&full[warp][b]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, uint32_t(n) * 512u);
+        for (int i = 0; i < n;) {
+            const int run = min(n - i, nb - blk);
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(wbuf + uint32_t(b) * kNvUnitBytes + uint32_t(i) * 512u),
+                "l"(reinterpret_cast<uint64_t>(X + row * ldx + int64_t(blk) * kBlock)),
+                "r"(uint32_t(run) * 512u), "r"(bar)
+                : "memory");
+            i += run;
+            blk += run;
+            if (blk == nb) {
+                blk = 0;
+                ++row;
+            }
+        }
+    };
+
+    const int64_t b_first = gw * kNvUnitBlocks;
+    int64_t row0 = b_first / nb;  // first block of this warp's current unit
+    int blk0 = int(b_first - row0 * nb);
+    int64_t irow = row0;           // first block of the next unit to stage
+    int iblk = blk0;
+    if (lane == 0) {
+        for (int j = 0; j < kNvWarpBufs; ++j) {
+            if (gw + j * wstep < nunits) issue(gw + j * wstep, irow, iblk, j);
+            advance(irow, iblk);
+        }
     }
     float s_t = 0.0f;
     if (kPass == 2) s_t = __fdiv_rn(__fmul_rn(__uint_as_float(*amax_bits), 0.0625f), 2688.0f);
     const float c6 = nvfp4_scale_rcp(s_t);
     float local_max = 0.0f;
-    for (int i = 0; g0 + i * step < ngroups; ++i) {
-        const int64_t g = g0 + i * step;
-        const int b = i & 1;
-        const bool ok = mbar_wait_bounded(smem_u32(&full[b]), uint32_t(i >> 1) & 1u, limit_ns,
-                                          nullptr);
-        const int64_t row = g * R + row_local;
-        const bool active = ok && row_local < R && row < M;
-        float2 P[kPairs];
-        const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
-                            uint32_t(col0) * 2u;
-        if (active)
-            load_block_smem<true>(sa, 0, P);
-        else
-            zero_block(P);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) atomicMax(err, kDevErrTimeout);
+    int b = 0;
+    uint32_t par = 0;
+    for (int64_t u = gw; u < nunits; u += wstep) {
+        const bool ok = mbar_wait_bounded(smem_u32(&full[warp][b]), par, limit_ns, nullptr);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+            if (lane == 0) atomicMax(err, kDevErrTimeout);
+            // let a late copy land before the CTA's shared memory is released
             const uint64_t t0 = globaltimer_ns();
             while (globaltimer_ns() - t0 < 200000ull) {
             }
             break;
         }
-        if (tid == 0 && g + 2 * step < ngroups) issue(g + 2 * step, b);
+        // this quad's block: qw blocks past the unit's first
+        int64_t row = row0;
+        int blk = blk0 + qw;
+        while (blk >= nb) {
+            blk -= nb;
+            ++row;
+        }
+        const bool active = u * kNvUnitBlocks + qw < nblocks;
+        float2 P[kPairs];
+        if (active)
+            load_block_smem<true>(wbuf + uint32_t(b) * kNvUnitBytes + uint32_t(qw) * 512u +
+                                      16u * uint32_t(t),
+                                  0, P);
+        else
+            zero_block(P);
+        __syncwarp();
+        if (lane == 0 && u + kNvWarpBufs * wstep < nunits)
+            issue(u + kNvWarpBufs * wstep, irow, iblk, b);
+        if (lane == 0) advance(irow, iblk);
+        advance(row0, blk0);
         butterflies<true>(P, t);
         if constexpr (kPass == 1) {
             local_max = fmaxf(local_max, block_absmax(P));
         } else {
+            const int col0 = blk * kBlock + 8 * t;
 #pragma unroll
             for (int c = 0; c < 8; c += 2) {
                 uint32_t bsc;
@@ -1553,12 +1598,16 @@ nvfp4_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
                 }
             }
         }
+        if (++b == kNvWarpBufs) {
+            b = 0;
+            par ^= 1u;
+        }
     }
     if (kPass == 1) {
-        // the quads' maxima are equal within a quad; one atomic per quad
-        if (t == 0 && local_max > 0.0f) atomicMax(&s_max, __float_as_uint(local_max));
-        __syncthreads();
-        if (tid == 0 && s_max != 0u) atomicMax(amax_bits, s_max);
+        float m = local_max;
+#pragma unroll
+        for (int l = 1; l < 32; l <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, l));
+        if (lane == 0 && m > 0.0f) atomicMax(amax_bits, __float_as_uint(m));
     }
 }
 
@@ -1729,61 +1778,47 @@ cudaError_t launch_nvfp4_impl(const TIn *X, int64_t M, int64_t K, int64_t ldx, u
     return cudaGetLastError();
 }
 
-std::map<std::tuple<int, int, int, size_t>, int> g_nvfp4_bulk_occupancy;
-
-template <int kPass>
-cudaError_t nvfp4_bulk_blocks_per_sm(int dev, int threads, size_t smem, int *out) {
-    std::lock_guard<std::mutex> lock(g_occ_mutex);
-    const auto key = std::make_tuple(dev, kPass, threads, smem);
-    auto it = g_nvfp4_bulk_occupancy.find(key);
-    if (it != g_nvfp4_bulk_occupancy.end()) {
-        *out = it->second;
-        return cudaSuccess;
-    }
-    cudaError_t e = cudaFuncSetAttribute(nvfp4_bulk_kernel<kPass>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(kBulkSmemBudget));
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_bulk_kernel<kPass>, threads,
-                                                      smem);
-    if (e != cudaSuccess) return e;
-    g_nvfp4_bulk_occupancy[key] = per_sm;
-    *out = per_sm;
-    return cudaSuccess;
-}
-
 cudaError_t launch_quant_nvfp4_bf16(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     uint8_t *Q, uint8_t *S, size_t s_bytes, float *s_t,
                                     unsigned *err, int num_sms, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
-    const int nb = static_cast<int>(K / kBlock);
-    const int max_rows = std::min(static_cast<int>(kBulkSmemBudget / (2 * size_t(K) * 2)),
-                                  kMaxRowsPerCta);
-    if (max_rows < 1 || 4 * nb > kMaxThreads)
-        return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
-    int threads = 0;
-    const int rows = pick_rows_per_cta(nb, 4, max_rows, kMaxThreads, 256, &threads);
-    const size_t smem = 2 * size_t(rows) * size_t(K) * 2;
+    const size_t smem = size_t(kNvWarpsPerCta) * kNvWarpBufs * kNvUnitBytes;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    int per_sm1 = 0, per_sm2 = 0;
-    if ((e = nvfp4_bulk_blocks_per_sm<1>(dev, threads, smem, &per_sm1)) != cudaSuccess) return e;
-    if ((e = nvfp4_bulk_blocks_per_sm<2>(dev, threads, smem, &per_sm2)) != cudaSuccess) return e;
-    if (per_sm1 < 1 || per_sm2 < 1)
-        return launch_nvfp4_impl(X, M, K, ldx, Q, S, s_bytes, s_t, stream);
-    const int64_t groups = (M + rows - 1) / rows;
-    const unsigned grid1 = unsigned(std::min<int64_t>(groups, int64_t(per_sm1) * num_sms));
-    const unsigned grid2 = unsigned(std::min<int64_t>(groups, int64_t(per_sm2) * num_sms));
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_occ_mutex);
+        const auto key = std::make_tuple(dev, 3000, kNvWarpThreads, smem);
+        auto it = g_bulk_occupancy.find(key);
+        if (it != g_bulk_occupancy.end()) {
+            per_sm = it->second;
+        } else {
+            for (auto *fn : {nvfp4_warp_kernel<1>, nvfp4_warp_kernel<2>}) {
+                e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+                if (e != cudaSuccess) return e;
+            }
+            int p1 = 0, p2 = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p1, nvfp4_warp_kernel<1>, kNvWarpThreads, smem);
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p2, nvfp4_warp_kernel<2>, kNvWarpThreads, smem);
+            if (e != cudaSuccess) return e;
+            per_sm = std::min(p1, p2);
+            g_bulk_occupancy[key] = per_sm;
+        }
+    }
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t units = (M * (K / kBlock) + kNvUnitBlocks - 1) / kNvUnitBlocks;
+    const int64_t ctas = (units + kNvWarpsPerCta - 1) / kNvWarpsPerCta;
+    const unsigned grid = unsigned(std::min<int64_t>(ctas, int64_t(per_sm) * num_sms));
     e = cudaMemsetAsync(s_t, 0, sizeof(float), stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(S, 0, s_bytes, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(S, 0, s_bytes, stream);  // the layout's padding
     if (e != cudaSuccess) return e;
     unsigned *amax = reinterpret_cast<unsigned *>(s_t);
-    nvfp4_bulk_kernel<1><<<grid1, threads, smem, stream>>>(X, M, static_cast<int>(K), ldx, rows,
-                                                         amax, Q, S, err, kDefaultWaitLimitNs);
-    nvfp4_bulk_kernel<2><<<grid2, threads, smem, stream>>>(X, M, static_cast<int>(K), ldx, rows,
-                                                         amax, Q, S, err, kDefaultWaitLimitNs);
+    nvfp4_warp_kernel<1><<<grid, kNvWarpThreads, smem, stream>>>(
+        X, M, static_cast<int>(K), ldx, amax, Q, S, err, kDefaultWaitLimitNs);
+    nvfp4_warp_kernel<2><<<grid, kNvWarpThreads, smem, stream>>>(
+        X, M, static_cast<int>(K), ldx, amax, Q, S, err, kDefaultWaitLimitNs);
     nvfp4_scale_kernel<<<1, 1, 0, stream>>>(s_t);
     return cudaGetLastError();
 }
