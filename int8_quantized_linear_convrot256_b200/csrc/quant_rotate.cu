@@ -1481,6 +1481,7 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
     const int lane = threadIdx.x & 31;
     const int t = lane & 3;
     const int qw = lane >> 2;
+    const int sw5 = qw & 1;  // chunk swizzle of this quad (see load_block_smem)
     const int nb = K >> 8;
     const int C = K >> 4;
     const int64_t nblocks = M * nb;
@@ -1572,7 +1573,7 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
         if (active)
             load_block_smem<true>(wbuf + uint32_t(b) * kNvUnitBytes + uint32_t(qw) * 512u +
                                       16u * uint32_t(t),
-                                  0, P);
+                                  sw5, P);
         else
             zero_block(P);
         __syncwarp();
@@ -1580,21 +1581,23 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
             issue(u + kNvWarpBufs * wstep, irow, iblk, b);
         if (lane == 0) advance(irow, iblk);
         advance(row0, blk0);
-        butterflies<true>(P, t);
+        butterflies<true>(P, t, sw5);
         if constexpr (kPass == 1) {
             local_max = fmaxf(local_max, block_absmax(P));
         } else {
+            // register group i holds chunk i ^ sw5: elements col0 + 32 (i ^ sw5) .. + 7
             const int col0 = blk * kBlock + 8 * t;
+            uint8_t *qr = Q + row * int64_t(K / 2);
 #pragma unroll
             for (int c = 0; c < 8; c += 2) {
                 uint32_t bsc;
                 const uint2 packed = nvfp4_codes_pair(P, c, t, s_t, c6, &bsc);
                 if (active) {
-                    const int e0 = col0 + 32 * c;
-                    uint8_t *qr = Q + row * int64_t(K / 2);
-                    *reinterpret_cast<uint32_t *>(qr + e0 / 2) = packed.x;
-                    *reinterpret_cast<uint32_t *>(qr + (e0 + 32) / 2) = packed.y;
-                    S[nvfp4_sf_offset(row, (e0 + 32 * (t & 1)) >> 4, C)] = uint8_t(bsc);
+                    const int ea = col0 + 32 * (c + sw5);      // group c
+                    const int eb = col0 + 32 * (c + 1 - sw5);  // group c + 1
+                    *reinterpret_cast<uint32_t *>(qr + ea / 2) = packed.x;
+                    *reinterpret_cast<uint32_t *>(qr + eb / 2) = packed.y;
+                    S[nvfp4_sf_offset(row, ((t & 1) ? eb : ea) >> 4, C)] = uint8_t(bsc);
                 }
             }
         }
