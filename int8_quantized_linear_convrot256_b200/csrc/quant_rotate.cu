@@ -299,11 +299,70 @@ __device__ __forceinline__ float2 widen_stage1(uint32_t w) {
         : "=f"(s), "=f"(d) : "r"(w), "f"(c));
     return make_float2(s, d);
 }
+// silu and tanh-form gelu through a table of exact results. Every bf16 input
+// with |x| in [2^-9, 2^7) has its own entry, (|h| - 0x3B00) + 2048 sign for
+// the bits h, filled by each CTA from act_bf16x2 (fast path with the
+// double-precision redo, the same results bit for bit). Outside the table:
+//  * |x| >= 2^7: x when x > 0, -0 when x < 0. The exact value differs from
+//    those by x e^-x / (1 + e^-x) (silu; gelu's term is smaller still), far
+//    below half a bf16 spacing of x, or is below 2^-134 in magnitude.
+//  * 2^-125 <= |x| < 2^-9, and x = +-0: x / 2 (exact: x / 2 is a normal bf16
+//    value). act(x) = x / 2 + c x^2 + O(x^3) with c = 1/4 (silu) or
+//    sqrt(2/pi) / 2 (gelu), so the difference is below half a spacing of
+//    x / 2 on either side for |x| < 2^-8.67.
+//  * 0 < |x| < 2^-125 (where x / 2 leaves bf16's normal range), infinities
+//    and NaN: `rare` is raised and the caller takes act_bf16x2_exact.
+// Every bf16 input is checked against the CPU oracle through the test hook,
+// which uses this same function.
+constexpr uint32_t kActTabLo = 0x3B00u;  // 2^-9
+constexpr int kActTabWords = 2048;       // 4096 entries of 16 bits
+
+template <int kAct>
+__device__ __forceinline__ void act_table_fill(uint32_t *tab, int tid, int nthreads) {
+    for (int i = tid; i < kActTabWords; i += nthreads) {
+        const uint32_t e = 2u * uint32_t(i);  // entries e, e + 1: same sign
+        const uint32_t h = ((e & 0x800u) << 4) | (kActTabLo + (e & 0x7FFu));
+        tab[i] = act_bf16x2<kAct>(h | ((h + 1u) << 16));
+    }
+}
+
+__device__ __forceinline__ __nv_bfloat162 bf162_bits(uint32_t w) {
+    return *reinterpret_cast<const __nv_bfloat162 *>(&w);
+}
+__device__ __forceinline__ uint32_t bits_bf162(__nv_bfloat162 v) {
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Index of value h's entry (its low 11 bits of |h| - 0x3B00, so every input
+// gives an index inside the table; only the window's are used).
+__device__ __forceinline__ uint32_t act_tab_index(uint32_t h) {
+    return (((h & 0x7FFFu) - kActTabLo) & 0x7FFu) | ((h >> 4) & 0x800u);
+}
+
+template <int kAct>
+__device__ __forceinline__ uint32_t act_word_tab(uint32_t w, const uint16_t *tab, bool &rare) {
+    const uint32_t a2 = w & 0x7FFF7FFFu;
+    const __nv_bfloat162 wb = bf162_bits(w);
+    const __nv_bfloat162 ab = bf162_bits(a2);
+    const uint32_t small = __hlt2_mask(ab, bf162_bits(0x3B003B00u));  // |x| < 2^-9
+    const uint32_t inside = ~small & __hlt2_mask(ab, bf162_bits(0x43004300u));  // < 2^7
+    const uint32_t half = bits_bf162(__hmul2(wb, bf162_bits(0x3F003F00u)));   // x * 0.5
+    const uint32_t big = bits_bf162(__hmax2(wb, bf162_bits(0x80008000u)));    // max(x, -0)
+    const uint32_t lo = tab[act_tab_index(w & 0xFFFFu)];
+    const uint32_t hi = tab[act_tab_index(w >> 16)];
+    const uint32_t t2 = lo | (hi << 16);
+    const uint32_t rule = (half & small) | (big & ~small);
+    const uint32_t tiny = __hlt2_mask(ab, bf162_bits(0x01000100u)) & ~__heq2_mask(ab, bf162_bits(0u));
+    const uint32_t finite = __hlt2_mask(ab, bf162_bits(0x7F807F80u));
+    rare = rare || ((tiny | ~finite) != 0u);
+    return (t2 & inside) | (rule & ~inside);
+}
+
 // Applies the input activation in place to this lane's 64 staged bf16 values
 // (8 chunks of 16 bytes at saddr + 64 i, read and written only by this lane).
 // A rolled loop keeps one copy of the activation code in the kernel.
 template <int kAct>
-__device__ __forceinline__ void act_in_smem(uint32_t saddr) {
+__device__ __forceinline__ void act_in_smem(uint32_t saddr, const uint16_t *tab) {
 #pragma unroll 1
     for (int i = 0; i < 8; ++i) {
         uint32_t x, y, z, w;
@@ -312,10 +371,18 @@ __device__ __forceinline__ void act_in_smem(uint32_t saddr) {
                      : "r"(saddr + 64u * i));
         // one flag per word: only a flagged word is redone
         bool ex = false, ey = false, ez = false, ew = false;
-        uint32_t ax = act_bf16x2<kAct>(x, ex);
-        uint32_t ay = act_bf16x2<kAct>(y, ey);
-        uint32_t az = act_bf16x2<kAct>(z, ez);
-        uint32_t aw = act_bf16x2<kAct>(w, ew);
+        uint32_t ax, ay, az, aw;
+        if (kAct != kActSilu && kAct != kActGeluTanh) {
+            ax = act_bf16x2<kAct>(x, ex);
+            ay = act_bf16x2<kAct>(y, ey);
+            az = act_bf16x2<kAct>(z, ez);
+            aw = act_bf16x2<kAct>(w, ew);
+        } else {
+            ax = act_word_tab<kAct>(x, tab, ex);
+            ay = act_word_tab<kAct>(y, tab, ey);
+            az = act_word_tab<kAct>(z, tab, ez);
+            aw = act_word_tab<kAct>(w, tab, ew);
+        }
         if (ex | ey | ez | ew) {
             if (ex) ax = act_bf16x2_exact<kAct>(x);
             if (ey) ay = act_bf16x2_exact<kAct>(y);
@@ -335,13 +402,16 @@ template <int kAct>
 __global__ void __launch_bounds__(128)
 input_act_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Y, int64_t n16) {
     __shared__ __align__(16) uint4 buf[1024];
+    __shared__ uint32_t tab[kAct == kActSilu || kAct == kActGeluTanh ? kActTabWords : 1];
     const int t = threadIdx.x;
     const int64_t base = int64_t(blockIdx.x) * 1024;
+    if (kAct == kActSilu || kAct == kActGeluTanh) act_table_fill<kAct>(tab, t, 128);
     for (int i = t; i < 1024; i += 128)
         buf[i] = base + i < n16 ? X[base + i] : make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
     // lane l of quad q: chunks 32 q + l + 4 i (i = 0..7), 64 bytes apart
-    act_in_smem<kAct>(smem_u32(&buf[32 * (t >> 2) + (t & 3)]));
+    act_in_smem<kAct>(smem_u32(&buf[32 * (t >> 2) + (t & 3)]),
+                      reinterpret_cast<const uint16_t *>(tab));
     __syncthreads();
     for (int i = t; i < 1024; i += 128)
         if (base + i < n16) Y[base + i] = buf[i];
@@ -676,6 +746,8 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     extern __shared__ __align__(128) uint8_t stage_raw[];
     __shared__ unsigned s_amax[3][kMaxRowsPerCta];
     __shared__ __align__(8) uint64_t full[kBulkBufs];
+    constexpr bool kTab = kAct == kActSilu || kAct == kActGeluTanh;
+    __shared__ uint32_t act_tab[kTab ? kActTabWords : 1];
     const int tid = threadIdx.x;
     const int t = tid & 3;
     const int quad = tid >> 2;
@@ -685,6 +757,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     const int blk = quad - row_local * nb;
     const int col0 = blk * kBlock + 8 * t;
     const int sw5 = quad & 1;  // chunk swizzle of this lane (see load_block_smem)
+    if (kTab) act_table_fill<kAct>(act_tab, tid, blockDim.x);
     const int64_t ngroups = (M + R - 1) / R;
     const uint32_t row_bytes = uint32_t(K) * 2u;
     const uint32_t buf0 = smem_u32(stage_raw);
@@ -731,7 +804,7 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
                             uint32_t(col0) * 2u;
         if (active) {
-            if (kAct != kActNone) act_in_smem<kAct>(sa);
+            if (kAct != kActNone) act_in_smem<kAct>(sa, reinterpret_cast<const uint16_t *>(act_tab));
             load_block_smem<kRotate>(sa, sw5, P);
         } else {
             zero_block(P);
