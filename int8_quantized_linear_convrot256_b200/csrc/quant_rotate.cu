@@ -358,46 +358,45 @@ __device__ __forceinline__ uint32_t act_word_tab(uint32_t w, const uint16_t *tab
     return (t2 & inside) | (rule & ~inside);
 }
 
-// Applies the input activation in place to this lane's 64 staged bf16 values
-// (8 chunks of 16 bytes at saddr + 64 i, read and written only by this lane).
-// A rolled loop keeps one copy of the activation code in the kernel.
+// The input activation of one 16-byte chunk (4 words, 8 values): relu
+// computed, silu and tanh-form gelu from the table; a word holding a value
+// outside the table's reach is redone by act_bf16x2_exact.
+template <int kAct>
+__device__ __forceinline__ void act_chunk(const uint32_t (&w)[4], uint32_t (&a)[4],
+                                          const uint16_t *tab) {
+    bool rare[4] = {false, false, false, false};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        a[q] = (kAct == kActSilu || kAct == kActGeluTanh) ? act_word_tab<kAct>(w[q], tab, rare[q])
+                                                          : act_bf16x2<kAct>(w[q], rare[q]);
+    if (rare[0] | rare[1] | rare[2] | rare[3]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (rare[q]) a[q] = act_bf16x2_exact<kAct>(w[q]);
+    }
+}
+
+// Applies the input activation in place to a lane's 64 bf16 values in
+// shared memory (8 chunks of 16 bytes at saddr + 64 i), chunk by chunk with
+// act_chunk, the function the staged quantiser applies to each loaded chunk.
 template <int kAct>
 __device__ __forceinline__ void act_in_smem(uint32_t saddr, const uint16_t *tab) {
 #pragma unroll 1
     for (int i = 0; i < 8; ++i) {
-        uint32_t x, y, z, w;
+        uint32_t w[4], a[4];
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
                      : "r"(saddr + 64u * i));
-        // one flag per word: only a flagged word is redone
-        bool ex = false, ey = false, ez = false, ew = false;
-        uint32_t ax, ay, az, aw;
-        if (kAct != kActSilu && kAct != kActGeluTanh) {
-            ax = act_bf16x2<kAct>(x, ex);
-            ay = act_bf16x2<kAct>(y, ey);
-            az = act_bf16x2<kAct>(z, ez);
-            aw = act_bf16x2<kAct>(w, ew);
-        } else {
-            ax = act_word_tab<kAct>(x, tab, ex);
-            ay = act_word_tab<kAct>(y, tab, ey);
-            az = act_word_tab<kAct>(z, tab, ez);
-            aw = act_word_tab<kAct>(w, tab, ew);
-        }
-        if (ex | ey | ez | ew) {
-            if (ex) ax = act_bf16x2_exact<kAct>(x);
-            if (ey) ay = act_bf16x2_exact<kAct>(y);
-            if (ez) az = act_bf16x2_exact<kAct>(z);
-            if (ew) aw = act_bf16x2_exact<kAct>(w);
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr + 64u * i), "r"(ax),
-                     "r"(ay), "r"(az), "r"(aw)
+        act_chunk<kAct>(w, a, tab);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr + 64u * i), "r"(a[0]),
+                     "r"(a[1]), "r"(a[2]), "r"(a[3])
                      : "memory");
     }
 }
 
 // Test hook: the input activation exactly as the staged quantiser applies it
-// (act_in_smem on each quad's 512-byte block of 256 values), on whole 16-byte
-// chunks; 8192 values per CTA of 128 threads.
+// (act_chunk on 16-byte chunks, the table filled per CTA as there); 8192
+// values per CTA of 128 threads.
 template <int kAct>
 __global__ void __launch_bounds__(128)
 input_act_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Y, int64_t n16) {
@@ -435,6 +434,25 @@ __device__ __forceinline__ void load_block_smem(uint32_t saddr, int sw5, float2 
                      : "r"(base[i & 1] + 64u * i));
 #pragma unroll
         for (int q = 0; q < 4; ++q) P[4 * i + q] = kStage1 ? widen_stage1(w[q]) : widen_bf16x2(w[q]);
+    }
+}
+
+// load_block_smem with the input activation applied to each chunk as it
+// arrives (act_chunk, as the test hook applies it).
+template <bool kStage1, int kAct>
+__device__ __forceinline__ void load_block_smem_act(uint32_t saddr, int sw5, float2 (&P)[kPairs],
+                                                    const uint16_t *tab) {
+    const uint32_t base[2] = {saddr + 64u * uint32_t(sw5), saddr - 64u * uint32_t(sw5)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t w[4];
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(base[i & 1] + 64u * i));
+        uint32_t a[4];
+        act_chunk<kAct>(w, a, tab);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) P[4 * i + q] = kStage1 ? widen_stage1(a[q]) : widen_bf16x2(a[q]);
     }
 }
 
@@ -804,8 +822,11 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
                             uint32_t(col0) * 2u;
         if (active) {
-            if (kAct != kActNone) act_in_smem<kAct>(sa, reinterpret_cast<const uint16_t *>(act_tab));
-            load_block_smem<kRotate>(sa, sw5, P);
+            if (kAct != kActNone)
+                load_block_smem_act<kRotate, kAct>(sa, sw5, P,
+                                                   reinterpret_cast<const uint16_t *>(act_tab));
+            else
+                load_block_smem<kRotate>(sa, sw5, P);
         } else {
             zero_block(P);
         }
