@@ -190,6 +190,35 @@ def test_large_inputs_limits():
     assert abs(_bits_to_float(s) - (-90.0 * np.exp(-90.0))) <= 2.0 ** -8 * 90.0 * np.exp(-90.0)
 
 
+@pytest.mark.parametrize("name", ["silu", "gelu_tanh"])
+def test_closed_forms_far_from_and_near_zero(name):
+    """Properties of the definitions over every bf16 input, which the
+    quantiser's activation table relies on outside |x| in [2^-9, 2^7):
+    act(x) = x (1 - e^-x / (1 + e^-x)) rounds to x for x >= 2^7 and to -0
+    for x <= -2^7 (the exact value is below 2^-134 in magnitude there);
+    act(x) = x / 2 + c x^2 + O(x^3), c = 1/4 (silu) or sqrt(2/pi)/2 (gelu),
+    rounds to x / 2 for 2^-125 <= |x| < 2^-9, and act(+-0) = +-0."""
+    h = np.arange(65536, dtype=np.uint32)
+    got = oracle.act_bf16(name, h.astype(np.uint16)).astype(np.uint32)
+    mag = h & 0x7FFF
+    neg = (h & 0x8000) != 0
+    big = (mag >= 0x4300) & (mag < 0x7F80)
+    assert np.array_equal(got[big & ~neg], h[big & ~neg])
+    assert (got[big & neg] == 0x8000).all()
+    small = (mag >= 0x0100) & (mag < 0x3B00)
+    assert np.array_equal(got[small], h[small] - 0x80)  # one less in the exponent field
+    assert got[0] == 0x0000 and got[0x8000] == 0x8000
+    # and they do not hold one binade further in: silu's large-|x| form
+    # fails for some |x| in [2^6, 2^7), gelu's x / 2 for some |x| in
+    # [2^-9, 2^-8)
+    if name == "silu":
+        far = (mag >= 0x4280) & (mag < 0x4300)
+        assert (got[far] != np.where(neg[far], 0x8000, h[far])).any()
+    else:
+        near = (mag >= 0x3B00) & (mag < 0x3B80)
+        assert (got[near] != h[near] - 0x80).any()
+
+
 @pytest.mark.parametrize("name,fn", [
     ("silu", lambda t: torch.nn.functional.silu(t)),
     ("gelu_tanh", lambda t: torch.nn.functional.gelu(t, approximate="tanh")),
