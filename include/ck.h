@@ -141,8 +141,11 @@ typedef enum ck_act {
  * page names the argument only. The kernel evaluates act in fp32 (its own
  * e^x: Cody-Waite reduction and a degree-7 Taylor polynomial) and redoes in
  * double precision every value whose fp32 result lies near a bf16 rounding
- * midpoint, so the stored bf16 values are those of the definition. Other
- * arguments as for ck_quantize_rotate_rowwise.
+ * midpoint, so the stored bf16 values are those of the definition; for silu
+ * and gelu_tanh each CTA evaluates that once per bf16 input with |x| in
+ * [2^-9, 2^7) into a table, and the other inputs have closed forms (x, -0
+ * or x/2) or take the double path. Other arguments as for
+ * ck_quantize_rotate_rowwise.
  */
 ck_status ck_quantize_rotate_rowwise_act(const ck_bf16 *X, int64_t M, int64_t K, int64_t ldx,
                                          int act, int8_t *Qx, float *s_x, ck_stream_t stream);
