@@ -1369,6 +1369,22 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
 // approximation: r = inf).
 // cvt.e2m1x2 puts its first source in the upper nibble; mov packs the four
 // bytes low byte first.
+// The rare path of nvfp4_encode8, kept out of line (it holds eight IEEE
+// divisions): v[k] = fl(y[k] / d) for the values whose u lies within 2^-16
+// of a multiple of 1/4 (all of them when r is not finite).
+struct F8 {
+    float v[8];
+};
+__device__ __noinline__ F8 nvfp4_encode8_redo(F8 y, F8 v, float r, float d) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float u = __fmul_rn(y.v[k], r);
+        const float q = __fadd_rn(__fadd_rn(u, kMagic4), -kMagic4);
+        if (!(fabsf(__fadd_rn(u, -q)) >= kNearQuarter)) v.v[k] = __fdiv_rn(y.v[k], d);
+    }
+    return v;
+}
+
 __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) {
     if (d == 0.0f) return 0u;
     float r;
@@ -1392,12 +1408,15 @@ __device__ __forceinline__ uint32_t nvfp4_encode8(const float (&y)[8], float d) 
     if (dmin < kNearQuarter) {
         // only the values near a multiple of 1/4 take the division (all of
         // them when r is not finite: |du| is then NaN)
+        F8 yy, vv;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const float u = __fmul_rn(y[k], r);
-            const float q = __fadd_rn(__fadd_rn(u, kMagic4), -kMagic4);
-            if (!(fabsf(__fadd_rn(u, -q)) >= kNearQuarter)) v[k] = __fdiv_rn(y[k], d);
+            yy.v[k] = y[k];
+            vv.v[k] = v[k];
         }
+        vv = nvfp4_encode8_redo(yy, vv, r, d);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = vv.v[k];
     }
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
@@ -1428,12 +1447,16 @@ __device__ __forceinline__ float nvfp4_scale_rcp(float s_t) {
 // 8 units of the half-way pattern 0x80000. Those blocks, values below 2^-6
 // (E4M3's subnormal range, where the rounding position moves) and c6 = 0
 // take the two IEEE divisions.
+__device__ __noinline__ uint32_t nvfp4_block_scale_exact(float m, float s_t) {
+    return e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m, 6.0f), s_t));
+}
+
 __device__ __forceinline__ uint32_t nvfp4_block_scale(float m, float s_t, float c6) {
     if (!(s_t > 0.0f)) return 0u;
     const float q = __fmul_rn(m, c6);
     const uint32_t low = __float_as_uint(q) & 0xFFFFFu;
     if (q >= 0.0156265625f && low - 0x7FFF8u >= 16u) return e4m3_rne_sat(q);
-    return e4m3_rne_sat(__fdiv_rn(__fdiv_rn(m, 6.0f), s_t));
+    return nvfp4_block_scale_exact(m, s_t);
 }
 
 // Scale blocks of register groups c and c + 1 (c even) of a lane. The lanes
