@@ -198,9 +198,21 @@ __device__ __forceinline__ uint32_t act_window(float e, float v) {
 // bf16x2 word -> activation of both values -> bf16x2 word (round to nearest
 // even). `redo` is raised when a value needs the double-precision path; then
 // act_bf16x2_exact gives the word.
+__device__ __forceinline__ __nv_bfloat162 bf162_bits(uint32_t w) {
+    return *reinterpret_cast<const __nv_bfloat162 *>(&w);
+}
+__device__ __forceinline__ uint32_t bits_bf162(__nv_bfloat162 v) {
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 template <int kAct>
 __device__ __forceinline__ uint32_t act_bf16x2(uint32_t w, bool &redo) {
     if (kAct == kActNone) return w;
+    // relu: max(x, +0) of both halves in one instruction (max returns the
+    // non-NaN operand, so NaN gives +0 as x > 0 ? x : 0 does; max(-0, +0)
+    // is +0; every bf16 input is compared with the oracle through the test
+    // hook)
+    if (kAct == kActRelu) return bits_bf162(__hmax2(bf162_bits(w), bf162_bits(0u)));
     const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
     float2 a;
     if (kAct == kActRelu) {
@@ -324,13 +336,6 @@ __device__ __forceinline__ void act_table_fill(uint32_t *tab, int tid, int nthre
         const uint32_t h = ((e & 0x800u) << 4) | (kActTabLo + (e & 0x7FFu));
         tab[i] = act_bf16x2<kAct>(h | ((h + 1u) << 16));
     }
-}
-
-__device__ __forceinline__ __nv_bfloat162 bf162_bits(uint32_t w) {
-    return *reinterpret_cast<const __nv_bfloat162 *>(&w);
-}
-__device__ __forceinline__ uint32_t bits_bf162(__nv_bfloat162 v) {
-    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 // Index of value h's entry (its low 11 bits of |h| - 0x3B00, so every input
