@@ -338,12 +338,6 @@ __device__ __forceinline__ void act_table_fill(uint32_t *tab, int tid, int nthre
     }
 }
 
-// Index of value h's entry (its low 11 bits of |h| - 0x3B00, so every input
-// gives an index inside the table; only the window's are used).
-__device__ __forceinline__ uint32_t act_tab_index(uint32_t h) {
-    return (((h & 0x7FFFu) - kActTabLo) & 0x7FFu) | ((h >> 4) & 0x800u);
-}
-
 template <int kAct>
 __device__ __forceinline__ uint32_t act_word_tab(uint32_t w, const uint16_t *tab, bool &rare) {
     const uint32_t a2 = w & 0x7FFF7FFFu;
@@ -353,8 +347,12 @@ __device__ __forceinline__ uint32_t act_word_tab(uint32_t w, const uint16_t *tab
     const uint32_t inside = ~small & __hlt2_mask(ab, bf162_bits(0x43004300u));  // < 2^7
     const uint32_t half = bits_bf162(__hmul2(wb, bf162_bits(0x3F003F00u)));   // x * 0.5
     const uint32_t big = bits_bf162(__hmax2(wb, bf162_bits(0x80008000u)));    // max(x, -0)
-    const uint32_t lo = tab[act_tab_index(w & 0xFFFFu)];
-    const uint32_t hi = tab[act_tab_index(w >> 16)];
+    // both entries' indices at once: per half 0x8000 + |h| - 0x3B00 (no
+    // borrow between the halves), its low 11 bits, then the sign as bit 11.
+    // Every input gives an index inside the table; only the window's are used.
+    const uint32_t i2 = (((w | 0x80008000u) - 0x3B003B00u) & 0x07FF07FFu) | ((w >> 4) & 0x08000800u);
+    const uint32_t lo = tab[i2 & 0xFFFFu];
+    const uint32_t hi = tab[i2 >> 16];
     const uint32_t t2 = lo | (hi << 16);
     const uint32_t rule = (half & small) | (big & ~small);
     const uint32_t tiny = __hlt2_mask(ab, bf162_bits(0x01000100u)) & ~__heq2_mask(ab, bf162_bits(0u));
