@@ -655,9 +655,60 @@ __device__ __forceinline__ void store_group(const uint32_t (&u)[8], int i, const
     }
 }
 
+// The two rare paths of a group of 8 values out of line (each holds eight
+// IEEE divisions), for the kernels whose unrolled loop body is largest (the
+// activation table's); inline they timed faster in the plain quantiser.
+struct Z8 {
+    float v[8];
+};
+struct U8 {
+    uint32_t v[8];
+};
+// Every value by the definition (rows too small for the fast path).
+__device__ __noinline__ U8 codes8_exact(Z8 z, RowQuant rq) {
+    U8 u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) u.v[k] = code_exact(z.v[k], rq);
+    return u;
+}
+// A flagged group: the values near a half-integer by the definition, the
+// others' fast codes recomputed.
+__device__ __noinline__ U8 codes8_redo(Z8 z, RowQuant rq) {
+    U8 u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float m = __fmaf_rn(z.v[k], rq.rc, kMagic);
+        const float d = __fmaf_rn(z.v[k], -rq.rc, __fadd_rn(m, -kMagic));
+        u.v[k] = fabsf(d) >= kNearHalf ? code_exact(z.v[k], rq) : __float_as_uint(m);
+    }
+    return u;
+}
+
+__device__ __forceinline__ Z8 group_values(const float2 (&P)[kPairs], int i) {
+    Z8 z;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        z.v[2 * k] = P[4 * i + k].x;
+        z.v[2 * k + 1] = P[4 * i + k].y;
+    }
+    return z;
+}
+
 template <bool kPack4>
+__device__ __forceinline__ void store_group_u8(const U8 &u, int i, const CodeDst &dst) {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w[k] = u.v[k];
+    store_group<kPack4>(w, i, dst);
+}
+
+template <bool kPack4, bool kOutOfLine>
 __device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int i,
                                                   const RowQuant &rq, const CodeDst &dst) {
+    if (kOutOfLine) {
+        store_group_u8<kPack4>(codes8_exact(group_values(P, i), rq), i, dst);
+        return;
+    }
     uint32_t u[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -672,13 +723,13 @@ __device__ __forceinline__ void store_group_exact(const float2 (&P)[kPairs], int
 // stores every group without branching and records which groups hold a value
 // near a half-integer; those (rare) groups are then recomputed exactly and
 // stored again.
-template <bool kPack4 = false>
+template <bool kPack4 = false, bool kOutOfLine = false>
 __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const RowQuant &rq,
                                                int8_t *qbase, int sw5 = 0) {
     const CodeDst dst(qbase, sw5);
     if (!rq.fast) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) store_group_exact<kPack4>(P, i, rq, dst);
+        for (int i = 0; i < 8; ++i) store_group_exact<kPack4, kOutOfLine>(P, i, rq, dst);
         return;
     }
     const FastQuant fq(rq.rc);
@@ -701,17 +752,20 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[kPairs], const 
         // exact path; the others keep their fast codes (recomputed).
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            if (redo & (1u << i)) {
-                uint32_t u[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float z = (k & 1) ? P[4 * i + (k >> 1)].y : P[4 * i + (k >> 1)].x;
-                    const float m = __fmaf_rn(z, rq.rc, kMagic);
-                    const float d = __fmaf_rn(z, -rq.rc, __fadd_rn(m, -kMagic));
-                    u[k] = fabsf(d) >= kNearHalf ? code_exact(z, rq) : __float_as_uint(m);
-                }
-                store_group<kPack4>(u, i, dst);
+            if (!(redo & (1u << i))) continue;
+            if (kOutOfLine) {
+                store_group_u8<kPack4>(codes8_redo(group_values(P, i), rq), i, dst);
+                continue;
             }
+            uint32_t u[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float z = (k & 1) ? P[4 * i + (k >> 1)].y : P[4 * i + (k >> 1)].x;
+                const float m = __fmaf_rn(z, rq.rc, kMagic);
+                const float d = __fmaf_rn(z, -rq.rc, __fadd_rn(m, -kMagic));
+                u[k] = fabsf(d) >= kNearHalf ? code_exact(z, rq) : __float_as_uint(m);
+            }
+            store_group<kPack4>(u, i, dst);
         }
     }
 }
@@ -851,7 +905,8 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         if (active) {
             const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[slot][row_local]));
             if (blk == 0 && t == 0) S[row] = rq.s;
-            quantize_store(P, rq, Q + row * static_cast<int64_t>(K) + col0, sw5);
+            quantize_store<false, kAct == kActSilu || kAct == kActGeluTanh>(
+                P, rq, Q + row * static_cast<int64_t>(K) + col0, sw5);
         }
         slot = slot == 2 ? 0 : slot + 1;
         if (++b == kBulkBufs) {
