@@ -477,6 +477,23 @@ ck_status ck_get_device_error(void);
 /* Resets the current device's error word (synchronous with the device). */
 ck_status ck_clear_device_error(void);
 
+/*
+ * The checked build. libck_checked.so is this library compiled with
+ * CK_CHECKED: its kernels test index invariants at their memory accesses
+ * (global stores and loads inside their tensor's rows and columns,
+ * shared-memory accesses and bulk copies inside the CTA's allocation, TMEM
+ * columns inside the allocation). A failed check skips the access and sets
+ * its class bit (1 global store, 2 global load, 4 shared memory, 8 bulk copy,
+ * 16 TMEM) in a device word; nothing traps. A bulk copy that was skipped
+ * leaves its stage's wait to run out, which ck_get_device_error() then
+ * reports as CK_ERR_DEVICE_TIMEOUT. ck_is_checked_build() returns 1 in that
+ * build and 0 in libck.so. ck_checked_violations() synchronises the current
+ * device, returns the class bits set since its last call on that device and
+ * clears them (0 in libck.so; bit 31 if the words could not be read).
+ */
+int ck_is_checked_build(void);
+unsigned ck_checked_violations(void);
+
 /* ---- test hooks (used by the test suite; stable, but not part of the method) ---- */
 
 /*
@@ -510,6 +527,14 @@ ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck
  * the INT8 GEMM's roofline a measured denominator.
  */
 ck_status ck_test_i8_mma_peak(int64_t mmas_per_pair, int *pairs, ck_stream_t stream);
+
+/*
+ * One thread whose index check fails on purpose (class bit 4, shared memory)
+ * with no memory access behind it: in libck_checked.so the next
+ * ck_checked_violations() then returns 4; in libck.so nothing happens. It
+ * shows that the checked build's words are set, read and cleared.
+ */
+ck_status ck_test_checked_fire(ck_stream_t stream);
 
 /*
  * Fault injection for the bounded waits, host side only: with mode 1 the next

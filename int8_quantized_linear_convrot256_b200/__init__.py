@@ -5,7 +5,9 @@ every function here only checks and marshals its arguments and calls the
 entry point of the same name; all arithmetic runs in the library's CUDA
 kernels. PyTorch supplies device memory and streams. There is no CPU path:
 if ``libck.so`` is missing, importing this package raises ImportError, and a
-call on a device that is not a B200 raises ``CKError`` (CK_ERR_ARCH).
+call on a device that is not a B200 raises ``CKError`` (CK_ERR_ARCH). With
+the environment variable CK_LIBRARY=libck_checked.so the package loads the
+checked build instead (device-side bounds checks; ``checked_violations()``).
 
     import int8_quantized_linear_convrot256_b200 as ck
     Qw, s_w = ck.rotate_quant_weight(W_fp32_cuda)          # offline, once
@@ -26,7 +28,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libck.so")
+LIB_PATH = os.path.join(_HERE, os.path.basename(os.environ.get("CK_LIBRARY", "libck.so")))
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "ck.h")
 
 CK_OK = 0
@@ -44,6 +46,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with `python int8_quantized_linear_convrot256_b200/build.py`"
+        " (add --checked for libck_checked.so)"
         " (there is no CPU fallback)")
 
 _i64 = ctypes.c_int64
@@ -93,12 +96,15 @@ _SIGS = {
                                   _vp, ctypes.c_size_t, _vp]),
     "ck_status_string": (ctypes.c_char_p, [_st]),
     "ck_get_device_error": (_st, []),
+    "ck_is_checked_build": (ctypes.c_int, []),
+    "ck_checked_violations": (ctypes.c_uint, []),
     "ck_clear_device_error": (_st, []),
     "ck_test_int8_gemm_i32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "ck_test_quantize_rowwise_norotate": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_test_inject_producer_stall": (_st, [ctypes.c_int, _i64]),
     "ck_test_input_act": (_st, [_vp, _i64, _st, _vp, _vp]),
     "ck_test_i8_mma_peak": (_st, [_i64, ctypes.POINTER(ctypes.c_int), _vp]),
+    "ck_test_checked_fire": (_st, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -638,6 +644,24 @@ test_i8_mma_peak.__test__ = False
 def device_error() -> int:
     """Synchronises the device; returns CK_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait."""
     return int(lib.ck_get_device_error())
+
+
+def is_checked_build() -> bool:
+    """True when the loaded library is the checked build (libck_checked.so)."""
+    return bool(lib.ck_is_checked_build())
+
+
+def checked_violations() -> int:
+    """Class bits of the checked build's failed checks since the last call
+    (1 global store, 2 global load, 4 shared memory, 8 bulk copy, 16 TMEM),
+    then cleared; always 0 for libck.so. Synchronises the current device."""
+    return int(lib.ck_checked_violations())
+
+
+def test_checked_fire(stream=None) -> None:
+    """Test hook: one failed index check with no access behind it (class bit
+    4 in the checked build; a no-op in libck.so)."""
+    _check(lib.ck_test_checked_fire(_stream(stream)), "ck_test_checked_fire")
 
 
 def clear_device_error() -> None:

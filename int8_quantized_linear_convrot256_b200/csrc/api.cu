@@ -935,6 +935,15 @@ ck_status ck_test_i8_mma_peak(int64_t mmas_per_pair, int *pairs, ck_stream_t str
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
+ck_status ck_test_checked_fire(ck_stream_t stream) {
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    return ck::launch_test_checked_fire(reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CK_OK
+               : CK_ERR_CUDA;
+}
+
 const char *ck_status_string(ck_status status) {
     switch (status) {
         case CK_OK: return "CK_OK";
@@ -957,6 +966,24 @@ ck_status ck_get_device_error(void) {
     unsigned v = 0;
     if (cudaMemcpy(&v, st->err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return CK_ERR_CUDA;
     return v ? static_cast<ck_status>(v) : CK_OK;
+}
+
+int ck_is_checked_build(void) {
+#ifdef CK_CHECKED
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+unsigned ck_checked_violations(void) {
+#ifdef CK_CHECKED
+    if (cudaDeviceSynchronize() != cudaSuccess) return 0x80000000u;
+    return ck::check_word_quant() | ck::check_word_gemm_i8() | ck::check_word_gemm_nvfp4() |
+           ck::check_word_dequant() | ck::check_word_rmsnorm();
+#else
+    return 0u;
+#endif
 }
 
 ck_status ck_clear_device_error(void) {

@@ -14,6 +14,49 @@ constexpr unsigned kDevErrTimeout = 7u;
 // Default bound on any single device-side wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;
 
+// ---------------------------------------------------------------- checks
+// The CK_CHECKED build (libck_checked.so) tests index invariants at the
+// kernels' memory accesses: global stores and loads inside the rows and
+// columns of their tensor, shared-memory accesses inside the CTA's
+// allocation, bulk copies inside both, TMEM columns inside the allocation.
+// A failed check sets its class bit in a word of the translation unit and
+// the access is skipped; nothing traps. The normal build compiles the checks
+// away. ck_checked_violations() reads and clears the words.
+constexpr unsigned kChkGlobalStore = 1u;
+constexpr unsigned kChkGlobalLoad = 2u;
+constexpr unsigned kChkShared = 4u;
+constexpr unsigned kChkBulkCopy = 8u;
+constexpr unsigned kChkTmem = 16u;
+#ifdef CK_CHECKED
+namespace {
+__device__ unsigned g_ck_check;  // one per translation unit
+}  // namespace
+__device__ __forceinline__ bool ck_check(bool ok, unsigned cls) {
+    if (!ok) atomicOr(&g_ck_check, cls);
+    return ok;
+}
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+    return r;
+}
+#define CK_CHECK(cond, cls) ::ck::ck_check(static_cast<bool>(cond), (cls))
+// Host side, one per translation unit: the word's value, then cleared.
+#define CK_DEFINE_CHECK_READER(name)                                       \
+    unsigned name() {                                                      \
+        unsigned v = 0;                                                    \
+        const unsigned zero = 0;                                           \
+        if (cudaMemcpyFromSymbol(&v, g_ck_check, sizeof v) != cudaSuccess) \
+            v = 0x80000000u;                                               \
+        cudaMemcpyToSymbol(g_ck_check, &zero, sizeof zero);                \
+        return v;                                                          \
+    }
+#else
+#define CK_CHECK(cond, cls) true
+#define CK_DEFINE_CHECK_READER(name) \
+    unsigned name() { return 0u; }
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -141,4 +141,6 @@ cudaError_t launch_quantize_int8_tensorwise(const uint16_t *X, int64_t M, int64_
     return cudaGetLastError();
 }
 
+CK_DEFINE_CHECK_READER(check_word_dequant)
+
 }  // namespace ck

@@ -545,6 +545,8 @@ __device__ __forceinline__ void store_accumulators_tma(const GemmParams &p,
     for (int c = 0; c < 256 / 32; ++c) {
         uint32_t r[32];
         __syncwarp();
+        if (!CK_CHECK((tbase & 0xFFFFu) + uint32_t(c * 32) + 32u <= kTmemCols, kChkTmem))
+            continue;  // warp-uniform
         tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
         tmem_ld_wait();
         const int n0 = n_tile0 + c * 32;
@@ -557,7 +559,7 @@ __device__ __forceinline__ void store_accumulators_tma(const GemmParams &p,
         for (int g = 0; g < 4; ++g) {
             const int n = n0 + 8 * g;
             uint4 out = make_uint4(0u, 0u, 0u, 0u);
-            if (n < p.N) {
+            if (n < p.N && CK_CHECK(n + 8 <= p.N, kChkGlobalLoad)) {
                 const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
                 const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + n + 4));
                 const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -615,6 +617,8 @@ __device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t
     for (int c = 0; c < 256 / 32; ++c) {
         uint32_t r[32];
         __syncwarp();
+        if (!CK_CHECK((tbase & 0xFFFFu) + uint32_t(c * 32) + 32u <= kTmemCols, kChkTmem))
+            continue;  // warp-uniform
         tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
         tmem_ld_wait();
         const int n0 = n_tile0 + c * 32;
@@ -623,6 +627,7 @@ __device__ __forceinline__ void store_accumulators(const GemmParams &p, uint32_t
         for (int g = 0; g < 4; ++g) {
             const int n = n0 + 8 * g;
             if (n >= p.N) break;
+            if (!CK_CHECK(n + 8 <= p.N, kChkGlobalStore | kChkGlobalLoad)) break;
             if (kRaw) {
                 int4 *dst = reinterpret_cast<int4 *>(p.acc + int64_t(row) * p.N + n);
                 dst[0] = make_int4(int(r[8 * g + 0]), int(r[8 * g + 1]), int(r[8 * g + 2]),
@@ -854,5 +859,7 @@ cudaError_t launch_gemm_i8(const CUtensorMap &tmA, const CUtensorMap &tmB, const
     if (raw_i32) return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<true>, tmA, tmB, tmY, p);
     return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<false>, tmA, tmB, tmY, p);
 }
+
+CK_DEFINE_CHECK_READER(check_word_gemm_i8)
 
 }  // namespace ck

@@ -347,6 +347,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 __syncwarp();
+                if (!CK_CHECK((tbase & 0xFFFFu) + uint32_t(c * 32) + 32u <= kTmemCols, kChkTmem))
+                    continue;  // warp-uniform
                 tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r);
                 tmem_ld_wait();
                 if (!row_ok) continue;
@@ -354,6 +356,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 for (int g = 0; g < 4; ++g) {
                     const int n = nt * BN + c * 32 + 8 * g;
                     if (n >= p.N) break;
+                    if (!CK_CHECK(n + 8 <= p.N, kChkGlobalStore | kChkGlobalLoad)) break;
                     float b[8];
                     if (p.bias) {
                         const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
@@ -701,21 +704,24 @@ gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t tbase =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(half * 128);
             uint32_t r[4][32];
+            const bool cols_ok = CK_CHECK((tbase & 0xFFFFu) + 128u <= kTmemCols, kChkTmem);
+            if (cols_ok) {  // warp-uniform
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r[c]);
-            tmem_ld_wait();
+                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), r[c]);
+                tmem_ld_wait();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tmem_empty);
             acc_phase ^= 1u;
             const int row = mt * kPairBMn + int(rank) * kPairRowsN + quarter * 32 + lane;
-            if (row < p.M) {
+            if (row < p.M && cols_ok) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         const int n = nt * kPairBNn + half * 128 + c * 32 + 8 * g;
-                        if (n < p.N) {
+                        if (n < p.N && CK_CHECK(n + 8 <= p.N, kChkGlobalStore | kChkGlobalLoad)) {
                             float b[8];
                             if (p.bias) {
                                 const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + n));
@@ -839,5 +845,7 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB,
     gemm_nvfp4_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
     return cudaGetLastError();
 }
+
+CK_DEFINE_CHECK_READER(check_word_gemm_nvfp4)
 
 }  // namespace ck

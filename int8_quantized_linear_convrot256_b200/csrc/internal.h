@@ -159,4 +159,15 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB,
                               const Nvfp4GemmParams &p, int num_sms, bool allow_pair,
                               cudaStream_t stream);
 
+// Test hook: one thread failing an index check (class bit kChkShared), no access.
+cudaError_t launch_test_checked_fire(cudaStream_t stream);
+
+// The CK_CHECKED build's per-file check words (class bits of failed checks),
+// read and cleared; always 0 in the normal build.
+unsigned check_word_quant();
+unsigned check_word_gemm_i8();
+unsigned check_word_gemm_nvfp4();
+unsigned check_word_dequant();
+unsigned check_word_rmsnorm();
+
 }  // namespace ck

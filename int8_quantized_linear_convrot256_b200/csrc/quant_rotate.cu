@@ -789,8 +789,10 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     const int col0 = blk * kBlock + 8 * t;
 
     if (tid < rows_per_cta) s_amax[tid] = 0u;
+    // the lane's 8 chunks end at col0 + 232 (its last chunk starts 224 on)
+    const bool in_row = CK_CHECK(!active || col0 + 232 <= K, kChkGlobalLoad | kChkGlobalStore);
     float2 P[kPairs];
-    if (active)
+    if (active && in_row)
         load_block<kAct>(X + row * ldx + col0, P);
     else
         zero_block(P);
@@ -799,7 +801,7 @@ quant_rows_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     __syncthreads();  // s_amax initialised
     if (active && t == 0) atomicMax(&s_amax[row_local], __float_as_uint(m));
     __syncthreads();
-    if (!active) return;
+    if (!active || !in_row) return;
     const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[row_local]));
     if (blk == 0 && t == 0) S[row] = rq.s;
     if (kPack4)
@@ -854,9 +856,14 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
         for (int r = 0; r < n; ++r) {
             const uint16_t *src = X + (r0 + r) * ldx;
+            const uint32_t off = uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes;
+#ifdef CK_CHECKED
+            if (!CK_CHECK(r0 + r < M && off + row_bytes <= dynamic_smem_bytes(), kChkBulkCopy))
+                continue;  // the wait on this group then runs out and reports the timeout
+#endif
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                ::"r"(buf0 + uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes),
+                ::"r"(buf0 + off),
                 "l"(reinterpret_cast<uint64_t>(src)), "r"(row_bytes), "r"(bar)
                 : "memory");
         }
@@ -874,10 +881,16 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const int64_t g = g0 + i * step;
         const bool ok = mbar_wait_bounded(smem_u32(&full[b]), par, limit_ns, nullptr);
         const int64_t row = g * R + row_local;
-        const bool active = ok && row_local < R && row < M;
+        bool active = ok && row_local < R && row < M;
         float2 P[kPairs];
         const uint32_t sa = buf0 + uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes +
                             uint32_t(col0) * 2u;
+#ifdef CK_CHECKED
+        // the lane reads [sa, sa + 464) of the buffer; its codes span col0 .. col0 + 232
+        if (active && !CK_CHECK(sa - buf0 + 464u <= dynamic_smem_bytes() && col0 + 232 <= K,
+                                kChkShared))
+            active = false;
+#endif
         if (active) {
             if (kAct != kActNone)
                 load_block_smem_act<kRotate, kAct>(sa, sw5, P,
@@ -1048,12 +1061,18 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const int64_t ld = res ? na.ldr : ldx;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
-        for (int r = 0; r < n; ++r)
+        for (int r = 0; r < n; ++r) {
+#ifdef CK_CHECKED
+            if (!CK_CHECK(r0 + r < M && dst + uint32_t(r + 1) * row_bytes - buf0 <= dynamic_smem_bytes(),
+                          kChkBulkCopy))
+                continue;  // the wait on this group then runs out and reports the timeout
+#endif
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                 ::"r"(dst + uint32_t(r) * row_bytes),
                 "l"(reinterpret_cast<uint64_t>(src + (r0 + r) * ld)), "r"(row_bytes), "r"(bar)
                 : "memory");
+        }
     };
 
     const int64_t g0 = blockIdx.x;
@@ -1073,8 +1092,18 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         if (kResidual)
             ok = ok && mbar_wait_bounded(smem_u32(&full[2]), uint32_t(i) & 1u, limit_ns, nullptr);
         const int64_t row = g * R + row_local;
-        const bool active = ok && row_local < R && row < M;
+        bool active = ok && row_local < R && row < M;
         const uint32_t rowoff = uint32_t(row_local) * row_bytes + uint32_t(col0) * 2u;
+#ifdef CK_CHECKED
+        // x, the residual and the weight: [.. + rowoff, + 464) of their buffers;
+        // the residual output and the codes: columns col0 .. col0 + 232 of the row
+        if (active && !CK_CHECK((kResidual ? rbuf : buf0 + uint32_t(b) * buf_bytes) + rowoff + 464u -
+                                        buf0 <= dynamic_smem_bytes() &&
+                                    sg0 + 2u * uint32_t(col0) + 464u - buf0 <= dynamic_smem_bytes() &&
+                                    col0 + 232 <= K,
+                                kChkShared))
+            active = false;
+#endif
         const uint32_t sx = buf0 + uint32_t(b) * buf_bytes + rowoff;
         // h of this lane's 64 values (register group i = chunk i ^ sw5),
         // stored as the residual output, and its sum of squares (one
@@ -1230,7 +1259,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
     for (int b0 = 0; b0 < nb; b0 += kTwoPassQuads) {
         const int blk = b0 + quad;
         float2 P[kPairs];
-        if (blk < nb)
+        if (blk < nb && CK_CHECK(row < M && blk * kBlock + 8 * t + 232 <= K, kChkGlobalLoad))
             load_block<kAct>(xrow + blk * kBlock + 8 * t, P);
         else
             zero_block(P);
@@ -1245,7 +1274,7 @@ quant_rows_two_pass_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t 
     for (int b0 = 0; b0 < nb; b0 += kTwoPassQuads) {
         const int blk = b0 + quad;
         float2 P[kPairs];
-        if (blk < nb)
+        if (blk < nb && CK_CHECK(row < M && blk * kBlock + 8 * t + 232 <= K, kChkGlobalLoad))
             load_block<kAct>(xrow + blk * kBlock + 8 * t, P);
         else
             zero_block(P);
@@ -1551,6 +1580,11 @@ __device__ __forceinline__ uint2 nvfp4_codes_pair(const float2 (&P)[kPairs], int
 // Offset of the scale of row r, scale column c (of C) in the blocked layout:
 // 512-byte tiles of 128 rows x 4 columns, column tiles fastest; rows r, r + 32,
 // r + 64, r + 96 of a tile share the 16-byte line r % 32.
+__device__ __forceinline__ bool nvfp4_sf_in_range(int64_t off, int64_t M, int C) {
+    return CK_CHECK(off >= 0 && off < ((M + 127) / 128) * 128 * int64_t((C + 3) / 4 * 4),
+                    kChkGlobalStore);
+}
+
 __device__ __forceinline__ int64_t nvfp4_sf_offset(int64_t r, int c, int C) {
     const int64_t tile = (r >> 7) * int64_t((C + 3) >> 2) + (c >> 2);
     return tile * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
@@ -1570,7 +1604,8 @@ nvfp4_amax_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int 
     const int row_local = quad / nb;
     const int blk = quad - row_local * nb;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + row_local;
-    const bool active = row_local < rows_per_cta && row < M;
+    const bool active = row_local < rows_per_cta && row < M &&
+                        CK_CHECK(blk * kBlock + 8 * t + 232 <= K, kChkGlobalLoad);
     if (tid == 0) s_max = 0u;
     float2 P[kPairs];
     if (active)
@@ -1600,8 +1635,9 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
     const int row_local = quad / nb;
     const int blk = quad - row_local * nb;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + row_local;
-    const bool active = row_local < rows_per_cta && row < M;
     const int col0 = blk * kBlock + 8 * t;
+    const bool active = row_local < rows_per_cta && row < M &&
+                        CK_CHECK(col0 + 232 <= K, kChkGlobalLoad | kChkGlobalStore);
     float2 P[kPairs];
     if (active)
         load_block<kActNone>(X + row * ldx + col0, P);
@@ -1621,7 +1657,8 @@ nvfp4_quant_kernel(const TIn *__restrict__ X, int64_t M, int K, int64_t ldx, int
             uint8_t *qr = Q + row * int64_t(K / 2);
             *reinterpret_cast<uint32_t *>(qr + e0 / 2) = packed.x;
             *reinterpret_cast<uint32_t *>(qr + (e0 + 32) / 2) = packed.y;
-            S[nvfp4_sf_offset(row, (e0 + 32 * (t & 1)) >> 4, C)] = uint8_t(b);
+            const int64_t so = nvfp4_sf_offset(row, (e0 + 32 * (t & 1)) >> 4, C);
+            if (nvfp4_sf_in_range(so, M, C)) S[so] = uint8_t(b);
         }
     }
 }
@@ -1694,6 +1731,16 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
         mbar_arrive_expect_tx(bar, uint32_t(n) * 512u);
         for (int i = 0; i < n;) {
             const int run = min(n - i, nb - blk);
+#ifdef CK_CHECKED
+            if (!CK_CHECK(row < M && blk + run <= nb &&
+                              (wbuf - smem_u32(stage_raw)) + uint32_t(b) * kNvUnitBytes +
+                                      uint32_t(i + run) * 512u <=
+                                  dynamic_smem_bytes(),
+                          kChkBulkCopy)) {
+                i += run;  // the wait on this unit then runs out and reports the timeout
+                continue;
+            }
+#endif
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                 ::"r"(wbuf + uint32_t(b) * kNvUnitBytes + uint32_t(i) * 512u),
@@ -1743,7 +1790,17 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
             blk -= nb;
             ++row;
         }
-        const bool active = u * kNvUnitBlocks + qw < nblocks;
+        bool active = u * kNvUnitBlocks + qw < nblocks;
+#ifdef CK_CHECKED
+        // the quad's block in the warp's buffer; the codes and scales of its row
+        if (active &&
+            !CK_CHECK(row < M && blk < nb &&
+                          (wbuf - smem_u32(stage_raw)) + uint32_t(b) * kNvUnitBytes +
+                                  uint32_t(qw + 1) * 512u <=
+                              dynamic_smem_bytes(),
+                      kChkShared))
+            active = false;
+#endif
         float2 P[kPairs];
         if (active)
             load_block_smem<true>(wbuf + uint32_t(b) * kNvUnitBytes + uint32_t(qw) * 512u +
@@ -1772,7 +1829,8 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
                     const int eb = col0 + 32 * (c + 1 - sw5);  // group c + 1
                     *reinterpret_cast<uint32_t *>(qr + ea / 2) = packed.x;
                     *reinterpret_cast<uint32_t *>(qr + eb / 2) = packed.y;
-                    S[nvfp4_sf_offset(row, ((t & 1) ? eb : ea) >> 4, C)] = uint8_t(bsc);
+                    const int64_t so = nvfp4_sf_offset(row, ((t & 1) ? eb : ea) >> 4, C);
+                    if (nvfp4_sf_in_range(so, M, C)) S[so] = uint8_t(bsc);
                 }
             }
         }
@@ -1807,7 +1865,10 @@ __global__ void nvfp4_dequant_kernel(const uint8_t *__restrict__ Q, const uint8_
         const int64_t r = g / (K / 8);
         const int k0 = int(g - r * (K / 8)) * 8;
         const uint32_t w = *reinterpret_cast<const uint32_t *>(Q + r * int64_t(K / 2) + k0 / 2);
-        const float scale = __fmul_rn(st, e4m3_to_f32(S[nvfp4_sf_offset(r, k0 >> 4, C)]));
+        const int64_t so = nvfp4_sf_offset(r, k0 >> 4, C);
+        if (!CK_CHECK(so < ((rows + 127) / 128) * 128 * int64_t((C + 3) / 4 * 4), kChkGlobalLoad))
+            continue;
+        const float scale = __fmul_rn(st, e4m3_to_f32(S[so]));
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -2017,5 +2078,16 @@ cudaError_t launch_dequant_nvfp4(const uint8_t *Q, const uint8_t *S, const float
         Q, S, s_t, rows, static_cast<int>(K), hi_first ? 1 : 0, out);
     return cudaGetLastError();
 }
+
+namespace {
+__global__ void checked_fire_kernel(int n) { CK_CHECK(int(threadIdx.x) >= n, kChkShared); }
+}  // namespace
+
+cudaError_t launch_test_checked_fire(cudaStream_t stream) {
+    checked_fire_kernel<<<1, 1, 0, stream>>>(1);
+    return cudaGetLastError();
+}
+
+CK_DEFINE_CHECK_READER(check_word_quant)
 
 }  // namespace ck

@@ -17,6 +17,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "ck_device.cuh"
 #include "internal.h"
 
 namespace ck {
@@ -130,5 +131,7 @@ cudaError_t launch_rmsnorm_rows(const uint16_t *X, int64_t ldx, const uint16_t *
         X, ldx, R, ldr, Rout, ldo, g, eps, M, static_cast<int>(K), Y);
     return cudaGetLastError();
 }
+
+CK_DEFINE_CHECK_READER(check_word_rmsnorm)
 
 }  // namespace ck

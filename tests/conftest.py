@@ -19,3 +19,15 @@ def oracle_lib():
 
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _no_failed_index_checks(request):
+    """Under the checked build (CK_LIBRARY=libck_checked.so), every GPU test
+    must also leave no failed device-side index check behind."""
+    yield
+    if "gpu" in request.keywords and os.environ.get("CK_LIBRARY", "").endswith("libck_checked.so"):
+        import int8_quantized_linear_convrot256_b200 as ck
+
+        bits = ck.checked_violations()
+        assert bits == 0, f"failed index checks in the checked build, class bits {bits:#x}"

@@ -3,6 +3,7 @@ function include/ck.h declares, and its host-side validation returns the
 documented status before touching the device (fake, never-dereferenced
 addresses are enough for that)."""
 import ctypes
+import os
 import re
 
 import pytest
@@ -25,6 +26,20 @@ def test_every_declared_function_is_exported():
     for n in names:
         assert hasattr(ck.lib, n), n
     assert set(names) == set(ck._SIGS), "binding and header disagree"
+
+
+def test_checked_build_exports_the_same_functions():
+    """libck_checked.so (the build with device-side index checks) has the
+    same C ABI, and says which build it is."""
+    path = os.path.join(os.path.dirname(ck.LIB_PATH), "libck_checked.so")
+    if not os.path.exists(path):
+        pytest.skip("libck_checked.so not built")
+    checked = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(checked, n), n
+    checked.ck_is_checked_build.restype = ctypes.c_int
+    assert checked.ck_is_checked_build() == 1
+    assert ck.lib.ck_is_checked_build() == (1 if ck.LIB_PATH.endswith("libck_checked.so") else 0)
 
 
 def test_status_strings():
