@@ -374,6 +374,20 @@ def run_ours(args, cfg, rank, world, local_rank):
     spread = [srt[len(srt) // 2], srt[0], srt[-1]]  # median, min, max of the steps
     ms_step, ms_q, ms_g, *spread = max_over_ranks([ms_step, ms_q, ms_g, *spread], dev)
 
+    # ---- the quantiser by itself (context for its in-step time: here no GEMM
+    # runs before it, so the SM clock has not been held at the power cap)
+    q_alone = []
+    for _ in range(SUBPATH_STEPS):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        quantize()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        q_alone.append(e0.elapsed_time(e1))
+    ms_q_alone = sorted(q_alone)[len(q_alone) // 2]
+
     # ---- end to end through the public composite call, host buffers
     if args.no_e2e or args.path in ("w4a4", "nvfp4", "norm"):
         ms_e2e = float("nan")
@@ -399,7 +413,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         if ck.device_error() != ck.CK_OK:
             raise RuntimeError("device error while timing the other paths")
     return report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e,
-                  clocks, t_wall0, t_wall1, spread, probe_tops, probe_clocks, subpaths)
+                  clocks, t_wall0, t_wall1, spread, probe_tops, probe_clocks, subpaths,
+                  ms_q_alone)
 
 
 SUBPATH_STEPS = 10
@@ -567,7 +582,8 @@ def run_e2e(args, X, Xd, Qw, s_w, bd, Y, ws, stream, world, dev):
 
 
 def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e, clocks,
-           t_wall0, t_wall1, spread=None, probe_tops=None, probe_clocks=None, subpaths=None):
+           t_wall0, t_wall1, spread=None, probe_tops=None, probe_clocks=None, subpaths=None,
+           ms_q_alone=None):
     # per-rank work: the full batch (weak, replicas) or this rank's row shard
     # (strong); the job's total is world x per-rank (weak) or the whole batch
     M, N, K = X.shape[0], cfg.N, cfg.K
@@ -652,7 +668,13 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                                       "quant_rows_two_pass_kernel") + " (ConvRot256 + per-row INT8)"),
                           "bound": "hbm", "achieved": q_gbs, "peak": P["hbm_gbs"], "unit": "GB/s",
                           "frac": q_gbs / P["hbm_gbs"], "frac_of_spec_8000": q_gbs / 8000.0,
-                          "bytes_per_launch": q_bytes, "ms_per_launch": ms_q},
+                          "bytes_per_launch": q_bytes, "ms_per_launch": ms_q,
+                          **({"alone": {"ms_per_launch": ms_q_alone,
+                                        "frac": q_bytes / (ms_q_alone / 1e3) / 1e9 / P["hbm_gbs"],
+                                        "note": f"median of {SUBPATH_STEPS} launches timed by "
+                                                "themselves after the timed region, L2 flushed "
+                                                "before each; not the metric"}}
+                             if ms_q_alone else {})},
             "cpu_baseline": cpu,
             "e2e": None if (args.no_e2e or args.path in ("w4a4", "nvfp4", "norm")) else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(M * N * 2),
