@@ -32,7 +32,8 @@
  *  - Every pointer argument is DEVICE memory (cudaMalloc, a PyTorch CUDA
  *    tensor, ...) on the current device, owned by the caller. The library
  *    allocates nothing, keeps no pointer after returning, and never
- *    synchronises the stream or the device (except ck_get_device_error).
+ *    synchronises the stream or the device (except ck_get_device_error,
+ *    ck_clear_device_error and ck_checked_violations).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and runs asynchronously: on CK_OK the results are valid once the
  *    stream reaches that point.
