@@ -519,6 +519,21 @@ ck_status ck_test_quantize_rowwise_norotate(const ck_bf16 *X, int64_t M, int64_t
 ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck_stream_t stream);
 
 /*
+ * The per-row divisor and reciprocal of the rotated quantiser, for n row
+ * absmax values (all device memory, fp32, n elements each):
+ *   amax [n] (input), div [n], rc [n] (outputs); q = 127 (INT8) or 7 (INT4).
+ * For amax >= 2^-103 (finite) div is the IEEE quotient fl(amax / q), which
+ * the row scale is derived from, and rc the reciprocal of div that the fast
+ * rounding path multiplies by (within 2^-24 + 2^-43 of 1 / div relative);
+ * smaller absmax values take the quantiser's exact path (div = the row
+ * scale, rc = 0). CK_ERR_INVALID_VALUE for n < 0, another q, or a null
+ * pointer with n > 0. Lets the tests compare the division with the IEEE
+ * quotient for every fp32 significand.
+ */
+ck_status ck_test_row_quant_params(const float *amax, int64_t n, int q, float *div, float *rc,
+                                   ck_stream_t stream);
+
+/*
  * The INT8 tensor-core ceiling, measured: on every pair of SMs the GEMM uses
  * (*pairs receives their number), mmas_per_pair back-to-back
  * tcgen05.mma.cta_group::2.kind::i8 of the GEMM's shape (M 256, N 256, K 32:

@@ -103,6 +103,7 @@ _SIGS = {
     "ck_test_quantize_rowwise_norotate": (_st, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ck_test_inject_producer_stall": (_st, [ctypes.c_int, _i64]),
     "ck_test_input_act": (_st, [_vp, _i64, _st, _vp, _vp]),
+    "ck_test_row_quant_params": (_st, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "ck_test_i8_mma_peak": (_st, [_i64, ctypes.POINTER(ctypes.c_int), _vp]),
     "ck_test_checked_fire": (_st, [_vp]),
 }
@@ -627,6 +628,21 @@ def test_input_act(X: torch.Tensor, act: str, out: torch.Tensor | None = None,
 
 
 test_input_act.__test__ = False
+
+
+def test_row_quant_params(amax: torch.Tensor, q: int = 127, stream=None):
+    """The rotated quantiser's per-row divisor and reciprocal for each row
+    absmax in `amax` (contiguous CUDA fp32; test hook). Returns (div, rc)."""
+    if amax.dtype != torch.float32 or not amax.is_cuda or not amax.is_contiguous():
+        raise ValueError("amax must be a contiguous CUDA float32 tensor")
+    div = torch.empty_like(amax)
+    rc = torch.empty_like(amax)
+    _check(lib.ck_test_row_quant_params(_ptr(amax), amax.numel(), q, _ptr(div), _ptr(rc),
+                                        _stream(stream)), "ck_test_row_quant_params")
+    return div, rc
+
+
+test_row_quant_params.__test__ = False
 
 
 def test_i8_mma_peak(mmas_per_pair: int, stream=None) -> int:

@@ -925,6 +925,19 @@ ck_status ck_test_input_act(const ck_bf16 *X, int64_t n, int act, ck_bf16 *Y, ck
     return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
+ck_status ck_test_row_quant_params(const float *amax, int64_t n, int q, float *div, float *rc,
+                                   ck_stream_t stream) {
+    if (n < 0 || (q != 127 && q != 7)) return CK_ERR_INVALID_VALUE;
+    if (n > 0 && (!amax || !div || !rc)) return CK_ERR_INVALID_VALUE;
+    if (n == 0) return CK_OK;
+    DeviceState *st = nullptr;
+    ck_status s = device_state(&st);
+    if (s != CK_OK) return s;
+    cudaError_t e = ck::launch_test_row_quant_params(amax, n, q, div, rc,
+                                                     reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
 ck_status ck_test_i8_mma_peak(int64_t mmas_per_pair, int *pairs, ck_stream_t stream) {
     if (mmas_per_pair <= 0 || !pairs) return CK_ERR_INVALID_VALUE;
     DeviceState *st = nullptr;

@@ -46,6 +46,8 @@ cudaError_t launch_quant_norm_bf16(const uint16_t *X, int64_t M, int64_t K, int6
 
 // Test hook: the input activation of n bf16 values (n % 256 == 0) as the
 // staged quantiser applies it (0 none, 1 relu, 2 silu, 3 tanh-form gelu).
+cudaError_t launch_test_row_quant_params(const float *amax, int64_t n, int q, float *div,
+                                         float *rc, cudaStream_t stream);
 cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,
                                   cudaStream_t stream);
 

@@ -31,8 +31,9 @@
 //  * The exact * 1/16 is folded into the scale: with z = 16 y (the butterfly
 //    output), amax_y = amax_z / 16 and s = fl(amax_z / 127) / 16 exactly, and
 //    fl(y / s) = fl(z / fl(amax_z / 127)), as long as nothing is subnormal:
-//    rows with amax_z >= 2^-93 take this path (values with |z| < 2^-122, whose
-//    y would be subnormal, give code 0 either way because |z / s| < 2^-22).
+//    rows with amax_z >= 2^-103 take this path (values with |z| < 2^-122,
+//    whose y would be subnormal, give code 0 either way: the divisor
+//    fl(amax_z / 127) is at least 2^-110, so |z / divisor| < 2^-12).
 //    Smaller rows follow the definition step by step (y = fl(z / 16), then the
 //    exact division).
 //  * Division: q needs round-half-even of the IEEE quotient fl(y / s). With
@@ -81,7 +82,7 @@ constexpr float kMagic4 = 3145728.0f;                // 1.5 * 2^21 (spacing 1/4 
 constexpr float kNearQuarter = 1.52587890625e-05f;   // 2^-16
 constexpr float kNearHalf = 0.4999847412109375f;     // 0.5 - 2^-16
 constexpr float kMinFastScale = 7.52316384526264e-37f;  // 2^-120
-constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-93
+constexpr float kMinFoldAmax = 9.8607613152626476e-32f;  // 2^-103
 constexpr size_t kBulkSmemBudget = 112 * 1024;       // per-CTA staging budget (all buffers)
 constexpr int kBulkBufs = 2;                         // row groups staged per CTA of the INT8 quantiser (3 timed no faster)
 
@@ -563,8 +564,49 @@ struct RowQuant {
     float qmax;   // codes lie in [-qmax, qmax]
 };
 
-// kQ = 127: INT8 codes; kQ = 7: signed INT4 codes (convrot_w4a4_linear). The
-// reciprocal fast path's bound holds a fortiori for |z / d| <= 7.
+// fl(a / kQ), the IEEE quotient, for kQ = 127 or 7 and finite a >= 2^-103,
+// by one product and one fma with a two-word reciprocal hi + lo of 1 / kQ
+// (hi = fl(1 / kQ), lo = fl(1 / kQ - hi); hi + lo is within 2^-56 (127) or
+// 2^-51 (7) of 1 / kQ relative). The fma's exact sum a hi + fl(a lo) is
+// within 2^-48 of a / kQ relative while fl(a lo) is a normal number; below
+// that (a under about 2^-91 for 127, 2^-98.8 for 7) its absolute error, at
+// most 2^-150, is below 2^-40 a / kQ. Why that suffices:
+// with a = A 2^e (A a 24-bit integer) the bits of A / kQ beyond fp32's
+// 24 repeat with period 7 (127 = 2^7 - 1) or 3 (7 = 2^3 - 1), so the part
+// of a / kQ beyond the last kept bit is r / kQ of a unit in the last place
+// for an integer r. It is therefore 0 (a / kQ exact) or at least 1 / 254
+// (resp. 1 / 14) of a unit, about 2^-32 relative, away from the rounding
+// midpoint, far more than 2^-40: the sum rounds as a / kQ does. Checked
+// against the IEEE quotient for every fp32 significand by the test hook
+// ck_test_row_quant_params.
+template <int kQ>
+__device__ __forceinline__ float div_by_q(float a) {
+    static_assert(kQ == 127 || kQ == 7, "two-word reciprocal for 127 and 7 only");
+    constexpr float hi = kQ == 127 ? 0x1.020408p-7f : 0x1.24924ap-3f;
+    constexpr float lo = kQ == 127 ? 0x1.020408p-35f : -0x1.b6db6ep-28f;
+    return __fmaf_rn(a, hi, __fmul_rn(a, lo));
+}
+
+// Reciprocal of a normal d within 2^-24 + 2^-43 relative (not necessarily
+// the correctly rounded one): the hardware approximation r0 (relative error
+// e0 <= 2^-22) and one Newton-Raphson step r0 + r0 (1 - d r0), whose
+// relative error before the last rounding is at most e0^2 + 2^-24 e0.
+__device__ __forceinline__ float rcp_newton(float d) {
+    float r0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(d));
+    const float e = __fmaf_rn(-d, r0, 1.0f);
+    return __fmaf_rn(r0, e, r0);
+}
+
+// kQ = 127: INT8 codes; kQ = 7: signed INT4 codes (convrot_w4a4_linear).
+// The fast path's reciprocal rc = rcp_newton(d) is within 2^-24 + 2^-43 of
+// 1 / d relative, so for |z| <= amax the exact z rc lies within
+// 127.00001 (2^-24 + 2^-43) + 2^-18 < 1.14e-5 of fl(z / d) (the second term: half
+// a unit in the last place below 128). A value whose computed distance to
+// the nearest integer is below 0.5 - 2^-16 (the distance itself rounded once,
+// to within 2^-26) lies more than 2^-16 - 2^-26 = 1.52e-5 from every
+// half-integer, so fl(z / d) rounds to the same integer. The bound holds a
+// fortiori for |z / d| <= 7.
 template <bool kRotate, int kQ = 127>
 __device__ __forceinline__ RowQuant row_quant(float amax) {
     RowQuant r;
@@ -572,7 +614,7 @@ __device__ __forceinline__ RowQuant row_quant(float amax) {
     r.qmax = qmax;
     if (kRotate) {
         if (amax >= kMinFoldAmax) {
-            r.div = __fdiv_rn(amax, qmax);
+            r.div = div_by_q<kQ>(amax);
             r.s = __fmul_rn(r.div, 0.0625f);
             r.fast = true;
             r.scale16 = false;
@@ -588,8 +630,22 @@ __device__ __forceinline__ RowQuant row_quant(float amax) {
         r.fast = r.s >= kMinFastScale;
         r.scale16 = false;
     }
-    r.rc = r.fast ? __frcp_rn(r.div) : 0.0f;
+    r.rc = r.fast ? rcp_newton(r.div) : 0.0f;
     return r;
+}
+
+// Test hook: the divisor and the reciprocal that row_quant gives a rotated
+// row of absmax amax[i] (grid-stride over n values).
+template <int kQ>
+__global__ void __launch_bounds__(256)
+row_quant_params_kernel(const float *__restrict__ amax, int64_t n, float *__restrict__ div,
+                        float *__restrict__ rc) {
+    const int64_t step = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += step) {
+        const RowQuant r = row_quant<true, kQ>(amax[i]);
+        div[i] = r.div;
+        rc[i] = r.rc;
+    }
 }
 
 // Exact path for one value, as the definition states it; returns the bit
@@ -840,38 +896,41 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     const uint32_t buf0 = smem_u32(stage_raw);
     const uint32_t buf_bytes = uint32_t(R) * row_bytes;
 
+    // The per-row work of a group (staging the row, clearing its absmax slot,
+    // storing its scale) falls to the row's leader, lane t = 0 of its block
+    // 0, so no one warp does all of it and reaches the CTA barrier late. A
+    // buffer's mbarrier expects one arrival per row slot.
+    const bool leader = row_local < R && blk == 0 && t == 0;
     if (tid == 0) {
-        for (int j = 0; j < kBulkBufs; ++j) mbar_init(smem_u32(&full[j]), 1);
+        for (int j = 0; j < kBulkBufs; ++j) mbar_init(smem_u32(&full[j]), uint32_t(R));
         fence_mbar_init();
     }
     for (int i = tid; i < 3 * kMaxRowsPerCta; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
     __syncthreads();
 
-    // Thread 0: stage the rows of group g into buffer b.
+    // A leader: stage its row of group g into buffer b (past the last row it
+    // only arrives).
     auto issue = [&](int64_t g, int b) {
-        const int64_t r0 = g * R;
-        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
+        const int64_t r = g * R + row_local;
         const uint32_t bar = smem_u32(&full[b]);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
-        for (int r = 0; r < n; ++r) {
-            const uint16_t *src = X + (r0 + r) * ldx;
-            const uint32_t off = uint32_t(b) * buf_bytes + uint32_t(r) * row_bytes;
+        mbar_arrive_expect_tx(bar, r < M ? row_bytes : 0u);
+        if (r >= M) return;
+        const uint32_t off = uint32_t(b) * buf_bytes + uint32_t(row_local) * row_bytes;
 #ifdef CK_CHECKED
-            if (!CK_CHECK(r0 + r < M && off + row_bytes <= dynamic_smem_bytes(), kChkBulkCopy))
-                continue;  // the wait on this group then runs out and reports the timeout
+        if (!CK_CHECK(off + row_bytes <= dynamic_smem_bytes(), kChkBulkCopy))
+            return;  // the wait on this group then runs out and reports the timeout
 #endif
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                ::"r"(buf0 + off),
-                "l"(reinterpret_cast<uint64_t>(src)), "r"(row_bytes), "r"(bar)
-                : "memory");
-        }
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+            ::"r"(buf0 + off),
+            "l"(reinterpret_cast<uint64_t>(X + r * ldx)), "r"(row_bytes), "r"(bar)
+            : "memory");
     };
 
     const int64_t g0 = blockIdx.x;
     const int64_t step = gridDim.x;
-    if (tid == 0)
+    if (leader)
         for (int j = 0; j < kBulkBufs; ++j)
             if (g0 + j * step < ngroups) issue(g0 + j * step, j);
     int slot = 0;  // i % 3
@@ -912,9 +971,9 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
             break;
         }
         // Buffer b has been read by every thread: refill it kBulkBufs groups ahead.
-        if (tid == 0 && g + kBulkBufs * step < ngroups) issue(g + kBulkBufs * step, b);
+        if (leader && g + kBulkBufs * step < ngroups) issue(g + kBulkBufs * step, b);
         const int clear = slot == 0 ? 2 : slot - 1;  // (i + 2) % 3
-        if (tid < R) s_amax[clear][tid] = 0u;
+        if (leader) s_amax[clear][row_local] = 0u;
         if (active) {
             const RowQuant rq = row_quant<kRotate, kQ>(__uint_as_float(s_amax[slot][row_local]));
             if (blk == 0 && t == 0) S[row] = rq.s;
@@ -1023,10 +1082,13 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     const uint32_t buf_bytes = uint32_t(R) * row_bytes;
     const uint32_t rbuf = buf0 + 2u * buf_bytes;  // residual rows (single buffer)
 
+    // per-row work of a group falls to the row's leader (lane t = 0 of its
+    // block 0), as in quant_rows_bulk_kernel; one arrival per row slot
+    const bool leader = row_local < R && blk == 0 && t == 0;
     if (tid == 0) {
-        mbar_init(smem_u32(&full[0]), 1);
-        mbar_init(smem_u32(&full[1]), 1);
-        mbar_init(smem_u32(&full[2]), 1);
+        mbar_init(smem_u32(&full[0]), uint32_t(R));
+        mbar_init(smem_u32(&full[1]), uint32_t(R));
+        mbar_init(smem_u32(&full[2]), uint32_t(R));
         fence_mbar_init();
     }
     for (int i = tid; i < 3 * kMaxRowsPerCta; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
@@ -1052,32 +1114,30 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
     }
     __syncthreads();
 
-    // Thread 0: stage the rows of group g (x, or the residual when res) into
-    // the buffer at dst, completing on barrier `bar`.
+    // A leader: stage its row of group g (x, or the residual when res) into
+    // the buffer at dst, completing on barrier `bar` (past the last row it
+    // only arrives).
     auto issue = [&](int64_t g, bool res, uint32_t dst, uint32_t bar) {
-        const int64_t r0 = g * R;
-        const int n = int(M - r0 < R ? M - r0 : int64_t(R));
+        const int64_t r = g * R + row_local;
         const uint16_t *src = res ? na.R : X;
         const int64_t ld = res ? na.ldr : ldx;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, uint32_t(n) * row_bytes);
-        for (int r = 0; r < n; ++r) {
+        mbar_arrive_expect_tx(bar, r < M ? row_bytes : 0u);
+        if (r >= M) return;
+        const uint32_t d = dst + uint32_t(row_local) * row_bytes;
 #ifdef CK_CHECKED
-            if (!CK_CHECK(r0 + r < M && dst + uint32_t(r + 1) * row_bytes - buf0 <= dynamic_smem_bytes(),
-                          kChkBulkCopy))
-                continue;  // the wait on this group then runs out and reports the timeout
+        if (!CK_CHECK(d + row_bytes - buf0 <= dynamic_smem_bytes(), kChkBulkCopy))
+            return;  // the wait on this group then runs out and reports the timeout
 #endif
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                ::"r"(dst + uint32_t(r) * row_bytes),
-                "l"(reinterpret_cast<uint64_t>(src + (r0 + r) * ld)), "r"(row_bytes), "r"(bar)
-                : "memory");
-        }
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+            ::"r"(d), "l"(reinterpret_cast<uint64_t>(src + r * ld)), "r"(row_bytes), "r"(bar)
+            : "memory");
     };
 
     const int64_t g0 = blockIdx.x;
     const int64_t step = gridDim.x;
-    if (tid == 0) {
+    if (leader) {
         if (g0 < ngroups) {
             issue(g0, false, buf0, smem_u32(&full[0]));
             if (kResidual) issue(g0, true, rbuf, smem_u32(&full[2]));
@@ -1165,13 +1225,13 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         }
         // every thread has its values in registers: refill x buffer b two
         // groups ahead and the residual buffer for the next group
-        if (tid == 0) {
+        if (leader) {
             if (g + 2 * step < ngroups) issue(g + 2 * step, false, buf0 + uint32_t(b) * buf_bytes,
                                               smem_u32(&full[b]));
             if (kResidual && g + step < ngroups) issue(g + step, true, rbuf, smem_u32(&full[2]));
         }
         const int clear = slot == 0 ? 2 : slot - 1;
-        if (tid < R) s_amax[clear][tid] = 0u;
+        if (leader) s_amax[clear][row_local] = 0u;
 
         float2 P[kPairs];
         if (active) {
@@ -1959,6 +2019,18 @@ cudaError_t launch_quant_norm_bf16(const uint16_t *X, int64_t M, int64_t K, int6
     const NormArgs na{R, ldr, Rout, ldo, g, eps};
     if (R) return launch_norm_bulk<true>(X, M, K, ldx, na, Q, S, err, num_sms, stream, launched);
     return launch_norm_bulk<false>(X, M, K, ldx, na, Q, S, err, num_sms, stream, launched);
+}
+
+cudaError_t launch_test_row_quant_params(const float *amax, int64_t n, int q, float *div,
+                                         float *rc, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t want = (n + 255) / 256;
+    const unsigned grid = unsigned(want < 148 * 16 ? want : 148 * 16);
+    if (q == 7)
+        row_quant_params_kernel<7><<<grid, 256, 0, stream>>>(amax, n, div, rc);
+    else
+        row_quant_params_kernel<127><<<grid, 256, 0, stream>>>(amax, n, div, rc);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_test_input_act(const uint16_t *X, int64_t n, int act, uint16_t *Y,

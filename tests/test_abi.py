@@ -132,6 +132,14 @@ def test_weight_and_gemm_validation():
     assert L.ck_test_inject_producer_stall(0, 0) == ck.CK_OK
 
 
+def test_row_quant_params_validation():
+    f = ck.lib.ck_test_row_quant_params
+    assert f(FAKE, 4, 126, FAKE, FAKE, None) == ck.CK_ERR_INVALID_VALUE
+    assert f(FAKE, -1, 127, FAKE, FAKE, None) == ck.CK_ERR_INVALID_VALUE
+    assert f(None, 4, 7, FAKE, FAKE, None) == ck.CK_ERR_INVALID_VALUE
+    assert f(None, 0, 127, None, None, None) == ck.CK_OK
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
 

@@ -127,6 +127,29 @@ def test_quantize_near_half_integers_take_exact_path(ck):
     assert np.all(np.abs(rq[:, 1:].astype(np.int32)) % 2 == 0)  # ties went to even
 
 
+@pytest.mark.parametrize("q", [127, 7])
+def test_row_divisor_is_the_ieee_quotient(ck, q):
+    """The quantiser's row divisor (one product and one fma in the kernel) is
+    the IEEE quotient fl(amax / q) for every fp32 significand of the lowest
+    binade the fast path takes (2^-103), of 1 and of the largest finite one;
+    its reciprocal (one Newton step) is within 2^-24 + 2^-43 of 1 / div. The
+    expected quotients are numpy's fp32 divisions on the host."""
+    sig = np.arange(1 << 23, dtype=np.uint32)
+    for e in (-103, 0, 127):
+        a = ((np.uint32(127 + e) << np.uint32(23)) | sig).view(np.float32)
+        div, rc = ck.test_row_quant_params(torch.from_numpy(a).cuda(), q)
+        expect = a / np.float32(q)
+        got = div.cpu().numpy()
+        bad = np.flatnonzero(got.view(np.uint32) != expect.view(np.uint32))
+        assert bad.size == 0, (e, a[bad[:5]])
+        # rc * div is exact in float64 (two 24-bit significands)
+        err = (rc.double() * div.double() - 1.0).abs().max().item()
+        assert err <= 2.0 ** -24 + 2.0 ** -43, (e, err)
+    # below 2^-103 the exact path is taken: no reciprocal
+    div, rc = ck.test_row_quant_params(torch.tensor([2.0 ** -104, 0.0], device="cuda"), q)
+    assert rc.cpu().tolist() == [0.0, 0.0]
+
+
 @pytest.mark.parametrize("N,K", [(8, 256), (264, 768), (520, 5376), (16, 33024)])
 def test_rotate_quant_weight_bit_exact(ck, N, K):
     cfg = workloads.custom(1, K, N, seed=N + K)
