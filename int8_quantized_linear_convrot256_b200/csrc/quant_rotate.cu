@@ -37,9 +37,11 @@
 //    Smaller rows follow the definition step by step (y = fl(z / 16), then the
 //    exact division).
 //  * Division: q needs round-half-even of the IEEE quotient fl(y / s). With
-//    d the divisor and r = fl(1/d), the exact product z r is within
-//    127.00001 * 2^-24 < 2^-17 of z/d, and |fl(z/d) - z/d| <= 2^-18 because
-//    |z/d| < 128; so if z r is farther than 2^-17 + 2^-18 from every
+//    d the divisor (fl(amax_z / 127), one product and one fma, see
+//    div_by_q) and r its reciprocal to within 2^-24 + 2^-43 (one Newton
+//    step, see rcp_newton), the exact product z r is within
+//    127.00001 (2^-24 + 2^-43) < 2^-17 of z/d, and |fl(z/d) - z/d| <= 2^-18
+//    because |z/d| < 128; so if z r is farther than 2^-17 + 2^-18 from every
 //    half-integer, rint(z r) = rint(fl(z/d)). One fma gives fl(z r + 1.5 * 2^23) =
 //    1.5 * 2^23 + rint(z r), whose low byte is the two's-complement code (no
 //    clamp is needed on that path); a second fma gives the distance of z r
