@@ -1877,7 +1877,8 @@ nvfp4_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx,
         advance(row0, blk0);
         butterflies<true>(P, t, sw5);
         if constexpr (kPass == 1) {
-            local_max = fmaxf(local_max, block_absmax(P));
+            // the lane's own maximum; the lanes are combined once, at the end
+            local_max = fmaxf(local_max, block_absmax<1>(P));
         } else {
             // register group i holds chunk i ^ sw5: elements col0 + 32 (i ^ sw5) .. + 7
             const int col0 = blk * kBlock + 8 * t;
