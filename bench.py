@@ -356,6 +356,23 @@ def run_ours(args, cfg, rank, world, local_rank):
         clocks.stop()
         raise RuntimeError(f"device error during the timed region: {ck.status_string(status)}")
 
+    # ---- the quantiser by itself (context for its in-step time: here no GEMM
+    # runs right before it, so the SM clock has not just been held at the
+    # power cap; a second of idle lets the board settle first, and it runs
+    # before the MMA-only probe below, which loads the board the same way)
+    time.sleep(1.0)
+    q_alone = []
+    for _ in range(SUBPATH_STEPS):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        quantize()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        q_alone.append(e0.elapsed_time(e1))
+    ms_q_alone = sorted(q_alone)[len(q_alone) // 2]
+
     probe_tops = None
     probe_clocks = None
     if args.path in ("int8", "norm") and not args.no_probe:
@@ -374,19 +391,6 @@ def run_ours(args, cfg, rank, world, local_rank):
     spread = [srt[len(srt) // 2], srt[0], srt[-1]]  # median, min, max of the steps
     ms_step, ms_q, ms_g, *spread = max_over_ranks([ms_step, ms_q, ms_g, *spread], dev)
 
-    # ---- the quantiser by itself (context for its in-step time: here no GEMM
-    # runs before it, so the SM clock has not been held at the power cap)
-    q_alone = []
-    for _ in range(SUBPATH_STEPS):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        quantize()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        q_alone.append(e0.elapsed_time(e1))
-    ms_q_alone = sorted(q_alone)[len(q_alone) // 2]
 
     # ---- end to end through the public composite call, host buffers
     if args.no_e2e or args.path in ("w4a4", "nvfp4", "norm"):
@@ -672,8 +676,9 @@ def report(args, cfg, rank, world, P, X, Wcpu, bias, ms_step, ms_q, ms_g, ms_e2e
                           **({"alone": {"ms_per_launch": ms_q_alone,
                                         "frac": q_bytes / (ms_q_alone / 1e3) / 1e9 / P["hbm_gbs"],
                                         "note": f"median of {SUBPATH_STEPS} launches timed by "
-                                                "themselves after the timed region, L2 flushed "
-                                                "before each; not the metric"}}
+                                                "themselves after the timed region and a second "
+                                                "of idle, L2 flushed before each; not the "
+                                                "metric"}}
                              if ms_q_alone else {})},
             "cpu_baseline": cpu,
             "e2e": None if (args.no_e2e or args.path in ("w4a4", "nvfp4", "norm")) else {"value": e2e_value, "unit": UNIT, "ms_per_step": ms_e2e,
