@@ -1002,9 +1002,10 @@ quant_rows_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
 // the smaller operand is below 2^-16 of the larger, far under half a bf16
 // spacing, so both give the larger operand's neighbourhood the same way).
 // The sum of squares runs in double (each h^2 exact): a lane's 64 values in
-// order, the quad's four lanes by shuffles, then the row's quads in block
-// order through shared memory, so one row gives one result. inv = 1 /
-// sqrt(ss / K + eps) in double, inv32 its fp32 rounding. Fast path per value:
+// order, the quad's four lanes by shuffles, then the row's block partials
+// through shared memory in one fixed order (four interleaved chains, combined
+// by shuffles), so one row gives one result. inv = 1 / sqrt(ss fl(1 / K) +
+// eps) in double, inv32 its fp32 rounding. Fast path per value:
 // hg = h g in fp32 (exact while the product is a normal fp32 number: 8-bit
 // significands), then a = fl(hg fl(inv32 (1 - 2^-21))) and
 // b = fl(hg fl(inv32 (1 + 2^-21))): four roundings of 2^-24 each and inv's
@@ -1146,6 +1147,7 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         }
         if (g0 + step < ngroups) issue(g0 + step, false, buf0 + buf_bytes, smem_u32(&full[1]));
     }
+    const double inv_k = 1.0 / double(K);  // mean = sum * fl(1 / K): within the bound
     int slot = 0;
     for (int i = 0; g0 + i * step < ngroups; ++i) {
         const int64_t g = g0 + i * step;
@@ -1235,21 +1237,21 @@ quant_norm_bulk_kernel(const uint16_t *__restrict__ X, int64_t M, int K, int64_t
         const int clear = slot == 0 ? 2 : slot - 1;
         if (leader) s_amax[clear][row_local] = 0u;
 
+        // the row's sum of squares from its blocks' partial sums: lane t of
+        // each quad adds the partials t, t + 4, t + 8, ... in that order, and
+        // the quad combines its four chains as (c0 + c1) + (c2 + c3). One
+        // fixed order, so every quad of the row gets the same sum.
+        double ssr = 0.0;
+        if (active) {
+            const double *part = &s_ss[row_local * nb];
+            for (int q = t; q < nb; q += 4) ssr = __dadd_rn(ssr, part[q]);
+        }
+        ssr = __dadd_rn(ssr, __shfl_xor_sync(0xFFFFFFFFu, ssr, 1));
+        ssr = __dadd_rn(ssr, __shfl_xor_sync(0xFFFFFFFFu, ssr, 2));
+
         float2 P[kPairs];
         if (active) {
-            // the row's sum in block order, four chains
-            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-            const double *part = &s_ss[row_local * nb];
-            int q = 0;
-            for (; q + 4 <= nb; q += 4) {
-                s0 = __dadd_rn(s0, part[q]);
-                s1 = __dadd_rn(s1, part[q + 1]);
-                s2 = __dadd_rn(s2, part[q + 2]);
-                s3 = __dadd_rn(s3, part[q + 3]);
-            }
-            for (; q < nb; ++q) s0 = __dadd_rn(s0, part[q]);
-            const double ssr = __dadd_rn(__dadd_rn(s0, s1), __dadd_rn(s2, s3));
-            const double inv = rsqrt(ssr / double(K) + double(na.eps));
+            const double inv = rsqrt(__dmul_rn(ssr, inv_k) + double(na.eps));
             const float inv32 = __double2float_rn(inv);
             const float ilo = __fmul_rn(inv32, kNormLo), ihi = __fmul_rn(inv32, kNormHi);
             const float2 lo2 = make_float2(ilo, ilo), hi2 = make_float2(ihi, ihi);
