@@ -391,8 +391,9 @@ gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             const uint32_t leader_full0 = mapa_shared(smem_u32(&ctl->full[0]), 0);
-            // Qw is re-read by every group of M-tiles: keep it in L2 while
-            // A (reused within a group only) and Y (written once) pass through
+            // the group's Qw columns serve every M-tile of the sweep: keep them
+            // in L2 while A (used by one group's N-tiles) and Y (written
+            // once) pass through
             const uint64_t keep = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_parity = 0;
