@@ -155,7 +155,10 @@ def _assert_gemm_close(Y_bits, Yr_bits, mag, K):
 
 
 @pytest.mark.parametrize("M,K,N", [(128, 256, 128), (1, 256, 8), (129, 768, 264), (300, 5376, 520),
-                                   (257, 1024, 136)])
+                                   (257, 1024, 136),
+                                   # the 2-SM kernel's raster walks groups of 32 N-tiles: a
+                                   # full group and a second, ragged one of 2, ragged M
+                                   (300, 256, 33 * 256 + 40)])
 def test_nvfp4_gemm_matches_oracle(ck, M, K, N):
     cfg = workloads.custom(M, K, N, seed=M + 3 * N + K)
     X, W, bias = workloads.make_inputs(cfg)

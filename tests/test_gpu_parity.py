@@ -164,7 +164,12 @@ def test_rotate_quant_weight_bit_exact(ck, N, K):
 
 
 GEMM_SHAPES = [(1, 8, 256), (3, 17 * 8, 256), (127, 256, 512), (128, 256, 512), (129, 264, 768),
-               (300, 520, 512), (257, 1032, 1024), (640, 512, 2048), (1, 256, 5376)]
+               (300, 520, 512), (257, 1032, 1024), (640, 512, 2048), (1, 256, 5376),
+               # the 2-SM kernel's raster walks groups of 21 N-tiles: a full group,
+               # a second group of 2 (the last one ragged), and ragged M
+               (300, 21 * 256 + 264, 256),
+               # three groups of 21, 21 and 1 N-tiles over three M-tiles
+               (520, 43 * 256 - 8, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -198,7 +203,9 @@ def _oracle_linear(X, W, bias):
 
 
 LINEAR_SHAPES = [(128, 512, 512), (1, 256, 8), (129, 768, 264), (255, 512, 520), (257, 1024, 256),
-                 (300, 5376, 512), (64, 28672, 264)]
+                 (300, 5376, 512), (64, 28672, 264),
+                 # the epilogue across the 2-SM raster's N-tile groups (21, then 2)
+                 (300, 256, 21 * 256 + 264)]
 
 
 @pytest.mark.parametrize("M,K,N", LINEAR_SHAPES)
